@@ -1,0 +1,460 @@
+"""Benchmark: cached block attention denoising steps per second on B200.
+
+One bench step = one block of block-diffusion decoding on the chosen workload
+(default: the LLaDA-8B-shaped layer, b1, 32 heads, d128, prefix 4096, block 32,
+32 denoising steps):
+    fbk_prefix_partial        (prefix state from the block's first queries)
+    32 x fbk_block_attn_merge (one per denoising step, fresh block Q/K/V each)
+    fbk_commit_block_rope_append (RoPE + append the finished block)
+The value is denoising steps per second over all ranks. Inputs are resident in
+HBM; the block is replayed as CUDA graphs; L2 is flushed (a 2x-L2 memset)
+before every timed block and the flush is outside the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+For N > 1 (torchrun), every rank runs an independent replica (no collective;
+weak scaling) and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "cached block-attn denoising steps/s + KV GB/s & TFLOP/s vs roofline (1×B200)"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llada8b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    import torch
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle timing
+
+def oracle_block(case, steps):
+    """The oracle's reuse schedule for one block (prefix state once, `steps`
+    denoising steps, commit): fp64 numpy on the host cores."""
+    from oracle import fbk_oracle as orc
+    kp, vp = case["kp"], case["vp"]
+    lens, hkv, base = case["lens"], case["hkv"], case["base"]
+    q0 = case["steps"][0][0]
+    pfx = orc.prefix_partial(q0, kp, vp, lens, hkv, 1.0, base)
+    for s in range(steps):
+        q, k, v = case["steps"][s % len(case["steps"])]
+        orc.step_output(pfx, q, k, v, lens, hkv, 1.0, base)
+    q, k, v = case["steps"][(steps - 1) % len(case["steps"])]
+    orc.commit_contiguous(case["kc"], case["vc"], k, case["vbits"], lens, base)
+
+
+def oracle_case(wl, n_step_inputs=2):
+    from cached_block_attention_b200 import synth
+    from oracle import fbk_oracle as orc
+    lens = wl.prefix_lens()
+    ks, vs = synth.gen_prefix(wl, lens)
+    kc, vc = synth.contiguous_cache(ks, vs, wl.n_kv_heads, wl.head_dim, int(lens.max()) + wl.block_len)
+    steps = []
+    vbits = None
+    for s in range(n_step_inputs):
+        q, k, v = synth.gen_step(wl, s)
+        steps.append((orc.bits_to_f64(q), orc.bits_to_f64(k), orc.bits_to_f64(v)))
+        vbits = v
+    return {"kp": [orc.bits_to_f64(k) for k in ks], "vp": [orc.bits_to_f64(v) for v in vs],
+            "lens": lens, "hkv": wl.n_kv_heads, "base": wl.rope_base, "steps": steps,
+            "kc": kc, "vc": vc, "vbits": vbits}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(int(i.get("num_threads", 1)) for i in threadpool_info()) or 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    """Time the oracle as it stands on a bounded sample: whole blocks of the
+    workload's reuse schedule, as many as fit in about `budget_s` seconds."""
+    case = oracle_case(wl)
+    t0 = time.perf_counter()
+    oracle_block(case, wl.steps)
+    one = time.perf_counter() - t0
+    n = max(1, min(20, int(budget_s / max(one, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(n):
+        oracle_block(case, wl.steps)
+    dt = time.perf_counter() - t0
+    return {"value": n * wl.steps / dt, "unit": "denoising steps/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} whole blocks of {wl.name} ({wl.steps} steps each, prefix state once, "
+                      f"commit), fp64 numpy"}
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    case = oracle_case(wl)
+    # each bench step is a bounded sample: one block with at most 8 denoising steps
+    s = min(wl.steps, 8)
+    for _ in range(args.warmup):
+        oracle_block(case, s)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_block(case, s)
+    dt = time.perf_counter() - t0
+    v = args.steps * s / dt
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "denoising steps/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "description": wl.description,
+                       "bench_step": f"one block sample: prefix state + {s} denoising steps + commit"},
+            "cpu_baseline": {"value": v, "unit": "denoising steps/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": f"one block with {s} of {wl.steps} steps per bench step"},
+            "e2e": {"value": v, "unit": "denoising steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, wl, rank, world, local):
+    import torch
+    from cached_block_attention_b200 import fbk, synth
+
+    dev = torch.device("cuda", local)
+    S = wl.steps
+    lens_np = wl.prefix_lens()
+    ks, vs = synth.gen_prefix(wl, lens_np)
+    extra = wl.block_len
+    if wl.page_size:
+        kp, vp, table = synth.paged_cache(ks, vs, wl.n_kv_heads, wl.head_dim, wl.page_size, extra, wl.page_seed)
+        k_cache = torch.from_numpy(kp.view(np.int16)).view(torch.bfloat16).to(dev)
+        v_cache = torch.from_numpy(vp.view(np.int16)).view(torch.bfloat16).to(dev)
+        page_table = torch.from_numpy(table).to(dev)
+    else:
+        kc, vc = synth.contiguous_cache(ks, vs, wl.n_kv_heads, wl.head_dim, int(lens_np.max()) + extra)
+        k_cache = torch.from_numpy(kc.view(np.int16)).view(torch.bfloat16).to(dev)
+        v_cache = torch.from_numpy(vc.view(np.int16)).view(torch.bfloat16).to(dev)
+        page_table = None
+    del ks, vs
+    lens0 = torch.from_numpy(lens_np.astype(np.int32)).to(dev)
+    lens = lens0.clone()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    cache = fbk.KVCache(k_cache, v_cache, lens, page_table, err)
+    shape = fbk.Shape(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.block_len, 1.0, wl.rope_base,
+                      fbk.BF16)
+    host_steps = [synth.gen_step(wl, s) for s in range(S)]
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_q = torch.stack([pin(q) for q, _, _ in host_steps])
+    h_k = torch.stack([pin(k) for _, k, _ in host_steps])
+    h_v = torch.stack([pin(v) for _, _, v in host_steps])
+    h_q, h_k, h_v = h_q.pin_memory(), h_k.pin_memory(), h_v.pin_memory()
+    d_q, d_k, d_v = h_q.to(dev), h_k.to(dev), h_v.to(dev)
+    pfx = fbk.Partial.empty(shape, dev)
+    ws = torch.empty(fbk.prefix_workspace_bytes(shape, cache, 0), dtype=torch.uint8, device=dev)
+    outs = torch.empty(S, wl.batch, wl.block_len, wl.n_q_heads, wl.head_dim, dtype=torch.bfloat16, device=dev)
+    h_out = torch.empty(outs.shape, dtype=torch.bfloat16).pin_memory()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    def seg_prefix():
+        lens.copy_(lens0)  # every bench step decodes the same block position
+        fbk.prefix_partial(shape, d_q[0], cache, pfx, ws)
+
+    def seg_steps():
+        for s in range(S):
+            fbk.block_attn_merge(shape, d_q[s], d_k[s], d_v[s], lens, pfx, outs[s])
+
+    def seg_commit():
+        fbk.commit_block_rope_append(shape, d_k[S - 1], d_v[S - 1], cache)
+
+    def seg_recompute():
+        lens.copy_(lens0)
+        for s in range(S):
+            fbk.prefix_partial(shape, d_q[s], cache, pfx, ws)
+            fbk.block_attn_merge(shape, d_q[s], d_k[s], d_v[s], lens, pfx, outs[s])
+        fbk.commit_block_rope_append(shape, d_k[S - 1], d_v[S - 1], cache)
+
+    # eager warm-up (also sets kernel attributes before capture)
+    for _ in range(2):
+        seg_prefix(); seg_steps(); seg_commit()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+
+    st = torch.cuda.Stream(dev)
+    st.wait_stream(torch.cuda.current_stream(dev))
+    graphs = []
+    with torch.cuda.stream(st):
+        for fn in (seg_prefix, seg_steps, seg_commit, seg_recompute):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st, capture_error_mode="thread_local"):
+                fn()
+            graphs.append(g)
+    torch.cuda.synchronize()
+    g_pfx, g_steps, g_commit, g_recomp = graphs
+
+    def timed_blocks(n, record):
+        """n blocks, each after an L2 flush; events bracket the three segments."""
+        evs = []
+        with torch.cuda.stream(st):
+            for _ in range(n):
+                flush.zero_()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                e[0].record(st)
+                g_pfx.replay()
+                e[1].record(st)
+                g_steps.replay()
+                e[2].record(st)
+                g_commit.replay()
+                e[3].record(st)
+                evs.append(e)
+        return evs
+
+    timed_blocks(args.warmup, False)
+    barrier(world)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    evs = timed_blocks(args.steps, True)
+    barrier(world)
+    clock_info = clocks.stop()
+    t_blocks = [e[0].elapsed_time(e[3]) for e in evs]
+    t_pfx = [e[0].elapsed_time(e[1]) for e in evs]
+    t_steps = [e[1].elapsed_time(e[2]) for e in evs]
+    t_commit = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = max_over_ranks(sum(t_blocks), world)
+    assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+
+    # recompute-every-step schedule, same flush discipline
+    rec = []
+    with torch.cuda.stream(st):
+        for _ in range(max(3, args.steps // 2)):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            g_recomp.replay()
+            b.record(st)
+            rec.append((a, b))
+    torch.cuda.synchronize()
+    rec_ms = statistics.mean(a.elapsed_time(b) for a, b in rec)
+
+    # end to end through the public API: pinned host inputs in, outputs back, eager calls
+    def e2e_block():
+        d_q.copy_(h_q, non_blocking=True)
+        d_k.copy_(h_k, non_blocking=True)
+        d_v.copy_(h_v, non_blocking=True)
+        lens.copy_(lens0)
+        fbk.prefix_partial(shape, d_q[0], cache, pfx, ws)
+        for s in range(S):
+            fbk.block_attn_merge(shape, d_q[s], d_k[s], d_v[s], lens, pfx, outs[s])
+        fbk.commit_block_rope_append(shape, d_k[S - 1], d_v[S - 1], cache)
+        h_out.copy_(outs, non_blocking=True)
+
+    with torch.cuda.stream(st):
+        for _ in range(2):
+            e2e_block()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, args.steps // 2)
+        a.record(st)
+        for _ in range(n_e2e):
+            flush.zero_()
+            e2e_block()
+        b.record(st)
+        torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world)
+    h2d = (h_q.numel() + h_k.numel() + h_v.numel()) * 2
+    d2h = h_out.numel() * 2
+
+    # roofline of the dominant kernel (by time share inside the timed region)
+    hbm_gbs, tflops, peak_kind = load_peaks()
+    L_sum = int(lens_np.sum())
+    kv_bytes = 4 * wl.n_kv_heads * wl.head_dim * L_sum
+    pfx_flops = 4 * wl.n_q_heads * wl.block_len * wl.head_dim * L_sum
+    rows = wl.batch * wl.n_q_heads * wl.block_len
+    step_bytes = (rows * wl.head_dim * 2                       # Q
+                  + 2 * wl.batch * wl.block_len * wl.n_kv_heads * wl.head_dim * 2  # K, V
+                  + rows * (wl.head_dim + 2) * 4               # prefix state read
+                  + rows * wl.head_dim * 2)                    # O write
+    mean = lambda x: sum(x) / len(x)
+    pfx_ms, steps_ms, commit_ms = mean(t_pfx), mean(t_steps), mean(t_commit)
+    step_launch_ms = steps_ms / S
+    units = {
+        "fbk_block_attn_merge": (steps_ms, step_bytes, step_launch_ms, S),
+        "fbk_prefix_partial": (pfx_ms, kv_bytes, pfx_ms, 1),
+    }
+    dom = max(units, key=lambda k: units[k][0])
+    _, dom_bytes, dom_launch_ms, _ = units[dom]
+    achieved = dom_bytes / (dom_launch_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                "frac": achieved / hbm_gbs, "traffic": None, "kernel": dom,
+                "peak_kind": f"{peak_kind} hbm_gbs",
+                "algorithmic_bytes_per_launch": dom_bytes, "launch_us": dom_launch_ms * 1e3}
+    pfx_gbs = kv_bytes / (pfx_ms * 1e-3) / 1e9
+    pfx_tfs = pfx_flops / (pfx_ms * 1e-3) / 1e12
+    n_per_block = 2 + S + 1
+
+    value = world * args.steps * S / (total_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "denoising steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "description": wl.description,
+                   "bench_step": f"one block: prefix state once + {S} denoising steps + commit",
+                   "l2": "flushed (2x L2 memset) before every timed block, outside the events",
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "schedule": "reuse (prefix state computed once per block)"},
+        "roofline": roofline,
+        "prefix_partial": {"us": pfx_ms * 1e3, "kv_gbs": pfx_gbs, "tflops": pfx_tfs,
+                           "hbm_frac": pfx_gbs / hbm_gbs, "tensor_frac": pfx_tfs * 1e3 / tflops,
+                           "kv_bytes": kv_bytes, "flops": pfx_flops},
+        "step_us": step_launch_ms * 1e3, "commit_us": commit_ms * 1e3,
+        "recompute_schedule": {"value": world * S / (rec_ms * 1e-3), "unit": "denoising steps/s",
+                               "ms_per_block": rec_ms},
+        "e2e": {"value": world * S / (e2e_ms * 1e-3), "unit": "denoising steps/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "eager API calls per block; block inputs H2D from pinned host, outputs D2H"},
+        "gpu_launches": n_per_block * args.steps,
+        "clocks": clock_info,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graphs, g_pfx, g_steps, g_commit, g_recomp
+
+
+def main():
+    args = parse()
+    from cached_block_attention_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, wl, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, wl, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

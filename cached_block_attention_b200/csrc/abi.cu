@@ -1,0 +1,209 @@
+// extern "C" entry points of libfbk.so (declared in include/fbk.h): host-side
+// argument checks, the kernel-side Geometry, workspace carving and dispatch.
+// No entry point allocates, synchronises or keeps state.
+#include <math.h>
+#include <string.h>
+
+#include "launch.h"
+
+namespace fbk {
+namespace {
+
+bool is_pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
+
+fbk_status check_shape(const fbk_shape *s) {
+  if (!s) return FBK_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_heads < 1 || s->block_len < 1 || s->head_dim < 1)
+    return FBK_ERR_INVALID_ARG;
+  if (s->mode != FBK_BF16 && s->mode != FBK_FP32_CHECK) return FBK_ERR_INVALID_ARG;
+  if (!isfinite(s->softmax_scale) || !isfinite(s->rope_base) || !(s->rope_base > 0.0))
+    return FBK_ERR_INVALID_ARG;
+  if (s->head_dim != 64 && s->head_dim != 128) return FBK_ERR_UNSUPPORTED;
+  if (s->n_q_heads % s->n_kv_heads != 0) return FBK_ERR_UNSUPPORTED;
+  if (s->block_len > 64) return FBK_ERR_UNSUPPORTED;
+  if ((long long)(s->n_q_heads / s->n_kv_heads) * s->block_len > 256) return FBK_ERR_UNSUPPORTED;
+  return FBK_OK;
+}
+
+fbk_status check_cache(const fbk_shape *s, const fbk_kv_cache *c) {
+  if (!c || !c->k || !c->v || !c->prefix_lens) return FBK_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(c->k) | reinterpret_cast<uintptr_t>(c->v)) & 15u)
+    return FBK_ERR_UNSUPPORTED;  // tensor-map and 16-byte vector access need 16-byte alignment
+  long long rows;
+  if (c->paged) {
+    if (!c->page_table || c->max_pages_per_seq < 1 || c->num_pages < 1) return FBK_ERR_INVALID_ARG;
+    if (!is_pow2(c->page_size) || c->page_size < 16) return FBK_ERR_UNSUPPORTED;
+    rows = c->num_pages * s->n_kv_heads * (long long)c->page_size;
+    if ((long long)c->max_pages_per_seq * c->page_size > 0x7fffffffll) return FBK_ERR_CAPACITY;
+  } else {
+    if (c->capacity_tokens < 1) return FBK_ERR_INVALID_ARG;
+    if (c->capacity_tokens > 0x7fffffffll) return FBK_ERR_CAPACITY;
+    rows = (long long)s->batch * s->n_kv_heads * c->capacity_tokens;
+  }
+  if (rows > 0x7fffffffll) return FBK_ERR_CAPACITY;  // TMA row coordinates are int32
+  return FBK_OK;
+}
+
+Geometry make_geometry(const fbk_shape *s, const fbk_kv_cache *c) {
+  Geometry g;
+  memset(&g, 0, sizeof(g));
+  g.batch = s->batch;
+  g.hq = s->n_q_heads;
+  g.hkv = s->n_kv_heads;
+  g.group = s->n_q_heads / s->n_kv_heads;
+  g.d = s->head_dim;
+  g.blk = s->block_len;
+  g.rows = g.group * g.blk;
+  g.tau = s->softmax_scale;
+  for (int i = 0; i < g.d / 2; ++i)
+    g.inv_freq_over_pi[i] = pow(s->rope_base, -2.0 * i / g.d) / M_PI;
+  if (c) {
+    g.kc = static_cast<const __nv_bfloat16 *>(c->k);
+    g.vc = static_cast<const __nv_bfloat16 *>(c->v);
+    g.paged = c->paged ? 1 : 0;
+    g.page_size = c->paged ? c->page_size : 0;
+    g.page_shift = 0;
+    while (c->paged && (1 << g.page_shift) < c->page_size) ++g.page_shift;
+    g.max_pages = c->paged ? c->max_pages_per_seq : 0;
+    g.cap = c->paged ? 0 : c->capacity_tokens;
+    g.num_pages = c->paged ? c->num_pages : 0;
+    g.page_table = c->page_table;
+    g.lens = c->prefix_lens;
+    g.err = c->error_flags;
+  }
+  return g;
+}
+
+int default_shares() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return sms;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace: per-share states for P + b*Hkv - 1 slots (share + unit).
+void ws_sizes(const fbk_shape *s, int shares, size_t *o_bytes, size_t *ml_bytes, long long *slots) {
+  const long long rows = (long long)(s->n_q_heads / s->n_kv_heads) * s->block_len;
+  *slots = (long long)shares + (long long)s->batch * s->n_kv_heads;
+  *o_bytes = align256((size_t)(*slots * rows * s->head_dim) * sizeof(float));
+  *ml_bytes = align256((size_t)(*slots * rows) * sizeof(float));
+}
+
+fbk_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FBK_OK : FBK_ERR_CUDA; }
+
+}  // namespace
+}  // namespace fbk
+
+using namespace fbk;
+
+extern "C" {
+
+int32_t fbk_default_num_splits(void) { return default_shares(); }
+
+size_t fbk_prefix_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache, int32_t num_splits) {
+  (void)cache;
+  if (check_shape(shape) != FBK_OK || num_splits < 0) return 0;
+  const int shares = num_splits ? num_splits : default_shares();
+  if (shares < 1) return 0;
+  size_t ob, mlb;
+  long long slots;
+  ws_sizes(shape, shares, &ob, &mlb, &slots);
+  return ob + 2 * mlb;
+}
+
+fbk_status fbk_prefix_partial(const fbk_shape *shape, const void *q_blk, const fbk_kv_cache *cache,
+                              const fbk_partial *out, void *ws, size_t ws_bytes, int32_t num_splits,
+                              void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if ((st = check_cache(shape, cache)) != FBK_OK) return st;
+  if (!q_blk || !out || !out->o_unnorm || !out->m || !out->l || num_splits < 0) return FBK_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(q_blk) & 15u) return FBK_ERR_UNSUPPORTED;
+  const int shares = num_splits ? num_splits : default_shares();
+  if (shares < 1) return FBK_ERR_CUDA;
+  size_t ob, mlb;
+  long long slots;
+  ws_sizes(shape, shares, &ob, &mlb, &slots);
+  if (!ws || ws_bytes < ob + 2 * mlb) return FBK_ERR_WORKSPACE;
+  Workspace w;
+  w.o = static_cast<float *>(ws);
+  w.m = reinterpret_cast<float *>(static_cast<char *>(ws) + ob);
+  w.l = reinterpret_cast<float *>(static_cast<char *>(ws) + ob + mlb);
+  w.slots = slots;
+  const Geometry g = make_geometry(shape, cache);
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_blk);
+  cudaError_t e = shape->mode == FBK_BF16 ? launch_prefix_tc(g, q, w, shares, s)
+                                          : launch_prefix_fp32(g, q, w, shares, s);
+  if (e != cudaSuccess) return FBK_ERR_CUDA;
+  return from_cuda(launch_split_reduce(g, w, shares, *out, s));
+}
+
+fbk_status fbk_block_attn_merge(const fbk_shape *shape, const void *q_blk, const void *k_blk,
+                                const void *v_blk, const int32_t *prefix_lens,
+                                const fbk_partial *prefix, void *out, float *lse, void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if (!q_blk || !k_blk || !v_blk || !prefix_lens || !prefix || !prefix->o_unnorm || !prefix->m ||
+      !prefix->l || !out)
+    return FBK_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q_blk) | reinterpret_cast<uintptr_t>(k_blk) |
+       reinterpret_cast<uintptr_t>(v_blk) | reinterpret_cast<uintptr_t>(out) |
+       reinterpret_cast<uintptr_t>(prefix->o_unnorm)) & 15u)
+    return FBK_ERR_UNSUPPORTED;
+  Geometry g = make_geometry(shape, nullptr);
+  g.lens = prefix_lens;
+  return from_cuda(launch_block_merge(g, static_cast<const __nv_bfloat16 *>(q_blk),
+                                      static_cast<const __nv_bfloat16 *>(k_blk),
+                                      static_cast<const __nv_bfloat16 *>(v_blk), *prefix, out, lse,
+                                      shape->mode == FBK_FP32_CHECK,
+                                      static_cast<cudaStream_t>(cuda_stream)));
+}
+
+fbk_status fbk_commit_block_rope_append(const fbk_shape *shape, const void *k_blk, const void *v_blk,
+                                        fbk_kv_cache *cache, void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if ((st = check_cache(shape, cache)) != FBK_OK) return st;
+  if (!k_blk || !v_blk) return FBK_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k_blk) | reinterpret_cast<uintptr_t>(v_blk)) & 15u)
+    return FBK_ERR_UNSUPPORTED;
+  const Geometry g = make_geometry(shape, cache);
+  return from_cuda(launch_commit(g, static_cast<const __nv_bfloat16 *>(k_blk),
+                                 static_cast<const __nv_bfloat16 *>(v_blk),
+                                 static_cast<__nv_bfloat16 *>(cache->k), static_cast<__nv_bfloat16 *>(cache->v),
+                                 cache->prefix_lens, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+fbk_status fbk_full_ref_attn(const fbk_shape *shape, const void *q_blk, const void *k_blk,
+                             const void *v_blk, const fbk_kv_cache *cache, void *out, float *lse,
+                             void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if ((st = check_cache(shape, cache)) != FBK_OK) return st;
+  if (!q_blk || !k_blk || !v_blk || !out) return FBK_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k_blk) | reinterpret_cast<uintptr_t>(v_blk) |
+       reinterpret_cast<uintptr_t>(q_blk)) & 3u)
+    return FBK_ERR_UNSUPPORTED;
+  const Geometry g = make_geometry(shape, cache);
+  return from_cuda(launch_full_ref(g, static_cast<const __nv_bfloat16 *>(q_blk),
+                                   static_cast<const __nv_bfloat16 *>(k_blk),
+                                   static_cast<const __nv_bfloat16 *>(v_blk), out, lse,
+                                   shape->mode == FBK_FP32_CHECK, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+const char *fbk_status_string(fbk_status status) {
+  switch (status) {
+    case FBK_OK: return "ok";
+    case FBK_ERR_INVALID_ARG: return "invalid argument";
+    case FBK_ERR_UNSUPPORTED: return "unsupported shape or alignment";
+    case FBK_ERR_CAPACITY: return "cache geometry exceeds the supported size";
+    case FBK_ERR_WORKSPACE: return "workspace missing or too small";
+    case FBK_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,209 @@
+// Shared device helpers of the cached block attention kernels (sm_100a).
+//
+// Contents: the kernel-side view of a call (Geometry), prefix-length checks,
+// the work list that splits the prefix keys into equal shares, RoPE angle
+// helpers, bf16 conversions and the device error flag.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+#include <stdint.h>
+
+#include "../../include/fbk.h"
+
+namespace fbk {
+
+// Keys per work-list tile: the prefix of every (sequence, kv-head) pair is cut
+// into ceil(L_b / KV_TILE) tiles, and all tiles of all pairs form one list.
+constexpr int KV_TILE = 64;
+
+// Everything a kernel needs to know about one call. Passed by value.
+struct Geometry {
+  int batch, hq, hkv, group, d, blk, rows;  // rows = group * blk (query rows per kv-head)
+  float tau;                                // softmax scale
+  double inv_freq_over_pi[64];              // base^(-2i/d) / pi, i < d/2
+  // cache
+  const __nv_bfloat16 *kc, *vc;
+  int paged, page_size, page_shift, max_pages;
+  long long cap, num_pages;
+  const int *page_table;
+  const int *lens;
+  int *err;
+};
+
+__device__ __forceinline__ void raise_flag(const Geometry &g, unsigned bits) {
+  if (g.err) atomicOr(g.err, (int)bits);
+}
+
+// Number of tokens the cache can hold for one sequence.
+__host__ __device__ __forceinline__ long long seq_capacity(const Geometry &g) {
+  return g.paged ? (long long)g.max_pages * g.page_size : g.cap;
+}
+
+// Committed prefix length of sequence b as the prefix kernels see it: a value
+// outside [0, capacity] is flagged and the sequence is treated as empty, so no
+// kernel reads outside the cache.
+__device__ __forceinline__ int prefix_len(const Geometry &g, int b) {
+  int L = g.lens[b];
+  if (L < 0 || (long long)L > seq_capacity(g)) {
+    raise_flag(g, FBK_DEVERR_PREFIX_LEN);
+    return 0;
+  }
+  return L;
+}
+
+__device__ __forceinline__ int tiles_of(int L) { return (L + KV_TILE - 1) / KV_TILE; }
+
+// Total tiles over all (sequence, kv-head) pairs.
+__device__ __forceinline__ long long total_tiles(const Geometry &g) {
+  long long t = 0;
+  for (int b = 0; b < g.batch; ++b) t += (long long)g.hkv * tiles_of(prefix_len(g, b));
+  return t;
+}
+
+// Share c of P covers list positions [c*T/P, (c+1)*T/P).
+__host__ __device__ __forceinline__ long long share_begin(long long c, long long T, long long P) {
+  return (c * T) / P;
+}
+
+// The share that holds list position x (largest c with share_begin(c) <= x).
+__device__ __forceinline__ long long share_of(long long x, long long T, long long P) {
+  return ((x + 1) * P - 1) / T;
+}
+
+// A piece: the intersection of one share with one (sequence, kv-head) unit.
+// Unit u = b * Hkv + kvh. Its state goes to workspace slot (share + u), which
+// is unique because every new piece of the list advances the share, the unit,
+// or both.
+struct Piece {
+  int b, kvh, u, L;
+  int tile_begin, tile_end;  // tile indices inside the unit
+};
+
+// Walks the pieces of one share in list order. Every warp role of a kernel
+// runs its own copy; the walk is deterministic, so all copies agree.
+struct PieceWalker {
+  long long pos, end;  // list positions still to cover
+  long long acc;       // list position where sequence b starts
+  int b, L, tb;        // current sequence, its length and tiles per kv-head
+
+  __device__ __forceinline__ void init(const Geometry &g, long long share, long long T,
+                                       long long P) {
+    pos = share_begin(share, T, P);
+    end = share_begin(share + 1, T, P);
+    acc = 0;
+    b = 0;
+    L = g.batch > 0 ? prefix_len(g, 0) : 0;
+    tb = tiles_of(L);
+  }
+
+  __device__ __forceinline__ bool next(const Geometry &g, Piece &p) {
+    if (pos >= end) return false;
+    while (pos >= acc + (long long)g.hkv * tb) {
+      acc += (long long)g.hkv * tb;
+      if (++b >= g.batch) {  // only if the lengths changed under a running kernel
+        pos = end;
+        return false;
+      }
+      L = prefix_len(g, b);
+      tb = tiles_of(L);
+    }
+    long long off = pos - acc;
+    int kvh = (int)(off / tb);
+    int j0 = (int)(off - (long long)kvh * tb);
+    long long unit_end = acc + (long long)(kvh + 1) * tb;
+    long long stop = unit_end < end ? unit_end : end;
+    p.b = b;
+    p.kvh = kvh;
+    p.u = b * g.hkv + kvh;
+    p.L = L;
+    p.tile_begin = j0;
+    p.tile_end = j0 + (int)(stop - pos);
+    pos = stop;
+    return true;
+  }
+};
+
+// Row (of the 2-D [rows, d] view of the cache) that holds token `pos` of
+// sequence b, kv-head kvh; -1 (and a flag) for a bad page id.
+__device__ __forceinline__ long long cache_row(const Geometry &g, int b, int kvh, long long pos) {
+  if (!g.paged) return ((long long)b * g.hkv + kvh) * g.cap + pos;
+  int page = g.page_table[(long long)b * g.max_pages + (pos >> g.page_shift)];
+  if (page < 0 || (long long)page >= g.num_pages) {
+    raise_flag(g, FBK_DEVERR_PAGE_ID);
+    return -1;
+  }
+  return ((long long)page * g.hkv + kvh) * g.page_size + (pos & (g.page_size - 1));
+}
+
+// ------------------------------------------------------------------ RoPE
+// Rotate-half RoPE: pair (x_i, x_{i+d/2}) turns by pos * theta_i with
+// theta_i = base^(-2i/d) (LaCache §3.3.2, Eq. 1; RoFormer). The angle is
+// formed in fp64 as a multiple of pi, reduced to [-1, 1] exactly in fp64, and
+// only then handed to CUDA's sincospi, so positions near 1.3e5 keep full
+// fp32 accuracy.
+__device__ __forceinline__ double rope_turns(int pos, double inv_freq_over_pi) {
+  double t = (double)pos * inv_freq_over_pi;
+  return t - 2.0 * rint(0.5 * t);
+}
+
+__device__ __forceinline__ float2 rope_cs_f32(int pos, double inv_freq_over_pi) {
+  float s, c;
+  sincospif((float)rope_turns(pos, inv_freq_over_pi), &s, &c);
+  return make_float2(c, s);
+}
+
+__device__ __forceinline__ void rope_cs_f64(int pos, double inv_freq_over_pi, double *c, double *s) {
+  sincospi(rope_turns(pos, inv_freq_over_pi), s, c);
+}
+
+// ------------------------------------------------------------------ bf16
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
+  return __uint_as_float(((uint32_t)h) << 16);
+}
+
+// fp64 -> bf16, one rounding to nearest even, from the IEEE encodings: keep the
+// exponent and the top 7 fraction bits of the fp64 pattern, round on the 45
+// dropped bits (a carry moves into the exponent by itself), then re-bias the
+// exponent from 1023 to 127. Values below bf16's normal range (|x| < 2^-126)
+// go through fp32.
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
+  unsigned long long u = (unsigned long long)__double_as_longlong(x);
+  unsigned long long sign = u >> 63;
+  unsigned long long a = u & 0x7FFFFFFFFFFFFFFFull;
+  if (a < 0x3810000000000000ull) return __bfloat16_as_ushort(__float2bfloat16_rn((float)x));
+  unsigned long long keep = a >> 45;
+  unsigned long long rem = a & ((1ull << 45) - 1);
+  const unsigned long long half = 1ull << 44;
+  keep += (rem > half || (rem == half && (keep & 1ull))) ? 1ull : 0ull;
+  return (uint16_t)((sign << 15) | (keep - (896ull << 7)));
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Scale factor e^(m_part - m) of a state whose max is m_part when the merged
+// max is m; an empty state (m_part = -inf) contributes 0.
+__device__ __forceinline__ float lse_weight(float m_part, float m) {
+  return m_part == -CUDART_INF_F ? 0.f : expf(m_part - m);
+}
+
+// Workspace view of the per-share states written by the prefix kernels.
+struct Workspace {
+  float *o;  // [slots, rows, d]
+  float *m;  // [slots, rows]
+  float *l;  // [slots, rows]
+  long long slots;
+};
+
+}  // namespace fbk

@@ -1,0 +1,511 @@
+// Prefix state on the 5th-generation tensor cores (FBK_BF16).
+//
+// What it computes: for every (sequence b, kv-head) unit, the online-softmax
+// state (O~, m, l) of the G*B block query rows of that kv-head over the cached
+// prefix keys 0..L_b-1: the FlashAttention recurrence of LaCache §3.3.3
+// (Eq. 2-6) whose result FACache keeps in HBM, here for the block's own query
+// rows (FlashBlock, Abstract: cached block-external attention).
+//
+// How (one CTA per SM-sized share of the flattened (unit, 64-key tile) list):
+//  * warp 0, one lane: TMA producer. Streams 64-key K and V tiles of the bf16
+//    cache (contiguous rows or pages) into an NS-stage ring, 128-byte swizzled,
+//    with an L2 evict-first policy (each KV byte is read once).
+//  * warp 1, one lane: MMA issuer. S = Q K^T (M=128 query rows, N=64 keys,
+//    K=d) into TMEM, then O += P V (M=128, N=d, K=64 keys) into a TMEM
+//    accumulator, all tcgen05.mma kind::f16 with fp32 accumulation. S of tile
+//    i+1 is issued before PV of tile i, and S is double-buffered in TMEM, so
+//    the tensor core works on the next tile while softmax runs.
+//  * warps 4..4+4*MT-1: one warpgroup per 128-row M-tile (MT = ceil(G*B/128)).
+//    GQA packing: all G query heads of a kv-head share each staged K/V tile,
+//    so every KV byte is read from HBM once per unit. Each thread owns one
+//    query row = one TMEM lane: it rotates and writes its Q row (bf16,
+//    swizzled) at the start of a piece, reads its S row from TMEM, applies
+//    the recurrence in the log2 domain and writes P~ (bf16) for the PV MMA.
+//    The O accumulator stays in TMEM; it is rescaled only when the running
+//    max grows by more than 2^8 over the reference max, which leaves the
+//    state exact (O~ and l share one reference max) and bounds P~ by 256.
+//    At the end of a piece the state is rebased to the true max and written
+//    to this share's workspace slot.
+// Every mbarrier wait is bounded (about a second); a timeout flags
+// FBK_DEVERR_TIMEOUT and all roles drain and return.
+#include <cudaTypedefs.h>
+
+#include "launch.h"
+#include "tc.cuh"
+
+namespace fbk {
+namespace {
+
+using namespace tc;
+
+template <int D, int MT>
+struct Cfg {
+  static constexpr int NS = (D == 128) ? (MT == 2 ? 3 : 4) : (MT == 2 ? 6 : 8);
+  static constexpr int Q_BYTES = 128 * D * 2;          // one M-tile of Q
+  static constexpr int KV_BYTES = KV_TILE * D * 2;     // one K (or V) stage
+  static constexpr int P_BYTES = 128 * KV_TILE * 2;    // one M-tile of P~
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + MT * Q_BYTES;
+  static constexpr int V_OFF = K_OFF + NS * KV_BYTES;
+  static constexpr int P_OFF = V_OFF + NS * KV_BYTES;
+  static constexpr int BAR_OFF = P_OFF + MT * P_BYTES;
+  // barrier indices
+  static constexpr int B_KFULL = 0, B_KEMPTY = NS, B_VFULL = 2 * NS, B_VEMPTY = 3 * NS;
+  static constexpr int B_QFULL = 4 * NS;
+  static constexpr int B_SFULL = B_QFULL + MT;        // [MT][2]
+  static constexpr int B_SEMPTY = B_SFULL + 2 * MT;   // [MT][2]
+  static constexpr int B_PFULL = B_SEMPTY + 2 * MT;
+  static constexpr int B_ODONE = B_PFULL + MT;
+  static constexpr int B_OFREE = B_ODONE + MT;
+  static constexpr int B_DRAIN = B_OFREE + MT;
+  static constexpr int NBAR = B_DRAIN + 1;
+  // per softmax warp: cos/sin(L theta_i) (float2) and theta_i (float), i < D/2
+  static constexpr int CS_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int TH_OFF = CS_OFF + 4 * MT * (D / 2) * 8;
+  static constexpr int MISC_OFF = TH_OFF + 4 * MT * (D / 2) * 4;
+  static constexpr int SMEM = MISC_OFF + 16 + 1024;   // + slack to align the base to 1024
+  static constexpr int THREADS = 128 + 128 * MT;
+  static constexpr int TMEM_S = 0;                    // S[mt][buf] at (2*mt + buf) * 64
+  static constexpr int TMEM_O = MT * 2 * KV_TILE;     // O[mt] at TMEM_O + mt * D
+  static constexpr int TMEM_USED = TMEM_O + MT * D;
+  static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(TMEM_USED <= 512, "tensor memory budget");
+};
+
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_test(bar, parity))
+    if (clock64() - t0 > WAIT_LIMIT_CLOCKS) return false;
+  return true;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128-byte
+// swizzled K-major tile (8-row atoms of 1024 bytes).
+__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <int D>
+__device__ __forceinline__ void load_kv_tile(const Geometry &g, const CUtensorMap *map, uint32_t dst,
+                                             const Piece &p, int j, int boxh, uint32_t bar,
+                                             uint64_t pol) {
+  for (int rb = 0; rb < KV_TILE / boxh; ++rb) {
+    const long long pos = (long long)j * KV_TILE + (long long)rb * boxh;
+    long long row = 0;  // rows at or past L are masked later; any valid row will do
+    if (pos < p.L) {
+      row = cache_row(g, p.b, p.kvh, pos);
+      if (row < 0) row = 0;
+    }
+#pragma unroll
+    for (int cb = 0; cb < D / 64; ++cb)
+      tma_load_2d(dst + cb * (KV_TILE * 128) + rb * boxh * 128, map, cb * 64, (int)row, bar, pol);
+  }
+}
+
+template <int D, int MT>
+__global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
+    prefix_tc_kernel(const __grid_constant__ Geometry g, const __nv_bfloat16 *__restrict__ q,
+                     const Workspace ws, const int shares, const __grid_constant__ CUtensorMap tmk,
+                     const __grid_constant__ CUtensorMap tmv, const int boxh) {
+  using C = Cfg<D, MT>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+  uint8_t *smem = smem_raw + pad;
+  const uint32_t sb = raw_addr + pad;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const long long T = total_tiles(g);
+  if (T == 0) return;
+  if (share_begin(blockIdx.x, T, shares) == share_begin(blockIdx.x + 1, T, shares)) return;
+
+  auto bar = [&](int idx) -> uint32_t { return sb + C::BAR_OFF + 8 * idx; };
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(bar(C::B_KFULL + s), 1);
+      mbar_init(bar(C::B_KEMPTY + s), 1);
+      mbar_init(bar(C::B_VFULL + s), 1);
+      mbar_init(bar(C::B_VEMPTY + s), 1);
+    }
+    for (int mt = 0; mt < MT; ++mt) {
+      mbar_init(bar(C::B_QFULL + mt), 128);
+      mbar_init(bar(C::B_SFULL + 2 * mt), 1);
+      mbar_init(bar(C::B_SFULL + 2 * mt + 1), 1);
+      mbar_init(bar(C::B_SEMPTY + 2 * mt), 128);
+      mbar_init(bar(C::B_SEMPTY + 2 * mt + 1), 128);
+      mbar_init(bar(C::B_PFULL + mt), 128);
+      mbar_init(bar(C::B_ODONE + mt), 1);
+      mbar_init(bar(C::B_OFREE + mt), 128);
+    }
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  // P~ rows of warps whose rows are all padding are never written: zero them once.
+  for (int i = threadIdx.x; i < MT * C::P_BYTES / 16; i += C::THREADS)
+    reinterpret_cast<uint4 *>(smem + C::P_OFF)[i] = make_uint4(0, 0, 0, 0);
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+  }
+  fence_proxy_async();
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      PieceWalker walk;
+      walk.init(g, blockIdx.x, T, shares);
+      Piece p;
+      int i = 0, k_issued = 0, v_issued = 0;
+      bool ok = true;
+      while (ok && walk.next(g, p)) {
+        for (int j = p.tile_begin; j < p.tile_end; ++j, ++i) {
+          const int st = i % C::NS;
+          const uint32_t ph = ((i / C::NS) & 1) ^ 1;
+          if (!mbar_wait(bar(C::B_KEMPTY + st), ph, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(bar(C::B_KFULL + st), C::KV_BYTES);
+          load_kv_tile<D>(g, &tmk, sb + C::K_OFF + st * C::KV_BYTES, p, j, boxh,
+                          bar(C::B_KFULL + st), pol);
+          ++k_issued;
+          if (!mbar_wait(bar(C::B_VEMPTY + st), ph, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(bar(C::B_VFULL + st), C::KV_BYTES);
+          load_kv_tile<D>(g, &tmv, sb + C::V_OFF + st * C::KV_BYTES, p, j, boxh,
+                          bar(C::B_VFULL + st), pol);
+          ++v_issued;
+        }
+      }
+      // no TMA write may be in flight when the CTA leaves
+      for (int n = max(0, k_issued - C::NS); n < k_issued; ++n)
+        mbar_wait_drain(bar(C::B_KFULL + n % C::NS), (n / C::NS) & 1);
+      for (int n = max(0, v_issued - C::NS); n < v_issued; ++n)
+        mbar_wait_drain(bar(C::B_VFULL + n % C::NS), (n / C::NS) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, KV_TILE, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
+      PieceWalker walk;
+      walk.init(g, blockIdx.x, T, shares);
+      Piece p;
+      int i = 0, pi = 0;
+      bool ok = true;
+      // O[mt] += P~[mt] V for tile ii (the piece's first tile overwrites O)
+      auto issue_pv = [&](int ii, bool first) -> bool {
+        const int st = ii % C::NS;
+        if (!mbar_wait(bar(C::B_VFULL + st), (ii / C::NS) & 1, abort_flag)) return false;
+        if (first && pi > 0)
+          for (int mt = 0; mt < MT; ++mt)
+            if (!mbar_wait(bar(C::B_OFREE + mt), (pi - 1) & 1, abort_flag)) return false;
+        for (int mt = 0; mt < MT; ++mt) {
+          if (!mbar_wait(bar(C::B_PFULL + mt), ii & 1, abort_flag)) return false;
+          fence_after_sync();
+          const uint32_t d_tmem = tmem + C::TMEM_O + mt * D;
+#pragma unroll
+          for (int kk = 0; kk < KV_TILE / 16; ++kk) {
+            const uint64_t a = sdesc_sw128(sb + C::P_OFF + mt * C::P_BYTES + kk * 32, 16, 1024);
+            const uint64_t b = sdesc_sw128(sb + C::V_OFF + st * C::KV_BYTES + kk * 2048,
+                                           KV_TILE * 128, 1024);
+            mma_bf16(d_tmem, a, b, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+          }
+          mma_commit(bar(C::B_ODONE + mt));
+        }
+        mma_commit(bar(C::B_VEMPTY + st));
+        return true;
+      };
+      while (ok && walk.next(g, p)) {
+        for (int mt = 0; mt < MT && ok; ++mt)
+          ok = mbar_wait(bar(C::B_QFULL + mt), pi & 1, abort_flag);
+        if (!ok) break;
+        fence_after_sync();
+        const int n = p.tile_end - p.tile_begin;
+        for (int jj = 0; jj < n && ok; ++jj, ++i) {
+          const int st = i % C::NS, buf = i & 1;
+          if (!mbar_wait(bar(C::B_KFULL + st), (i / C::NS) & 1, abort_flag)) { ok = false; break; }
+          fence_after_sync();
+          for (int mt = 0; mt < MT && ok; ++mt) {
+            if (!mbar_wait(bar(C::B_SEMPTY + 2 * mt + buf), ((i >> 1) & 1) ^ 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            fence_after_sync();
+            const uint32_t d_tmem = tmem + C::TMEM_S + (2 * mt + buf) * KV_TILE;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const int cb = kk >> 2, ko = (kk & 3) * 32;
+              const uint64_t a = sdesc_sw128(sb + C::Q_OFF + mt * C::Q_BYTES + cb * 128 * 128 + ko, 16, 1024);
+              const uint64_t b = sdesc_sw128(sb + C::K_OFF + st * C::KV_BYTES + cb * KV_TILE * 128 + ko, 16, 1024);
+              mma_bf16(d_tmem, a, b, IDESC_S, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(C::B_SFULL + 2 * mt + buf));
+          }
+          if (!ok) break;
+          mma_commit(bar(C::B_KEMPTY + st));
+          if (jj > 0 && !issue_pv(i - 1, jj == 1)) { ok = false; break; }
+        }
+        if (ok && !issue_pv(i - 1, n == 1)) ok = false;
+        ++pi;
+      }
+      mma_commit(bar(C::B_DRAIN));
+      mbar_wait_drain(bar(C::B_DRAIN), 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- softmax
+    const int mt = (warp - 4) >> 2, wq = warp & 3;
+    const int row = wq * 32 + lane;              // row inside the M-tile = TMEM lane
+    const int r = mt * 128 + row;                // query row inside the unit
+    const bool wact = mt * 128 + wq * 32 < g.rows;  // warp holds at least one real row
+    const uint32_t tl = (uint32_t)(wq * 32) << 16;
+    const float sl2 = g.tau * 1.4426950408889634f;  // scores in log2 units
+    // Per-warp RoPE tables, so the warps of a warpgroup never wait on each other
+    // (only bounded mbarrier waits cross warps).
+    const int wid = warp - 4;
+    float2 *csL = reinterpret_cast<float2 *>(smem + C::CS_OFF) + wid * (D / 2);
+    float *thf = reinterpret_cast<float *>(smem + C::TH_OFF) + wid * (D / 2);
+    for (int ii = lane; ii < D / 2; ii += 32) thf[ii] = (float)(g.inv_freq_over_pi[ii] * CUDART_PI);
+    // waits are made warp-uniform so that warp-collective TMEM accesses never diverge
+    auto wwait = [&](uint32_t b, uint32_t ph) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(b, ph, abort_flag));
+    };
+    PieceWalker walk;
+    walk.init(g, blockIdx.x, T, shares);
+    Piece p;
+    int i = 0;
+    bool ok = true;
+    while (ok && walk.next(g, p)) {
+      // cos/sin(L theta_i) for this piece; row t adds t theta_i by angle addition
+      __syncwarp();
+      for (int ii = lane; ii < D / 2; ii += 32) csL[ii] = rope_cs_f32(p.L, g.inv_freq_over_pi[ii]);
+      __syncwarp();
+      if (wact) {
+        const uint32_t qbase = sb + C::Q_OFF + mt * C::Q_BYTES;
+        const bool real = r < g.rows;
+        const int hl = real ? r / g.blk : 0, t = real ? r % g.blk : 0;
+        const __nv_bfloat16 *src = q + (((long long)p.b * g.blk + t) * g.hq + p.kvh * g.group + hl) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          uint4 a = make_uint4(0, 0, 0, 0), bq = make_uint4(0, 0, 0, 0);
+          if (real) {
+            a = *reinterpret_cast<const uint4 *>(src + 8 * c);
+            bq = *reinterpret_cast<const uint4 *>(src + D / 2 + 8 * c);
+          }
+          const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {bq.x, bq.y, bq.z, bq.w};
+          uint32_t y1w[4], y2w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float y1[2], y2[2];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int ii = 8 * c + 2 * e + h2;
+              const float x1 = __uint_as_float(h2 ? (aw[e] & 0xffff0000u) : (aw[e] << 16));
+              const float x2 = __uint_as_float(h2 ? (bw[e] & 0xffff0000u) : (bw[e] << 16));
+              float st_, ct_;
+              __sincosf((float)t * thf[ii], &st_, &ct_);
+              const float2 cl = csL[ii];
+              const float cs = cl.x * ct_ - cl.y * st_, sn = cl.y * ct_ + cl.x * st_;
+              y1[h2] = x1 * cs - x2 * sn;
+              y2[h2] = x2 * cs + x1 * sn;
+            }
+            y1w[e] = pack_bf16(y1[0], y1[1]);
+            y2w[e] = pack_bf16(y2[0], y2[1]);
+          }
+          const int e1 = 8 * c, e2 = D / 2 + 8 * c;  // first element of each chunk
+          st_shared_v4(qbase + (e1 / 64) * 16384 + sw128(row, (e1 % 64) / 8), y1w[0], y1w[1], y1w[2], y1w[3]);
+          st_shared_v4(qbase + (e2 / 64) * 16384 + sw128(row, (e2 % 64) / 8), y2w[0], y2w[1], y2w[2], y2w[3]);
+        }
+      }
+      fence_proxy_async();
+      mbar_arrive(bar(C::B_QFULL + mt));
+
+      float m_ref = -CUDART_INF_F, m_true = -CUDART_INF_F, lsum = 0.f;
+      const int n = p.tile_end - p.tile_begin;
+      for (int jj = 0; jj < n; ++jj, ++i) {
+        const int buf = i & 1;
+        if (!wwait(bar(C::B_SFULL + 2 * mt + buf), (i >> 1) & 1)) { ok = false; break; }
+        fence_after_sync();
+        uint32_t sr[64];
+        if (wact) {
+          const uint32_t ta = tmem + tl + C::TMEM_S + (2 * mt + buf) * KV_TILE;
+          tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(sr));
+          tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+          tmem_wait_ld();
+        }
+        fence_before_sync();
+        mbar_arrive(bar(C::B_SEMPTY + 2 * mt + buf));
+        uint32_t pk[32];
+        if (wact) {
+          const int j = p.tile_begin + jj;
+          const int nval = min(KV_TILE, p.L - j * KV_TILE);
+          float tmax = -CUDART_INF_F;  // S is scaled to log2 units in place
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float v = c < nval ? __uint_as_float(sr[c]) * sl2 : -CUDART_INF_F;
+            sr[c] = __float_as_uint(v);
+            tmax = fmaxf(tmax, v);
+          }
+          m_true = fmaxf(m_true, tmax);
+          const bool need = jj > 0 && tmax > m_ref + 8.f;
+          if (jj == 0) m_ref = tmax;
+          if (__any_sync(0xffffffffu, need)) {
+            // rescale this row's O~ (and l) to the new reference max
+            if (!wwait(bar(C::B_ODONE + mt), (i - 1) & 1)) ok = false;
+            fence_after_sync();
+            const float f = need ? exp2f(m_ref - tmax) : 1.f;
+            if (ok) {
+#pragma unroll 1
+              for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                const uint32_t ta = tmem + tl + C::TMEM_O + mt * D + cc * 32;
+                tmem_ld32(ta, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                tmem_st32(ta, o);
+              }
+              tmem_wait_st();
+            }
+            if (need) {
+              lsum *= f;
+              m_ref = tmax;
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const uint32_t w = pack_bf16(exp2f(__uint_as_float(sr[2 * c]) - m_ref),
+                                         exp2f(__uint_as_float(sr[2 * c + 1]) - m_ref));
+            lsum += __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
+            pk[c] = w;
+          }
+        }
+        if (!ok) break;
+        // P~ buffer is free once the previous tile's PV has completed
+        if (i > 0 && !wwait(bar(C::B_ODONE + mt), (i - 1) & 1)) { ok = false; break; }
+        if (wact) {
+          const uint32_t pbase = sb + C::P_OFF + mt * C::P_BYTES;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(pbase + sw128(row, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        mbar_arrive(bar(C::B_PFULL + mt));
+      }
+      if (!ok) break;
+      // epilogue: rebase to the true max and store this piece's state
+      if (!wwait(bar(C::B_ODONE + mt), (i - 1) & 1)) { ok = false; break; }
+      fence_after_sync();
+      if (wact) {
+        const float f = exp2f(m_ref - m_true);
+        const long long srow = ((long long)blockIdx.x + p.u) * g.rows + r;
+        float *dst = ws.o + srow * D;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tmem + tl + C::TMEM_O + mt * D + cc * 32, o);
+          tmem_wait_ld();
+          if (r < g.rows) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4 *>(dst + cc * 32 + e) =
+                  make_float4(__uint_as_float(o[e]) * f, __uint_as_float(o[e + 1]) * f,
+                              __uint_as_float(o[e + 2]) * f, __uint_as_float(o[e + 3]) * f);
+          }
+        }
+        if (r < g.rows) {
+          ws.m[srow] = m_true * 0.6931471805599453f;  // back to natural-log units
+          ws.l[srow] = lsum * f;
+        }
+      }
+      fence_before_sync();
+      mbar_arrive(bar(C::B_OFREE + mt));
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) raise_flag(g, FBK_DEVERR_TIMEOUT);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;  // driver entry point, looked up once
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over the cache viewed as [rows, d] bf16, boxes of 64 columns x boxh rows, 128B swizzle.
+bool make_map(CUtensorMap *m, const void *base, long long rows, int d, int boxh) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)boxh};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int MT>
+cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const Workspace &ws, int shares,
+                       cudaStream_t st) {
+  using C = Cfg<D, MT>;
+  const long long rows = g.paged ? g.num_pages * g.hkv * g.page_size : (long long)g.batch * g.hkv * g.cap;
+  const int boxh = g.paged ? min(g.page_size, KV_TILE) : KV_TILE;
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, g.kc, rows, D, boxh) || !make_map(&mv, g.vc, rows, D, boxh))
+    return cudaErrorInvalidValue;
+  auto kern = prefix_tc_kernel<D, MT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<shares, C::THREADS, C::SMEM, st>>>(g, q, ws, shares, mk, mv, boxh);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefix_tc(const Geometry &g, const __nv_bfloat16 *q, const Workspace &ws,
+                             int shares, cudaStream_t st) {
+  const bool two = g.rows > 128;
+  if (g.d == 128)
+    return two ? launch_cfg<128, 2>(g, q, ws, shares, st) : launch_cfg<128, 1>(g, q, ws, shares, st);
+  return two ? launch_cfg<64, 2>(g, q, ws, shares, st) : launch_cfg<64, 1>(g, q, ws, shares, st);
+}
+
+}  // namespace fbk

@@ -1,0 +1,206 @@
+"""Python binding of libfbk.so (the cached block attention C ABI, include/fbk.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library. Tensors are torch CUDA tensors (device memory and streams come from
+PyTorch); their data pointers and the current CUDA stream are passed through
+ctypes. Importing this module fails loudly when the library is not built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfbk.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m cached_block_attention_b200.build` "
+        "(there is no fallback implementation)")
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK = 0
+BF16 = 0
+FP32_CHECK = 1
+
+DEVERR_PREFIX_LEN = 1
+DEVERR_PAGE_ID = 2
+DEVERR_COMMIT = 4
+DEVERR_TIMEOUT = 8
+
+EXPORTS = ("fbk_prefix_workspace_bytes", "fbk_default_num_splits", "fbk_prefix_partial",
+           "fbk_block_attn_merge", "fbk_commit_block_rope_append", "fbk_full_ref_attn",
+           "fbk_status_string")
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("block_len", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+                ("rope_base", ctypes.c_double), ("mode", ctypes.c_int32)]
+
+
+class _Cache(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("paged", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+                ("capacity_tokens", ctypes.c_int64), ("num_pages", ctypes.c_int64),
+                ("page_table", ctypes.c_void_p), ("prefix_lens", ctypes.c_void_p),
+                ("error_flags", ctypes.c_void_p)]
+
+
+class _Partial(ctypes.Structure):
+    _fields_ = [("o_unnorm", ctypes.c_void_p), ("m", ctypes.c_void_p), ("l", ctypes.c_void_p)]
+
+
+_P = ctypes.POINTER
+_vp = ctypes.c_void_p
+_lib.fbk_prefix_workspace_bytes.argtypes = [_P(_Shape), _P(_Cache), ctypes.c_int32]
+_lib.fbk_prefix_workspace_bytes.restype = ctypes.c_size_t
+_lib.fbk_default_num_splits.argtypes = []
+_lib.fbk_default_num_splits.restype = ctypes.c_int32
+_lib.fbk_prefix_partial.argtypes = [_P(_Shape), _vp, _P(_Cache), _P(_Partial), _vp, ctypes.c_size_t,
+                                    ctypes.c_int32, _vp]
+_lib.fbk_prefix_partial.restype = ctypes.c_int
+_lib.fbk_block_attn_merge.argtypes = [_P(_Shape), _vp, _vp, _vp, _vp, _P(_Partial), _vp, _vp, _vp]
+_lib.fbk_block_attn_merge.restype = ctypes.c_int
+_lib.fbk_commit_block_rope_append.argtypes = [_P(_Shape), _vp, _vp, _P(_Cache), _vp]
+_lib.fbk_commit_block_rope_append.restype = ctypes.c_int
+_lib.fbk_full_ref_attn.argtypes = [_P(_Shape), _vp, _vp, _vp, _P(_Cache), _vp, _vp, _vp]
+_lib.fbk_full_ref_attn.restype = ctypes.c_int
+_lib.fbk_status_string.argtypes = [ctypes.c_int]
+_lib.fbk_status_string.restype = ctypes.c_char_p
+
+
+class FbkError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+def status_string(status: int) -> str:
+    return _lib.fbk_status_string(int(status)).decode()
+
+
+@dataclass
+class Shape:
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    block_len: int
+    softmax_scale: float = 1.0
+    rope_base: float = 1e4
+    mode: int = BF16
+
+    def c(self) -> _Shape:
+        return _Shape(self.batch, self.n_q_heads, self.n_kv_heads, self.head_dim, self.block_len,
+                      self.softmax_scale, self.rope_base, self.mode)
+
+
+@dataclass
+class KVCache:
+    """Contiguous: k, v [b, Hkv, cap, d] bf16. Paged: k, v [P, Hkv, page, d] bf16 plus
+    page_table int32 [b, max_pages]. prefix_lens int32 [b] on the device."""
+    k: torch.Tensor
+    v: torch.Tensor
+    prefix_lens: torch.Tensor
+    page_table: torch.Tensor | None = None
+    error_flags: torch.Tensor | None = None
+
+    @property
+    def paged(self) -> bool:
+        return self.page_table is not None
+
+    def c(self) -> _Cache:
+        pt = self.page_table
+        return _Cache(
+            self.k.data_ptr(), self.v.data_ptr(), 1 if pt is not None else 0,
+            self.k.shape[2] if pt is not None else 0,
+            pt.shape[1] if pt is not None else 0,
+            0 if pt is not None else self.k.shape[2],
+            self.k.shape[0] if pt is not None else 0,
+            pt.data_ptr() if pt is not None else None,
+            self.prefix_lens.data_ptr(),
+            self.error_flags.data_ptr() if self.error_flags is not None else None)
+
+
+@dataclass
+class Partial:
+    o_unnorm: torch.Tensor  # fp32 [b, Hq, B, d]
+    m: torch.Tensor         # fp32 [b, Hq, B]
+    l: torch.Tensor         # fp32 [b, Hq, B]
+
+    @staticmethod
+    def empty(shape: Shape, device="cuda") -> "Partial":
+        b, h, B, d = shape.batch, shape.n_q_heads, shape.block_len, shape.head_dim
+        return Partial(torch.empty(b, h, B, d, dtype=torch.float32, device=device),
+                       torch.empty(b, h, B, dtype=torch.float32, device=device),
+                       torch.empty(b, h, B, dtype=torch.float32, device=device))
+
+    def c(self) -> _Partial:
+        return _Partial(self.o_unnorm.data_ptr(), self.m.data_ptr(), self.l.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(status, what):
+    if status != OK:
+        raise FbkError(status, what)
+
+
+def default_num_splits() -> int:
+    return int(_lib.fbk_default_num_splits())
+
+
+def prefix_workspace_bytes(shape: Shape, cache: KVCache | None, num_splits: int = 0) -> int:
+    cs = shape.c()
+    cc = cache.c() if cache is not None else None
+    return int(_lib.fbk_prefix_workspace_bytes(ctypes.byref(cs), ctypes.byref(cc) if cc else None,
+                                               num_splits))
+
+
+def prefix_partial(shape: Shape, q_blk: torch.Tensor, cache: KVCache, out: Partial,
+                   ws: torch.Tensor, num_splits: int = 0, stream=None) -> None:
+    cs, cc, po = shape.c(), cache.c(), out.c()
+    _check(_lib.fbk_prefix_partial(ctypes.byref(cs), _ptr(q_blk), ctypes.byref(cc), ctypes.byref(po),
+                                   _ptr(ws), ws.numel() * ws.element_size(), num_splits,
+                                   _stream(stream)), "fbk_prefix_partial")
+
+
+def block_attn_merge(shape: Shape, q_blk, k_blk, v_blk, prefix_lens, prefix: Partial, out,
+                     lse=None, stream=None) -> None:
+    cs, po = shape.c(), prefix.c()
+    _check(_lib.fbk_block_attn_merge(ctypes.byref(cs), _ptr(q_blk), _ptr(k_blk), _ptr(v_blk),
+                                     _ptr(prefix_lens), ctypes.byref(po), _ptr(out), _ptr(lse),
+                                     _stream(stream)), "fbk_block_attn_merge")
+
+
+def commit_block_rope_append(shape: Shape, k_blk, v_blk, cache: KVCache, stream=None) -> None:
+    cs, cc = shape.c(), cache.c()
+    _check(_lib.fbk_commit_block_rope_append(ctypes.byref(cs), _ptr(k_blk), _ptr(v_blk),
+                                             ctypes.byref(cc), _stream(stream)),
+           "fbk_commit_block_rope_append")
+
+
+def full_ref_attn(shape: Shape, q_blk, k_blk, v_blk, cache: KVCache, out, lse=None,
+                  stream=None) -> None:
+    cs, cc = shape.c(), cache.c()
+    _check(_lib.fbk_full_ref_attn(ctypes.byref(cs), _ptr(q_blk), _ptr(k_blk), _ptr(v_blk),
+                                  ctypes.byref(cc), _ptr(out), _ptr(lse), _stream(stream)),
+           "fbk_full_ref_attn")
+
+
+# raw handles for tests of the C ABI itself
+lib = _lib
+CShape, CCache, CPartial = _Shape, _Cache, _Partial

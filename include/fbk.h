@@ -1,0 +1,178 @@
+/*
+ * fbk.h - C ABI of the cached block attention library (libfbk.so).
+ *
+ * One attention layer of one denoising step of block (semi-autoregressive)
+ * diffusion decoding. The current block of B query tokens of sequence b sits
+ * at absolute positions L_b .. L_b+B-1, after a cached prefix of L_b tokens
+ * (LaCache, "Exact Caching and Precision-Adaptive Inference for Diffusion Large
+ * Language Models", §3.3.1 Notation, App. B.1). The block attends
+ * bidirectionally to the prefix and to itself. The prefix contribution is kept
+ * as the FlashAttention online-softmax state (O~, m, l) of LaCache §3.3.3
+ * (FACache, Eq. 2-6), computed once per block and reused at every denoising
+ * step of the block (FlashBlock, "Attention Caching for Efficient Long-Context
+ * Block Diffusion", Abstract), where it is merged by log-sum-exp with a fresh
+ * in-block state. When the block is final, its K is rotated (RoPE) and K/V are
+ * appended to the cache (LaCache §3.3.2 RoPECache, Eq. 1).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Memory. Every pointer argument is DEVICE memory owned by the caller,
+ *    except the structs themselves (fbk_shape, fbk_kv_cache, fbk_partial),
+ *    which are host structs read during the call only. The library allocates
+ *    nothing, keeps no state between calls and never synchronises.
+ *  - Streams. `cuda_stream` is a cudaStream_t (NULL = legacy default stream).
+ *    Every call only enqueues work on it and returns.
+ *  - Errors. Argument errors are detected on the host and returned before any
+ *    launch. A launch failure returns FBK_ERR_CUDA. Conditions that depend on
+ *    device-resident values (prefix lengths, page ids) are checked on the
+ *    device: the offending sequence is skipped and a bit is OR-ed into
+ *    cache->error_flags (FBK_DEVERR_*), when that pointer is not NULL.
+ *  - Types. bf16 is IEEE bfloat16 (uint16 storage). fp32 state is IEEE float.
+ *  - Element order. Row-major; the last index is contiguous.
+ *
+ * Notation: b batch, Hq query heads, Hkv kv-heads (G = Hq/Hkv query heads per
+ * kv-head, head h reads kv-head floor(h*Hkv/Hq)), d head_dim, B block_len,
+ * L_b prefix length of sequence b, tau softmax scale.
+ */
+#ifndef FBK_H_
+#define FBK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fbk_status {
+  FBK_OK = 0,
+  FBK_ERR_INVALID_ARG = -1,  /* NULL pointer, non-positive size, bad struct field */
+  FBK_ERR_UNSUPPORTED = -2,  /* d not in {64,128}, Hq % Hkv != 0, G*B > 256, B > 64 ... */
+  FBK_ERR_CAPACITY = -3,     /* cache geometry cannot hold the request */
+  FBK_ERR_WORKSPACE = -4,    /* workspace NULL or smaller than fbk_prefix_workspace_bytes */
+  FBK_ERR_CUDA = -5          /* a CUDA runtime call or launch failed */
+} fbk_status;
+
+/* Arithmetic of a call.
+ *  FBK_BF16: production path. Block Q and the prefix P~ enter the tensor-core
+ *    products as bf16 (fp32 accumulation); the output O is bf16.
+ *  FBK_FP32_CHECK: the same operations on CUDA cores in fp32 from the same
+ *    bf16 inputs (no bf16 rounding of Q^ or P~); the output O is fp32. */
+typedef enum fbk_mode { FBK_BF16 = 0, FBK_FP32_CHECK = 1 } fbk_mode;
+
+/* Device error bits OR-ed into fbk_kv_cache.error_flags. */
+#define FBK_DEVERR_PREFIX_LEN 1u /* prefix_lens[b] < 0 or beyond the cache capacity: b skipped */
+#define FBK_DEVERR_PAGE_ID 2u    /* a page-table entry outside [0, num_pages) was needed */
+#define FBK_DEVERR_COMMIT 4u     /* commit would write past the capacity: block not appended */
+#define FBK_DEVERR_TIMEOUT 8u    /* a bounded device-side wait gave up (kernel returned early) */
+
+typedef struct fbk_shape {
+  int32_t batch;       /* b >= 1 */
+  int32_t n_q_heads;   /* Hq >= 1 */
+  int32_t n_kv_heads;  /* Hkv >= 1, Hq % Hkv == 0 */
+  int32_t head_dim;    /* d in {64, 128} */
+  int32_t block_len;   /* B in [1, 64]; G*B <= 256 */
+  float softmax_scale; /* tau: scores are tau * <RoPE(q), k> (the pages write S = Q K^T: tau = 1) */
+  double rope_base;    /* theta_i = rope_base^(-2i/d), rotate-half pairs (i, i + d/2) */
+  int32_t mode;        /* fbk_mode */
+} fbk_shape;
+
+/* The KV cache: post-RoPE K and V of every committed token (RoPECache).
+ * Contiguous: k, v are bf16 [b, Hkv, capacity_tokens, d]; token p of sequence
+ *   b, kv-head g is row (b*Hkv + g)*capacity_tokens + p.
+ * Paged (paged != 0): k, v are bf16 [num_pages, Hkv, page_size, d]; token p of
+ *   sequence b lives in page page_table[b*max_pages_per_seq + p/page_size] at
+ *   offset p % page_size. page_size is a power of two >= 16.
+ * prefix_lens: int32 [b], the committed length L_b of each sequence. It is
+ *   read by every call and advanced by B by fbk_commit_block_rope_append.
+ * error_flags: int32 [1] or NULL; FBK_DEVERR_* bits are OR-ed in, never cleared. */
+typedef struct fbk_kv_cache {
+  void *k;
+  void *v;
+  int32_t paged;
+  int32_t page_size;
+  int32_t max_pages_per_seq;
+  int64_t capacity_tokens; /* contiguous layout only */
+  int64_t num_pages;       /* paged layout only */
+  const int32_t *page_table;
+  int32_t *prefix_lens;
+  int32_t *error_flags;
+} fbk_kv_cache;
+
+/* An online-softmax state per (sequence, query head, block row), LaCache §3.3.3:
+ * o_unnorm = O~ fp32 [b, Hq, B, d]; m fp32 [b, Hq, B] (the running max of the
+ * scaled scores, natural-log units); l fp32 [b, Hq, B] (sum of exp(s - m)).
+ * O~ and l are relative to that m. A row with no keys holds (0, -inf, 0). */
+typedef struct fbk_partial {
+  float *o_unnorm;
+  float *m;
+  float *l;
+} fbk_partial;
+
+/* Bytes of scratch fbk_prefix_partial needs for `num_splits` work shares
+ * (0 = one share per SM of the current device). Depends only on b, Hkv, G*B,
+ * d and the share count, not on the prefix lengths. Returns 0 for an invalid
+ * shape. */
+size_t fbk_prefix_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache,
+                                  int32_t num_splits);
+
+/* The share count that num_splits = 0 selects on the current device. */
+int32_t fbk_default_num_splits(void);
+
+/* Prefix state of the block queries over the cached prefix (FACache's cached
+ * state, LaCache §3.3.3, Eq. 2-6, restricted to keys 0..L_b-1; FlashBlock's
+ * cached block-external attention).
+ *  q_blk: bf16 [b, B, Hq, d], PRE-RoPE; row t of sequence b is rotated at
+ *         position prefix_lens[b] + t inside the kernel.
+ *  out:   the state, written in full (every row of every head).
+ *  ws:    device scratch of at least fbk_prefix_workspace_bytes(...) bytes,
+ *         caller-owned, contents irrelevant on entry.
+ *  num_splits: number of equal shares of the flattened (sequence, kv-head,
+ *         64-key tile) work list, one CTA each (0 = one per SM).
+ * Two launches: the share kernel, then a fixed-order LSE reduction of the
+ * per-share states (deterministic run to run). */
+fbk_status fbk_prefix_partial(const fbk_shape *shape, const void *q_blk, const fbk_kv_cache *cache,
+                              const fbk_partial *out, void *ws, size_t ws_bytes,
+                              int32_t num_splits, void *cuda_stream);
+
+/* One denoising step: in-block bidirectional attention (no mask) of the block
+ * queries over the block keys, LSE-merged with the cached prefix state and
+ * normalised: O = (e^(m1-m) O~1 + e^(m2-m) O~2) / (e^(m1-m) l1 + e^(m2-m) l2),
+ * m = max(m1, m2), lse = m + log l (LaCache App. J, initialise with cache,
+ * final normalisation and logsumexp).
+ *  q_blk: bf16 [b, B, Hq, d] pre-RoPE; k_blk, v_blk: bf16 [b, B, Hkv, d], K pre-RoPE.
+ *  prefix_lens: int32 [b] device (positions are prefix_lens[b] + t).
+ *  prefix: a state from fbk_prefix_partial (read only).
+ *  out: [b, B, Hq, d], bf16 (FBK_BF16) or fp32 (FBK_FP32_CHECK).
+ *  lse: fp32 [b, Hq, B] or NULL. */
+fbk_status fbk_block_attn_merge(const fbk_shape *shape, const void *q_blk, const void *k_blk,
+                                const void *v_blk, const int32_t *prefix_lens,
+                                const fbk_partial *prefix, void *out, float *lse,
+                                void *cuda_stream);
+
+/* Commit a finished block: K^ = RoPE(k_blk, L_b + t) computed in fp64 and
+ * rounded once to bf16 (nearest even), V copied bit for bit, both written to
+ * cache slots L_b .. L_b+B-1; then prefix_lens[b] += B (RoPECache,
+ * LaCache §3.3.2, Eq. 1). A sequence whose block does not fit is left
+ * unchanged and FBK_DEVERR_COMMIT is flagged. One CTA per sequence. */
+fbk_status fbk_commit_block_rope_append(const fbk_shape *shape, const void *k_blk,
+                                        const void *v_blk, fbk_kv_cache *cache,
+                                        void *cuda_stream);
+
+/* Uncached reference: softmax attention of the block queries over
+ * [prefix keys 0..L_b-1 ; RoPE(k_blk)] in one fp32 pass on CUDA cores, with
+ * no cached state (the computation FACache must reproduce exactly, LaCache
+ * §3.1). Independent device code, used as a GPU cross-check. Output as in
+ * fbk_block_attn_merge. */
+fbk_status fbk_full_ref_attn(const fbk_shape *shape, const void *q_blk, const void *k_blk,
+                             const void *v_blk, const fbk_kv_cache *cache, void *out,
+                             float *lse, void *cuda_stream);
+
+/* Static text for a status code. */
+const char *fbk_status_string(fbk_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FBK_H_ */

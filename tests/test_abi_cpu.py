@@ -1,0 +1,127 @@
+"""CPU-side checks of the C ABI: the library loads, exports every entry point
+include/fbk.h declares, and rejects bad arguments on the host before any CUDA
+call (nothing here launches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fbk():
+    from cached_block_attention_b200 import build
+    build.build()
+    from cached_block_attention_b200 import fbk as m
+    return m
+
+
+def declared_entry_points():
+    text = open(os.path.join(ROOT, "include", "fbk.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fbk_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(fbk):
+    names = declared_entry_points()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(fbk.lib, n), n
+    assert set(fbk.EXPORTS) == set(names)
+
+
+def test_status_strings(fbk):
+    for code in (0, -1, -2, -3, -4, -5):
+        assert fbk.status_string(code) not in ("", "unknown status")
+    assert fbk.status_string(7) == "unknown status"
+
+
+def _shape(fbk, **kw):
+    s = dict(batch=1, n_q_heads=4, n_kv_heads=2, head_dim=128, block_len=32,
+             softmax_scale=1.0, rope_base=1e4, mode=0)
+    s.update(kw)
+    return fbk.CShape(**s)
+
+
+def _cache(fbk, **kw):
+    c = dict(k=0x10000, v=0x20000, paged=0, page_size=0, max_pages_per_seq=0,
+             capacity_tokens=1024, num_pages=0, page_table=None, prefix_lens=0x30000,
+             error_flags=None)
+    c.update(kw)
+    return fbk.CCache(**c)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(batch=0), -1), (dict(n_q_heads=0), -1), (dict(block_len=0), -1), (dict(mode=3), -1),
+    (dict(rope_base=-1.0), -1), (dict(softmax_scale=float("nan")), -1),
+    (dict(head_dim=96), -2), (dict(n_q_heads=6, n_kv_heads=4), -2), (dict(block_len=65), -2),
+    (dict(n_q_heads=16, n_kv_heads=2, block_len=64), -2),
+])
+def test_shape_validation(fbk, kw, code):
+    s = _shape(fbk, **kw)
+    c = _cache(fbk)
+    p = fbk.CPartial(0x40000, 0x50000, 0x60000)
+    st = fbk.lib.fbk_prefix_partial(ctypes.byref(s), ctypes.c_void_p(0x70000), ctypes.byref(c),
+                                    ctypes.byref(p), ctypes.c_void_p(0x80000), 1 << 30, 4, None)
+    assert st == code
+    st = fbk.lib.fbk_block_attn_merge(ctypes.byref(s), ctypes.c_void_p(0x70000), ctypes.c_void_p(0x70000),
+                                      ctypes.c_void_p(0x70000), ctypes.c_void_p(0x30000), ctypes.byref(p),
+                                      ctypes.c_void_p(0x90000), None, None)
+    assert st == code
+    assert fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), ctypes.byref(c), 4) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), -1), (dict(prefix_lens=None), -1), (dict(capacity_tokens=0), -1),
+    (dict(k=0x10008), -2),
+    (dict(paged=1, page_size=64, max_pages_per_seq=4, num_pages=8, page_table=None), -1),
+    (dict(paged=1, page_size=48, max_pages_per_seq=4, num_pages=8, page_table=0x1000), -2),
+    (dict(paged=1, page_size=8, max_pages_per_seq=4, num_pages=8, page_table=0x1000), -2),
+    (dict(capacity_tokens=1 << 31), -3),
+])
+def test_cache_validation(fbk, kw, code):
+    s = _shape(fbk)
+    c = _cache(fbk, **kw)
+    p = fbk.CPartial(0x40000, 0x50000, 0x60000)
+    st = fbk.lib.fbk_prefix_partial(ctypes.byref(s), ctypes.c_void_p(0x70000), ctypes.byref(c),
+                                    ctypes.byref(p), ctypes.c_void_p(0x80000), 1 << 30, 4, None)
+    assert st == code
+    st = fbk.lib.fbk_commit_block_rope_append(ctypes.byref(s), ctypes.c_void_p(0x70000),
+                                              ctypes.c_void_p(0x70000), ctypes.byref(c), None)
+    assert st == code
+    st = fbk.lib.fbk_full_ref_attn(ctypes.byref(s), ctypes.c_void_p(0x70000), ctypes.c_void_p(0x70000),
+                                   ctypes.c_void_p(0x70000), ctypes.byref(c), ctypes.c_void_p(0x90000),
+                                   None, None)
+    assert st == code
+
+
+def test_null_pointers(fbk):
+    s = _shape(fbk)
+    c = _cache(fbk)
+    p = fbk.CPartial(0x40000, 0x50000, 0x60000)
+    assert fbk.lib.fbk_prefix_partial(None, None, None, None, None, 0, 0, None) == -1
+    assert fbk.lib.fbk_prefix_partial(ctypes.byref(s), None, ctypes.byref(c), ctypes.byref(p),
+                                      ctypes.c_void_p(0x80000), 1 << 30, 4, None) == -1
+    bad = fbk.CPartial(0x40000, None, 0x60000)
+    assert fbk.lib.fbk_prefix_partial(ctypes.byref(s), ctypes.c_void_p(0x70000), ctypes.byref(c),
+                                      ctypes.byref(bad), ctypes.c_void_p(0x80000), 1 << 30, 4, None) == -1
+    assert fbk.lib.fbk_block_attn_merge(ctypes.byref(s), None, None, None, None, None, None, None, None) == -1
+
+
+def test_workspace_size_and_check(fbk):
+    s = _shape(fbk)  # G*B = 64 rows, d = 128, b*Hkv = 2 units
+    c = _cache(fbk)
+    n = fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), ctypes.byref(c), 10)
+    slots = 10 + 2
+    assert n >= slots * 64 * 130 * 4
+    assert n < slots * 64 * 130 * 4 + 3 * 256
+    p = fbk.CPartial(0x40000, 0x50000, 0x60000)
+    st = fbk.lib.fbk_prefix_partial(ctypes.byref(s), ctypes.c_void_p(0x70000), ctypes.byref(c),
+                                    ctypes.byref(p), ctypes.c_void_p(0x80000), n - 1, 10, None)
+    assert st == -4
+    st = fbk.lib.fbk_prefix_partial(ctypes.byref(s), ctypes.c_void_p(0x70000), ctypes.byref(c),
+                                    ctypes.byref(p), None, n, 10, None)
+    assert st == -4
+    assert fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), ctypes.byref(c), -1) == 0
