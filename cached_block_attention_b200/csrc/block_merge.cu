@@ -11,44 +11,58 @@
 // query rows, i.e. FlashBlock's reuse of block-external attention with fresh
 // block-internal attention (FlashBlock, Abstract).
 //
-// One CTA per (unit, chunk of 4*RPW query rows); everything in fp32 on CUDA
-// cores (B <= 64 keys per row). Row max / sum are warp-shuffle reductions with
-// lane j holding keys j and j+32.
+// The step is latency-bound (a few MB), so the kernel is built around a single
+// DRAM round trip: every input of the CTA (block K and V of its kv-head, its
+// query rows, their prefix-state rows) is requested at once with cp.async,
+// the RoPE cos/sin table is computed while those copies fly, and everything
+// after that runs from shared memory in fp32 on CUDA cores (B <= 64 keys per
+// row). Row max and sum are warp-shuffle reductions, lane j holding keys j and
+// j + 32. One CTA per (unit, chunk of 4*RPW query rows).
 #include "launch.h"
 
 namespace fbk {
 namespace {
 
 constexpr int WARPS = 4;
+constexpr int THREADS = WARPS * 32;
 
-struct Layout {
-  int kp, k_off, v_off, q_off, p_off, cs_off, floats;
+struct Layout {  // byte offsets, all 16-byte aligned
+  int kraw, vraw, qraw, opart, ml, kf, qf, cs, ps, bytes, kp;
   __host__ __device__ Layout(int d, int blk, int rc) {
     kp = d + 4;
-    k_off = 0;
-    v_off = k_off + blk * kp;
-    q_off = v_off + blk * d;
-    p_off = q_off + rc * d;
-    cs_off = p_off + rc * 64;
-    cs_off = (cs_off + 1) & ~1;  // float2 alignment
-    floats = cs_off + 2 * blk * (d / 2);
+    kraw = 0;
+    vraw = kraw + blk * d * 2;
+    qraw = vraw + blk * d * 2;
+    opart = qraw + rc * d * 2;
+    ml = opart + rc * d * 4;
+    kf = ml + ((2 * rc * 4 + 15) & ~15);
+    qf = kf + blk * kp * 4;
+    cs = qf + rc * d * 4;
+    ps = cs + blk * (d / 2) * 8;
+    bytes = ps + rc * 64 * 4;
   }
 };
 
 template <int D, int RPW, bool F32OUT>
-__global__ void __launch_bounds__(WARPS * 32) block_merge_kernel(
+__global__ void __launch_bounds__(THREADS) block_merge_kernel(
     Geometry g, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kb,
     const __nv_bfloat16 *__restrict__ vb, fbk_partial pfx, void *__restrict__ out,
     float *__restrict__ lse) {
-  constexpr int RC = WARPS * RPW, CPL = D / 32, HALF = D / 2;
+  constexpr int RC = WARPS * RPW, CPL = D / 32, HALF = D / 2, CH = D / 8, CHF = D / 4;
   extern __shared__ float4 smem_f4[];
-  float *sm = reinterpret_cast<float *>(smem_f4);
-  const Layout lay(D, g.blk, RC);
-  float *Kf = sm + lay.k_off;
-  float *Vf = sm + lay.v_off;
-  float *Qf = sm + lay.q_off;
-  float *Ps = sm + lay.p_off;
-  float2 *cs = reinterpret_cast<float2 *>(sm + lay.cs_off);
+  uint8_t *sm = reinterpret_cast<uint8_t *>(smem_f4);
+  const int blk = g.blk;
+  const Layout lay(D, blk, RC);
+  __nv_bfloat16 *Kraw = reinterpret_cast<__nv_bfloat16 *>(sm + lay.kraw);
+  __nv_bfloat16 *Vraw = reinterpret_cast<__nv_bfloat16 *>(sm + lay.vraw);
+  __nv_bfloat16 *Qraw = reinterpret_cast<__nv_bfloat16 *>(sm + lay.qraw);
+  float *Opart = reinterpret_cast<float *>(sm + lay.opart);
+  float *Mpart = reinterpret_cast<float *>(sm + lay.ml);
+  float *Lpart = Mpart + RC;
+  float *Kf = reinterpret_cast<float *>(sm + lay.kf);
+  float *Qf = reinterpret_cast<float *>(sm + lay.qf);
+  float2 *cs = reinterpret_cast<float2 *>(sm + lay.cs);
+  float *Ps = reinterpret_cast<float *>(sm + lay.ps);
 
   const int u = blockIdx.y, b = u / g.hkv, kvh = u % g.hkv;
   const int r0 = blockIdx.x * RC;
@@ -58,46 +72,69 @@ __global__ void __launch_bounds__(WARPS * 32) block_merge_kernel(
     raise_flag(g, FBK_DEVERR_PREFIX_LEN);
     L = 0;
   }
-  const int blk = g.blk;
 
-  for (int idx = tid; idx < blk * HALF; idx += WARPS * 32)
-    cs[idx] = rope_cs_f32(L + idx / HALF, g.inv_freq_over_pi[idx % HALF]);
+  // ---- one round of asynchronous copies for everything this CTA reads
+  const long long kv_row0 = ((long long)b * blk) * g.hkv + kvh;  // row of token t: kv_row0 + t*hkv
+  for (int idx = tid; idx < blk * CH; idx += THREADS) {
+    const int t = idx / CH, c = idx % CH;
+    const long long src = (kv_row0 + (long long)t * g.hkv) * D + c * 8;
+    cp_async16(Kraw + t * D + c * 8, kb + src);
+    cp_async16(Vraw + t * D + c * 8, vb + src);
+  }
+  for (int idx = tid; idx < RC * CH; idx += THREADS) {
+    const int rr = idx / CH, c = idx % CH, r = r0 + rr;
+    if (r < g.rows) {
+      const int t = r % blk, h = kvh * g.group + r / blk;
+      cp_async16(Qraw + rr * D + c * 8, q + (((long long)b * blk + t) * g.hq + h) * D + c * 8);
+    }
+  }
+  for (int idx = tid; idx < RC * CHF; idx += THREADS) {
+    const int rr = idx / CHF, c = idx % CHF, r = r0 + rr;
+    if (r < g.rows) {
+      const int t = r % blk, h = kvh * g.group + r / blk;
+      cp_async16(Opart + rr * D + c * 4, pfx.o_unnorm + (((long long)b * g.hq + h) * blk + t) * D + c * 4);
+    }
+  }
+  for (int rr = tid; rr < RC; rr += THREADS) {
+    const int r = r0 + rr;
+    if (r < g.rows) {
+      const int t = r % blk, h = kvh * g.group + r / blk;
+      const long long prow = ((long long)b * g.hq + h) * blk + t;
+      cp_async4(Mpart + rr, pfx.m + prow);
+      cp_async4(Lpart + rr, pfx.l + prow);
+    }
+  }
+  // ---- RoPE table of positions L .. L+B-1 while the copies are in flight
+  for (int idx = tid; idx < blk * HALF; idx += THREADS)
+    cs[idx] = rope_cs_fast(L + idx / HALF, g.inv_freq_over_pi[idx % HALF]);
+  cp_async_wait_all();
   __syncthreads();
 
-  for (int idx = tid; idx < blk * HALF; idx += WARPS * 32) {
+  // ---- rotate block K and the CTA's query rows into fp32
+  for (int idx = tid; idx < blk * HALF; idx += THREADS) {
     const int t = idx / HALF, i = idx % HALF;
-    const __nv_bfloat16 *src = kb + (((long long)b * blk + t) * g.hkv + kvh) * D;
-    const float x1 = __bfloat162float(src[i]), x2 = __bfloat162float(src[i + HALF]);
+    const float x1 = __bfloat162float(Kraw[t * D + i]), x2 = __bfloat162float(Kraw[t * D + i + HALF]);
     const float2 c = cs[idx];
     Kf[t * lay.kp + i] = x1 * c.x - x2 * c.y;
     Kf[t * lay.kp + i + HALF] = x2 * c.x + x1 * c.y;
-    const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162 *>(
-        vb + (((long long)b * blk + t) * g.hkv + kvh) * D + 2 * i);
-    const float2 vf = __bfloat1622float2(v2);
-    Vf[t * D + 2 * i] = vf.x;
-    Vf[t * D + 2 * i + 1] = vf.y;
   }
-  for (int idx = tid; idx < RC * HALF; idx += WARPS * 32) {
+  for (int idx = tid; idx < RC * HALF; idx += THREADS) {
     const int rr = idx / HALF, i = idx % HALF, r = r0 + rr;
-    float y1 = 0.f, y2 = 0.f;
     if (r < g.rows) {
-      const int hl = r / blk, t = r % blk, h = kvh * g.group + hl;
-      const __nv_bfloat16 *src = q + (((long long)b * blk + t) * g.hq + h) * D;
-      const float x1 = __bfloat162float(src[i]), x2 = __bfloat162float(src[i + HALF]);
-      const float2 c = cs[t * HALF + i];
-      y1 = x1 * c.x - x2 * c.y;
-      y2 = x2 * c.x + x1 * c.y;
+      const float x1 = __bfloat162float(Qraw[rr * D + i]), x2 = __bfloat162float(Qraw[rr * D + i + HALF]);
+      const float2 c = cs[(r % blk) * HALF + i];
+      Qf[rr * D + i] = x1 * c.x - x2 * c.y;
+      Qf[rr * D + i + HALF] = x2 * c.x + x1 * c.y;
     }
-    Qf[rr * D + i] = y1;
-    Qf[rr * D + i + HALF] = y2;
   }
   __syncthreads();
 
+  // ---- per query row: block scores, softmax, P V, merge, normalise, store
 #pragma unroll 1
   for (int rr = 0; rr < RPW; ++rr) {
     const int rl = warp * RPW + rr, r = r0 + rl;
     if (r >= g.rows) break;
-    const int hl = r / blk, t = r % blk, h = kvh * g.group + hl;
+    const int t = r % blk, h = kvh * g.group + r / blk;
     const float *qrow = Qf + rl * D;
     const int j0 = lane < blk ? lane : 0, j1 = lane + 32 < blk ? lane + 32 : 0;
     float s0 = 0.f, s1 = 0.f;
@@ -105,9 +142,11 @@ __global__ void __launch_bounds__(WARPS * 32) block_merge_kernel(
     for (int k = 0; k < D; k += 4) {
       const float4 qv = *reinterpret_cast<const float4 *>(qrow + k);
       const float4 a = *reinterpret_cast<const float4 *>(Kf + j0 * lay.kp + k);
-      const float4 c = *reinterpret_cast<const float4 *>(Kf + j1 * lay.kp + k);
       s0 += qv.x * a.x + qv.y * a.y + qv.z * a.z + qv.w * a.w;
-      s1 += qv.x * c.x + qv.y * c.y + qv.z * c.z + qv.w * c.w;
+      if (blk > 32) {
+        const float4 c = *reinterpret_cast<const float4 *>(Kf + j1 * lay.kp + k);
+        s1 += qv.x * c.x + qv.y * c.y + qv.z * c.z + qv.w * c.w;
+      }
     }
     s0 = lane < blk ? s0 * g.tau : -CUDART_INF_F;
     s1 = lane + 32 < blk ? s1 * g.tau : -CUDART_INF_F;
@@ -120,18 +159,23 @@ __global__ void __launch_bounds__(WARPS * 32) block_merge_kernel(
     float ob[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) ob[c] = 0.f;
+#pragma unroll 4
     for (int j = 0; j < blk; ++j) {
       const float pj = Ps[rl * 64 + j];
+      const __nv_bfloat16 *vr = Vraw + j * D + lane * CPL;
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) ob[c] += pj * Vf[j * D + lane * CPL + c];
+      for (int c = 0; c < CPL; c += 2) {
+        const float2 v2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(vr + c));
+        ob[c] += pj * v2.x;
+        ob[c + 1] += pj * v2.y;
+      }
     }
-    const long long prow = ((long long)b * g.hq + h) * blk + t;
-    const float m1 = pfx.m[prow], l1 = pfx.l[prow];
-    const float *o1 = pfx.o_unnorm + prow * D + lane * CPL;
+    const float m1 = Mpart[rl], l1 = Lpart[rl];
     const float mm = fmaxf(m1, m2);
     const float w1 = lse_weight(m1, mm), w2 = expf(m2 - mm);
     const float lt = w1 * l1 + w2 * l2;
     const float inv = 1.f / lt;
+    const float *o1 = Opart + rl * D + lane * CPL;
     const long long orow = (((long long)b * blk + t) * g.hq + h) * D + lane * CPL;
     float res[CPL];
 #pragma unroll
@@ -146,7 +190,7 @@ __global__ void __launch_bounds__(WARPS * 32) block_merge_kernel(
       for (int c = 0; c < CPL; c += 2)
         *reinterpret_cast<__nv_bfloat162 *>(dst + c) = __floats2bfloat162_rn(res[c], res[c + 1]);
     }
-    if (lse && lane == 0) lse[prow] = mm + logf(lt);
+    if (lse && lane == 0) lse[((long long)b * g.hq + h) * blk + t] = mm + logf(lt);
     __syncwarp();
   }
 }
@@ -157,12 +201,13 @@ cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfl
                        cudaStream_t st) {
   constexpr int RC = WARPS * RPW;
   const Layout lay(D, g.blk, RC);
-  const size_t bytes = sizeof(float) * lay.floats;
   auto kern = block_merge_kernel<D, RPW, F32OUT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e != cudaSuccess) return e;
+  if (lay.bytes > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.bytes);
+    if (e != cudaSuccess) return e;
+  }
   dim3 grid((g.rows + RC - 1) / RC, g.batch * g.hkv);
-  kern<<<grid, WARPS * 32, bytes, st>>>(g, q, kb, vb, pfx, out, lse);
+  kern<<<grid, THREADS, lay.bytes, st>>>(g, q, kb, vb, pfx, out, lse);
   return cudaGetLastError();
 }
 
@@ -172,8 +217,7 @@ cudaError_t launch_d(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloa
                      cudaStream_t st) {
   // Few rows per CTA when there are few units, so the grid still covers the SMs.
   const long long units = (long long)g.batch * g.hkv;
-  if (units * ((g.rows + 7) / 8) <= 512)
-    return launch_cfg<D, 2, F32OUT>(g, q, kb, vb, pfx, out, lse, st);
+  if (units * ((g.rows + 7) / 8) <= 512) return launch_cfg<D, 2, F32OUT>(g, q, kb, vb, pfx, out, lse, st);
   return launch_cfg<D, 8, F32OUT>(g, q, kb, vb, pfx, out, lse, st);
 }
 

@@ -154,6 +154,15 @@ __device__ __forceinline__ float2 rope_cs_f32(int pos, double inv_freq_over_pi) 
   return make_float2(c, s);
 }
 
+// Same angle, fp64-reduced to [-pi, pi], then CUDA's fast __sincosf: absolute
+// error ~5e-7, for the per-step kernels where a full sincospi per element would
+// dominate the latency.
+__device__ __forceinline__ float2 rope_cs_fast(int pos, double inv_freq_over_pi) {
+  float s, c;
+  __sincosf((float)(rope_turns(pos, inv_freq_over_pi) * CUDART_PI), &s, &c);
+  return make_float2(c, s);
+}
+
 __device__ __forceinline__ void rope_cs_f64(int pos, double inv_freq_over_pi, double *c, double *s) {
   sincospi(rope_turns(pos, inv_freq_over_pi), s, c);
 }
@@ -196,6 +205,23 @@ __device__ __forceinline__ float warp_sum(float v) {
 // max is m; an empty state (m_part = -inf) contributes 0.
 __device__ __forceinline__ float lse_weight(float m_part, float m) {
   return m_part == -CUDART_INF_F ? 0.f : expf(m_part - m);
+}
+
+// Ampere-style asynchronous global -> shared copies (issued together, waited once).
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 // Workspace view of the per-share states written by the prefix kernels.

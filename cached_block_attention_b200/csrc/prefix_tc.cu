@@ -307,15 +307,15 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
         const uint32_t qbase = sb + C::Q_OFF + mt * C::Q_BYTES;
         const bool real = r < g.rows;
         const int hl = real ? r / g.blk : 0, t = real ? r % g.blk : 0;
-        const __nv_bfloat16 *src = q + (((long long)p.b * g.blk + t) * g.hq + p.kvh * g.group + hl) * D;
-#pragma unroll 1
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            q + (((long long)p.b * g.blk + t) * g.hq + p.kvh * g.group + hl) * D);
+        uint4 raw[D / 8];  // the whole bf16 row, requested before any use
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) raw[c] = real ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
         for (int c = 0; c < D / 16; ++c) {
-          uint4 a = make_uint4(0, 0, 0, 0), bq = make_uint4(0, 0, 0, 0);
-          if (real) {
-            a = *reinterpret_cast<const uint4 *>(src + 8 * c);
-            bq = *reinterpret_cast<const uint4 *>(src + D / 2 + 8 * c);
-          }
-          const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {bq.x, bq.y, bq.z, bq.w};
+          const uint32_t aw[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+          const uint32_t bw[4] = {raw[c + D / 16].x, raw[c + D / 16].y, raw[c + D / 16].z, raw[c + D / 16].w};
           uint32_t y1w[4], y2w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {

@@ -4,7 +4,10 @@
 // Each share's state is the recurrence of LaCache §3.3.3 (Eq. 2-6) over its
 // own run of tiles; by associativity of that recurrence, the state over all
 // tiles is the LSE merge m = max_c m_c, l = sum_c e^(m_c - m) l_c,
-// O~ = sum_c e^(m_c - m) O~_c. One warp per query row; lanes hold d/32 columns.
+// O~ = sum_c e^(m_c - m) O~_c. One warp per query row: lane j fetches m and l
+// of the j-th share of a batch of 32 (one round trip for all of them), the
+// weights are broadcast by shuffle, and the O~ rows are read with the loop
+// unrolled so that several loads are in flight at once.
 #include "launch.h"
 
 namespace fbk {
@@ -13,7 +16,7 @@ namespace {
 constexpr int WARPS = 8;
 
 template <int D>
-__global__ void __launch_bounds__(WARPS * 32) split_reduce_kernel(Geometry g, Workspace ws,
+__global__ void __launch_bounds__(WARPS * 32, 2) split_reduce_kernel(Geometry g, Workspace ws,
                                                                    int shares, fbk_partial out) {
   constexpr int CPL = D / 32;
   const int u = blockIdx.x, b = u / g.hkv, kvh = u % g.hkv;
@@ -38,21 +41,34 @@ __global__ void __launch_bounds__(WARPS * 32) split_reduce_kernel(Geometry g, Wo
   float M = -CUDART_INF_F, Lsum = 0.f;
   if (tb > 0) {
     const long long c_lo = share_of(A, T, shares), c_hi = share_of(E - 1, T, shares);
-    for (long long c = c_lo; c <= c_hi; ++c) {
-      const long long lo = max(share_begin(c, T, shares), A);
-      const long long hi = min(share_begin(c + 1, T, shares), E);
-      if (lo < hi) M = fmaxf(M, ws.m[(c + u) * g.rows + r]);
-    }
-    for (long long c = c_lo; c <= c_hi; ++c) {
-      const long long lo = max(share_begin(c, T, shares), A);
-      const long long hi = min(share_begin(c + 1, T, shares), E);
-      if (lo >= hi) continue;
-      const long long row = (c + u) * g.rows + r;
-      const float w = expf(ws.m[row] - M);
-      Lsum += w * ws.l[row];
-      const float *src = ws.o + row * D + lane * CPL;
+    const long long first_row = (c_lo + u) * g.rows + r;  // share c_lo always holds a piece of u
+    for (long long base = c_lo; base <= c_hi; base += 32) {
+      const long long c = base + lane;
+      bool valid = false;
+      if (c <= c_hi) {
+        const long long lo = max(share_begin(c, T, shares), A);
+        const long long hi = min(share_begin(c + 1, T, shares), E);
+        valid = lo < hi;
+      }
+      const long long row = valid ? (c + u) * g.rows + r : first_row;
+      const float mc = valid ? ws.m[row] : -CUDART_INF_F;
+      const float lc = valid ? ws.l[row] : 0.f;
+      const float Mn = fmaxf(M, warp_max(mc));
+      const float keep = lse_weight(M, Mn);
+      const float wc = valid ? expf(mc - Mn) : 0.f;
+      Lsum = Lsum * keep + warp_sum(wc * lc);
 #pragma unroll
-      for (int cc = 0; cc < CPL; ++cc) acc[cc] += w * src[cc];
+      for (int cc = 0; cc < CPL; ++cc) acc[cc] *= keep;
+      const int n = (int)min(32ll, c_hi - base + 1);
+#pragma unroll 4
+      for (int j = 0; j < n; ++j) {
+        const float w = __shfl_sync(0xffffffffu, wc, j);
+        const long long rj = __shfl_sync(0xffffffffu, row, j);
+        const float *src = ws.o + rj * D + lane * CPL;  // empty shares read share c_lo's row, weight 0
+#pragma unroll
+        for (int cc = 0; cc < CPL; ++cc) acc[cc] += w * src[cc];
+      }
+      M = Mn;
     }
   }
   float *dst = out.o_unnorm + orow * D + lane * CPL;

@@ -44,7 +44,11 @@ def rel_l2(got, ref) -> float:
     return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))
 
 
-def assert_close(got, ref, mode, what=""):
+def assert_close(got, ref, mode, what="", f32_scale=1.0):
+    """f32_scale widens the fp32 check-mode bounds for inputs whose logits are
+    far from the workloads' O(0.1): fp32 rounding of a score s perturbs the
+    softmax weights by about |s| * 2^-24 * sqrt(d), so the bound grows with
+    the largest |logit| (tests pass that as f32_scale)."""
     got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
@@ -55,8 +59,8 @@ def assert_close(got, ref, mode, what=""):
         assert err.mean() <= BF16_MEAN_ABS, f"{what}: mean abs {err.mean():.3e}"
         assert r <= BF16_REL, f"{what}: rel l2 {r:.3e}"
     else:
-        assert err.max() <= F32_MAX_ABS, f"{what}: max abs {err.max():.3e}"
-        assert r <= F32_REL, f"{what}: rel l2 {r:.3e}"
+        assert err.max() <= F32_MAX_ABS * f32_scale, f"{what}: max abs {err.max():.3e}"
+        assert r <= F32_REL * f32_scale, f"{what}: rel l2 {r:.3e}"
     return float(err.max()), r
 
 
@@ -194,7 +198,7 @@ def partial_to_host(p):
     return host_f64(p.o_unnorm), host_f64(p.m), host_f64(p.l)
 
 
-def check_partial(got, ref, mode, what="partial", rows=None):
+def check_partial(got, ref, mode, what="partial", rows=None, f32_scale=1.0):
     """Compare two states through what is unique about them: the normalised
     output O~/l and the logsumexp m + log l, plus m itself; empty rows must be
     (0, -inf, 0) exactly."""
@@ -208,8 +212,8 @@ def check_partial(got, ref, mode, what="partial", rows=None):
         return
     gn = go[full] / gl[full][:, None]
     rn = ro[full] / rl[full][:, None]
-    assert_close(gn, rn, mode, what + " O~/l")
-    lse_tol = 2e-2 if mode == "bf16" else 1e-5
+    assert_close(gn, rn, mode, what + " O~/l", f32_scale)
+    lse_tol = 2e-2 if mode == "bf16" else 1e-5 * f32_scale
     assert np.abs((gm[full] + np.log(gl[full])) - (rm[full] + np.log(rl[full]))).max() <= lse_tol, \
         f"{what}: lse"
     assert np.abs(gm[full] - rm[full]).max() <= lse_tol + (1e-2 if mode == "bf16" else 1e-6) * np.abs(rm[full]).max(), \
