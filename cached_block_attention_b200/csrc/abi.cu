@@ -16,7 +16,8 @@ fbk_status check_shape(const fbk_shape *s) {
   if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_heads < 1 || s->block_len < 1 || s->head_dim < 1)
     return FBK_ERR_INVALID_ARG;
   if (s->mode != FBK_BF16 && s->mode != FBK_FP32_CHECK) return FBK_ERR_INVALID_ARG;
-  if (!isfinite(s->softmax_scale) || !isfinite(s->rope_base) || !(s->rope_base > 0.0))
+  if (!isfinite(s->softmax_scale) || !(s->softmax_scale > 0.f) || !isfinite(s->rope_base) ||
+      !(s->rope_base > 0.0))
     return FBK_ERR_INVALID_ARG;
   if (s->head_dim != 64 && s->head_dim != 128) return FBK_ERR_UNSUPPORTED;
   if (s->n_q_heads % s->n_kv_heads != 0) return FBK_ERR_UNSUPPORTED;
@@ -55,6 +56,7 @@ Geometry make_geometry(const fbk_shape *s, const fbk_kv_cache *c) {
   g.blk = s->block_len;
   g.rows = g.group * g.blk;
   g.tau = s->softmax_scale;
+  g.log2_base = log2(s->rope_base);
   for (int i = 0; i < g.d / 2; ++i)
     g.inv_freq_over_pi[i] = pow(s->rope_base, -2.0 * i / g.d) / M_PI;
   if (c) {

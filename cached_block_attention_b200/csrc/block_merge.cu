@@ -11,17 +11,279 @@
 // query rows, i.e. FlashBlock's reuse of block-external attention with fresh
 // block-internal attention (FlashBlock, Abstract).
 //
-// The step is latency-bound (a few MB), so the kernel is built around a single
-// DRAM round trip: every input of the CTA (block K and V of its kv-head, its
-// query rows, their prefix-state rows) is requested at once with cp.async,
-// the RoPE cos/sin table is computed while those copies fly, and everything
-// after that runs from shared memory in fp32 on CUDA cores (B <= 64 keys per
-// row). Row max and sum are warp-shuffle reductions, lane j holding keys j and
-// j + 32. One CTA per (unit, chunk of 4*RPW query rows).
+// The step moves a few MB and is latency-bound, so both variants are built
+// around one DRAM round trip: every input of the CTA is requested up front
+// (cp.async for block K/V and query rows, register loads for the prefix
+// state), the RoPE cos/sin table is computed while those requests fly, and
+// the rest runs from shared memory and registers.
+//  * FBK_BF16: a CTA holds one (sequence, kv-head) unit, up to 128 query rows
+//    (all G heads of the group share the staged K/V), and each warp owns 16
+//    rows: S = Q^ K^T and O = P~ V are warp-level bf16 tensor-core MMAs
+//    (mma.sync m16n8k16, fp32 accumulation; at 16 x B x d per warp these
+//    products are far too small for the TMEM/tcgen05 machinery to pay off),
+//    the softmax runs on the accumulator fragments with quad shuffles, and P~
+//    is re-packed in registers as the A operand of the second MMA.
+//  * FBK_FP32_CHECK: the same steps on CUDA cores in fp32 (no bf16 rounding of
+//    Q^, K^ or P~): lane j scores keys j and j + 32, warp-shuffle row max/sum.
 #include "launch.h"
 
 namespace fbk {
 namespace {
+
+// ====================================================================== bf16 (tensor cores)
+
+constexpr int MMA_MAX_ROWS = 128;  // query rows per CTA (8 warps x 16)
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                          uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+template <int D>
+struct MmaLayout {  // byte offsets in shared memory
+  static constexpr int RS = D * 2 + 16;  // padded bf16 row: ldmatrix rows hit distinct banks
+  int ks, vs, qs, cs, bytes;
+  __host__ __device__ MmaLayout(int blk) {
+    const int bpad = (blk + 15) & ~15;
+    ks = 0;
+    vs = ks + bpad * RS;
+    qs = vs + bpad * RS;
+    cs = qs + MMA_MAX_ROWS * RS;
+    bytes = cs + blk * (D / 2) * 8;
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) block_merge_mma_kernel(
+    Geometry g, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kb,
+    const __nv_bfloat16 *__restrict__ vb, fbk_partial pfx, __nv_bfloat16 *__restrict__ out,
+    float *__restrict__ lse) {
+  constexpr int HALF = D / 2, CH = D / 8, NTO = D / 8, RS = MmaLayout<D>::RS;
+  extern __shared__ float4 smem_f4[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>(smem_f4);
+  const int blk = g.blk, bpad = (blk + 15) & ~15;
+  const MmaLayout<D> lay(blk);
+  uint8_t *Ks = sm + lay.ks, *Vs = sm + lay.vs, *Qs = sm + lay.qs;
+  float2 *cs = reinterpret_cast<float2 *>(sm + lay.cs);
+
+  const int u = blockIdx.y, b = u / g.hkv, kvh = u % g.hkv;
+  const int r0 = blockIdx.x * MMA_MAX_ROWS;
+  const int rows_cta = min(MMA_MAX_ROWS, g.rows - r0);
+  const int nthreads = blockDim.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int L = g.lens[b];
+  if (L < 0) {
+    raise_flag(g, FBK_DEVERR_PREFIX_LEN);
+    L = 0;
+  }
+
+  // ---- 1. every global read of the CTA, issued at once
+  const long long kv_row0 = (long long)b * blk * g.hkv + kvh;  // token t: row kv_row0 + t*hkv
+  for (int idx = tid; idx < blk * CH; idx += nthreads) {
+    const int t = idx / CH, c = idx % CH;
+    const long long src = (kv_row0 + (long long)t * g.hkv) * D + c * 8;
+    cp_async16(Ks + t * RS + c * 16, kb + src);
+    cp_async16(Vs + t * RS + c * 16, vb + src);
+  }
+  for (int idx = tid; idx < rows_cta * CH; idx += nthreads) {
+    const int rr = idx / CH, c = idx % CH, r = r0 + rr;
+    const int t = r % blk, h = kvh * g.group + r / blk;
+    cp_async16(Qs + rr * RS + c * 16, q + (((long long)b * blk + t) * g.hq + h) * D + c * 8);
+  }
+  // padding key rows must be finite zeros (they meet P~ = 0 in the PV product)
+  for (int idx = tid; idx < (bpad - blk) * CH; idx += nthreads) {
+    const int t = blk + idx / CH, c = idx % CH;
+    *reinterpret_cast<uint4 *>(Ks + t * RS + c * 16) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4 *>(Vs + t * RS + c * 16) = make_uint4(0, 0, 0, 0);
+  }
+  const int nw_rows = (rows_cta + 15) / 16;
+  for (int idx = tid; idx < (nw_rows * 16 - rows_cta) * CH; idx += nthreads) {
+    const int rr = rows_cta + idx / CH, c = idx % CH;
+    *reinterpret_cast<uint4 *>(Qs + rr * RS + c * 16) = make_uint4(0, 0, 0, 0);
+  }
+  // this thread's two accumulator rows and their prefix state (registers)
+  const int lr = lane >> 2, lc = (lane & 3) * 2;
+  const int ra = r0 + warp * 16 + lr, rb = ra + 8;
+  const bool va = warp < nw_rows && ra < g.rows, vbr = warp < nw_rows && rb < g.rows;
+  const int ta = va ? ra % blk : 0, ha = va ? kvh * g.group + ra / blk : 0;
+  const int tb_ = vbr ? rb % blk : 0, hb = vbr ? kvh * g.group + rb / blk : 0;
+  const long long pa = ((long long)b * g.hq + ha) * blk + ta, pb = ((long long)b * g.hq + hb) * blk + tb_;
+  float2 o1a[NTO], o1b[NTO];
+  float m1a = -CUDART_INF_F, l1a = 0.f, m1b = -CUDART_INF_F, l1b = 0.f;
+#pragma unroll
+  for (int j = 0; j < NTO; ++j) {
+    o1a[j] = va ? __ldg(reinterpret_cast<const float2 *>(pfx.o_unnorm + pa * D + 8 * j + lc)) : make_float2(0.f, 0.f);
+    o1b[j] = vbr ? __ldg(reinterpret_cast<const float2 *>(pfx.o_unnorm + pb * D + 8 * j + lc)) : make_float2(0.f, 0.f);
+  }
+  if (va) { m1a = __ldg(pfx.m + pa); l1a = __ldg(pfx.l + pa); }
+  if (vbr) { m1b = __ldg(pfx.m + pb); l1b = __ldg(pfx.l + pb); }
+
+  // ---- 2. RoPE cos/sin of positions L .. L+B-1 (thread count is a multiple of d/2)
+  {
+    const int i = tid % HALF;
+    const double f = freq_over_pi(i, D, g.log2_base);
+    for (int t = tid / HALF; t < blk; t += nthreads / HALF) cs[t * HALF + i] = rope_cs_fast(L + t, f);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+
+  // ---- 3. rotate block K and the query rows in place (bf16)
+  for (int idx = tid; idx < (blk + rows_cta) * HALF; idx += nthreads) {
+    const int rowi = idx / HALF, i = idx % HALF;
+    const bool is_k = rowi < blk;
+    const int t = is_k ? rowi : (r0 + rowi - blk) % blk;
+    __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(is_k ? Ks + rowi * RS : Qs + (rowi - blk) * RS);
+    const float x1 = __bfloat162float(row[i]), x2 = __bfloat162float(row[i + HALF]);
+    const float2 c = cs[t * HALF + i];
+    row[i] = __float2bfloat16_rn(x1 * c.x - x2 * c.y);
+    row[i + HALF] = __float2bfloat16_rn(x2 * c.x + x1 * c.y);
+  }
+  __syncthreads();
+  if (warp >= nw_rows) return;
+
+  // ---- 4. S = Q^ K^T for this warp's 16 rows (up to 64 keys: 8 n-tiles)
+  const uint32_t qs_a = (uint32_t)__cvta_generic_to_shared(Qs), ks_a = (uint32_t)__cvta_generic_to_shared(Ks),
+                 vs_a = (uint32_t)__cvta_generic_to_shared(Vs);
+  float sacc[8][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+  const int a_row = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1), a_col = 8 * (lane >> 4);
+  const int b_row = (lane & 7) + 8 * (lane >> 4), b_col = 8 * ((lane >> 3) & 1);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4(qs_a + a_row * RS + (16 * kk + a_col) * 2, a0, a1, a2, a3);
+#pragma unroll
+    for (int jp = 0; jp < 4; ++jp) {
+      if (16 * jp < bpad) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(ks_a + (16 * jp + b_row) * RS + (16 * kk + b_col) * 2, b0, b1, b2, b3);
+        mma16816(sacc[2 * jp], a0, a1, a2, a3, b0, b1);
+        mma16816(sacc[2 * jp + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+  }
+
+  // ---- 5. block softmax on the fragments (rows lr and lr + 8 of the warp tile)
+  const float sl2 = g.tau * 1.4426950408889634f;
+  float mxa = -CUDART_INF_F, mxb = -CUDART_INF_F;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const bool ok = 8 * j + lc + e < blk;
+      sacc[j][e] = ok ? sacc[j][e] * sl2 : -CUDART_INF_F;
+      sacc[j][2 + e] = ok ? sacc[j][2 + e] * sl2 : -CUDART_INF_F;
+      mxa = fmaxf(mxa, sacc[j][e]);
+      mxb = fmaxf(mxb, sacc[j][2 + e]);
+    }
+  }
+  mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
+  mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
+  mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
+  mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
+  float sa = 0.f, sbs = 0.f;
+  uint32_t pa_frag[8], pb_frag[8];  // P~ as bf16 pairs: [n-tile] for rows lr and lr + 8
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float p0 = exp2f(sacc[j][0] - mxa), p1 = exp2f(sacc[j][1] - mxa);
+    const float p2 = exp2f(sacc[j][2] - mxb), p3 = exp2f(sacc[j][3] - mxb);
+    sa += p0 + p1;
+    sbs += p2 + p3;
+    pa_frag[j] = pack2(p0, p1);
+    pb_frag[j] = pack2(p2, p3);
+  }
+  sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+  sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+  sbs += __shfl_xor_sync(0xffffffffu, sbs, 1);
+  sbs += __shfl_xor_sync(0xffffffffu, sbs, 2);
+
+  // ---- 6. O~2 = P~ V
+  float oacc[NTO][4];
+#pragma unroll
+  for (int j = 0; j < NTO; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
+  const int v_row = (lane & 7) + 8 * ((lane >> 3) & 1), v_col = 8 * (lane >> 4);
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    if (16 * kk < bpad) {
+      const uint32_t a0 = pa_frag[2 * kk], a1 = pb_frag[2 * kk], a2 = pa_frag[2 * kk + 1], a3 = pb_frag[2 * kk + 1];
+#pragma unroll
+      for (int jp = 0; jp < D / 16; ++jp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vs_a + (16 * kk + v_row) * RS + (16 * jp + v_col) * 2, b0, b1, b2, b3);
+        mma16816(oacc[2 * jp], a0, a1, a2, a3, b0, b1);
+        mma16816(oacc[2 * jp + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+  }
+
+  // ---- 7. merge with the prefix state, normalise, store
+  const float LN2 = 0.6931471805599453f;
+  const float m2a = mxa * LN2, m2b = mxb * LN2;
+  const float Ma = fmaxf(m1a, m2a), Mb = fmaxf(m1b, m2b);
+  const float w1a = lse_weight(m1a, Ma), w2a = expf(m2a - Ma);
+  const float w1b = lse_weight(m1b, Mb), w2b = expf(m2b - Mb);
+  const float lta = w1a * l1a + w2a * sa, ltb = w1b * l1b + w2b * sbs;
+  const float ia = 1.f / lta, ib = 1.f / ltb;
+  __nv_bfloat16 *da = out + (((long long)b * blk + ta) * g.hq + ha) * D + lc;
+  __nv_bfloat16 *db = out + (((long long)b * blk + tb_) * g.hq + hb) * D + lc;
+#pragma unroll
+  for (int j = 0; j < NTO; ++j) {
+    if (va)
+      *reinterpret_cast<uint32_t *>(da + 8 * j) = pack2((w1a * o1a[j].x + w2a * oacc[j][0]) * ia,
+                                                        (w1a * o1a[j].y + w2a * oacc[j][1]) * ia);
+    if (vbr)
+      *reinterpret_cast<uint32_t *>(db + 8 * j) = pack2((w1b * o1b[j].x + w2b * oacc[j][2]) * ib,
+                                                        (w1b * o1b[j].y + w2b * oacc[j][3]) * ib);
+  }
+  if (lse && (lane & 3) == 0) {
+    if (va) lse[pa] = Ma + logf(lta);
+    if (vbr) lse[pb] = Mb + logf(ltb);
+  }
+}
+
+template <int D>
+cudaError_t launch_mma(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
+                       const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
+                       cudaStream_t st) {
+  const MmaLayout<D> lay(g.blk);
+  auto kern = block_merge_mma_kernel<D>;
+  if (lay.bytes > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.bytes);
+    if (e != cudaSuccess) return e;
+  }
+  const int rows_cta = g.rows < MMA_MAX_ROWS ? g.rows : MMA_MAX_ROWS;
+  int warps = (rows_cta + 15) / 16;
+  if (warps * 32 % (D / 2)) ++warps;  // the RoPE table loop needs a multiple of d/2 threads
+  dim3 grid((g.rows + MMA_MAX_ROWS - 1) / MMA_MAX_ROWS, g.batch * g.hkv);
+  kern<<<grid, warps * 32, lay.bytes, st>>>(g, q, kb, vb, pfx, static_cast<__nv_bfloat16 *>(out), lse);
+  return cudaGetLastError();
+}
+
+// ====================================================================== fp32 check (CUDA cores)
 
 constexpr int WARPS = 4;
 constexpr int THREADS = WARPS * 32;
@@ -43,10 +305,10 @@ struct Layout {  // byte offsets, all 16-byte aligned
   }
 };
 
-template <int D, int RPW, bool F32OUT>
-__global__ void __launch_bounds__(THREADS) block_merge_kernel(
+template <int D, int RPW>
+__global__ void __launch_bounds__(THREADS) block_merge_f32_kernel(
     Geometry g, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kb,
-    const __nv_bfloat16 *__restrict__ vb, fbk_partial pfx, void *__restrict__ out,
+    const __nv_bfloat16 *__restrict__ vb, fbk_partial pfx, float *__restrict__ out,
     float *__restrict__ lse) {
   constexpr int RC = WARPS * RPW, CPL = D / 32, HALF = D / 2, CH = D / 8, CHF = D / 4;
   extern __shared__ float4 smem_f4[];
@@ -73,8 +335,7 @@ __global__ void __launch_bounds__(THREADS) block_merge_kernel(
     L = 0;
   }
 
-  // ---- one round of asynchronous copies for everything this CTA reads
-  const long long kv_row0 = ((long long)b * blk) * g.hkv + kvh;  // row of token t: kv_row0 + t*hkv
+  const long long kv_row0 = ((long long)b * blk) * g.hkv + kvh;
   for (int idx = tid; idx < blk * CH; idx += THREADS) {
     const int t = idx / CH, c = idx % CH;
     const long long src = (kv_row0 + (long long)t * g.hkv) * D + c * 8;
@@ -104,13 +365,14 @@ __global__ void __launch_bounds__(THREADS) block_merge_kernel(
       cp_async4(Lpart + rr, pfx.l + prow);
     }
   }
-  // ---- RoPE table of positions L .. L+B-1 while the copies are in flight
-  for (int idx = tid; idx < blk * HALF; idx += THREADS)
-    cs[idx] = rope_cs_fast(L + idx / HALF, g.inv_freq_over_pi[idx % HALF]);
+  {  // RoPE table, accurate sincospi (check mode); each thread keeps one frequency
+    const int i = tid % HALF;
+    const double f = freq_over_pi(i, D, g.log2_base);
+    for (int t = tid / HALF; t < blk; t += THREADS / HALF) cs[t * HALF + i] = rope_cs_f32(L + t, f);
+  }
   cp_async_wait_all();
   __syncthreads();
 
-  // ---- rotate block K and the CTA's query rows into fp32
   for (int idx = tid; idx < blk * HALF; idx += THREADS) {
     const int t = idx / HALF, i = idx % HALF;
     const float x1 = __bfloat162float(Kraw[t * D + i]), x2 = __bfloat162float(Kraw[t * D + i + HALF]);
@@ -129,7 +391,6 @@ __global__ void __launch_bounds__(THREADS) block_merge_kernel(
   }
   __syncthreads();
 
-  // ---- per query row: block scores, softmax, P V, merge, normalise, store
 #pragma unroll 1
   for (int rr = 0; rr < RPW; ++rr) {
     const int rl = warp * RPW + rr, r = r0 + rl;
@@ -142,11 +403,9 @@ __global__ void __launch_bounds__(THREADS) block_merge_kernel(
     for (int k = 0; k < D; k += 4) {
       const float4 qv = *reinterpret_cast<const float4 *>(qrow + k);
       const float4 a = *reinterpret_cast<const float4 *>(Kf + j0 * lay.kp + k);
+      const float4 c = *reinterpret_cast<const float4 *>(Kf + j1 * lay.kp + k);
       s0 += qv.x * a.x + qv.y * a.y + qv.z * a.z + qv.w * a.w;
-      if (blk > 32) {
-        const float4 c = *reinterpret_cast<const float4 *>(Kf + j1 * lay.kp + k);
-        s1 += qv.x * c.x + qv.y * c.y + qv.z * c.z + qv.w * c.w;
-      }
+      s1 += qv.x * c.x + qv.y * c.y + qv.z * c.z + qv.w * c.w;
     }
     s0 = lane < blk ? s0 * g.tau : -CUDART_INF_F;
     s1 = lane + 32 < blk ? s1 * g.tau : -CUDART_INF_F;
@@ -176,49 +435,37 @@ __global__ void __launch_bounds__(THREADS) block_merge_kernel(
     const float lt = w1 * l1 + w2 * l2;
     const float inv = 1.f / lt;
     const float *o1 = Opart + rl * D + lane * CPL;
-    const long long orow = (((long long)b * blk + t) * g.hq + h) * D + lane * CPL;
-    float res[CPL];
+    float *dst = out + (((long long)b * blk + t) * g.hq + h) * D + lane * CPL;
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) res[c] = (w1 * o1[c] + w2 * ob[c]) * inv;
-    if (F32OUT) {
-      float *dst = reinterpret_cast<float *>(out) + orow;
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) dst[c] = res[c];
-    } else {
-      __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(out) + orow;
-#pragma unroll
-      for (int c = 0; c < CPL; c += 2)
-        *reinterpret_cast<__nv_bfloat162 *>(dst + c) = __floats2bfloat162_rn(res[c], res[c + 1]);
-    }
+    for (int c = 0; c < CPL; ++c) dst[c] = (w1 * o1[c] + w2 * ob[c]) * inv;
     if (lse && lane == 0) lse[((long long)b * g.hq + h) * blk + t] = mm + logf(lt);
     __syncwarp();
   }
 }
 
-template <int D, int RPW, bool F32OUT>
-cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
-                       const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
-                       cudaStream_t st) {
+template <int D, int RPW>
+cudaError_t launch_f32_cfg(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
+                           const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
+                           cudaStream_t st) {
   constexpr int RC = WARPS * RPW;
   const Layout lay(D, g.blk, RC);
-  auto kern = block_merge_kernel<D, RPW, F32OUT>;
+  auto kern = block_merge_f32_kernel<D, RPW>;
   if (lay.bytes > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.bytes);
     if (e != cudaSuccess) return e;
   }
   dim3 grid((g.rows + RC - 1) / RC, g.batch * g.hkv);
-  kern<<<grid, THREADS, lay.bytes, st>>>(g, q, kb, vb, pfx, out, lse);
+  kern<<<grid, THREADS, lay.bytes, st>>>(g, q, kb, vb, pfx, static_cast<float *>(out), lse);
   return cudaGetLastError();
 }
 
-template <int D, bool F32OUT>
-cudaError_t launch_d(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
-                     const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
-                     cudaStream_t st) {
-  // Few rows per CTA when there are few units, so the grid still covers the SMs.
+template <int D>
+cudaError_t launch_f32(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
+                       const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
+                       cudaStream_t st) {
   const long long units = (long long)g.batch * g.hkv;
-  if (units * ((g.rows + 7) / 8) <= 512) return launch_cfg<D, 2, F32OUT>(g, q, kb, vb, pfx, out, lse, st);
-  return launch_cfg<D, 8, F32OUT>(g, q, kb, vb, pfx, out, lse, st);
+  if (units * ((g.rows + 7) / 8) <= 512) return launch_f32_cfg<D, 2>(g, q, kb, vb, pfx, out, lse, st);
+  return launch_f32_cfg<D, 8>(g, q, kb, vb, pfx, out, lse, st);
 }
 
 }  // namespace
@@ -227,11 +474,11 @@ cudaError_t launch_block_merge(const Geometry &g, const __nv_bfloat16 *q,
                                const __nv_bfloat16 *kb, const __nv_bfloat16 *vb,
                                const fbk_partial &pfx, void *out, float *lse, bool f32_out,
                                cudaStream_t st) {
-  if (g.d == 128)
-    return f32_out ? launch_d<128, true>(g, q, kb, vb, pfx, out, lse, st)
-                   : launch_d<128, false>(g, q, kb, vb, pfx, out, lse, st);
-  return f32_out ? launch_d<64, true>(g, q, kb, vb, pfx, out, lse, st)
-                 : launch_d<64, false>(g, q, kb, vb, pfx, out, lse, st);
+  if (f32_out)
+    return g.d == 128 ? launch_f32<128>(g, q, kb, vb, pfx, out, lse, st)
+                      : launch_f32<64>(g, q, kb, vb, pfx, out, lse, st);
+  return g.d == 128 ? launch_mma<128>(g, q, kb, vb, pfx, out, lse, st)
+                    : launch_mma<64>(g, q, kb, vb, pfx, out, lse, st);
 }
 
 }  // namespace fbk

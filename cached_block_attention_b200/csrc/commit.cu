@@ -59,24 +59,72 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(THREADS)
   }
   __syncthreads();
 
-  for (int idx = threadIdx.x; idx < nt * g.hkv * HALF; idx += THREADS) {
-    const int i = idx % HALF, rowi = idx / HALF, kvh = rowi % g.hkv, tl = rowi / g.hkv, t = t0 + tl;
-    const __nv_bfloat16 *src = kb + (((long long)b * blk + t) * g.hkv + kvh) * D;
-    const double x1 = (double)__bfloat162float(src[i]);
-    const double x2 = (double)__bfloat162float(src[i + HALF]);
-    const double2 cs = tab[tl * HALF + i];
-    // plain rounded products and differences (no fused multiply-add)
-    const double y1 = __dsub_rn(__dmul_rn(x1, cs.x), __dmul_rn(x2, cs.y));
-    const double y2 = __dadd_rn(__dmul_rn(x2, cs.x), __dmul_rn(x1, cs.y));
-    const long long row = cache_row(g, b, kvh, (long long)L + t);
-    kc[row * D + i] = __ushort_as_bfloat16(f64_to_bf16_rne(y1));
-    kc[row * D + i + HALF] = __ushort_as_bfloat16(f64_to_bf16_rne(y2));
+  // K: an item is 8 rotation pairs, i.e. the 16-byte chunk c of each half of a
+  // row; every load of a batch is issued before the first use.
+  const int nk = nt * g.hkv * (D / 16);
+  for (int base = 0; base < nk; base += THREADS * 4) {
+    uint4 xa[4], xb[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int item = base + threadIdx.x + THREADS * k;
+      if (item < nk) {
+        const int c = item % (D / 16), rowi = item / (D / 16), kvh = rowi % g.hkv, t = t0 + rowi / g.hkv;
+        const uint4 *src = reinterpret_cast<const uint4 *>(kb + (((long long)b * blk + t) * g.hkv + kvh) * D);
+        xa[k] = src[c];
+        xb[k] = src[c + D / 16];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int item = base + threadIdx.x + THREADS * k;
+      if (item < nk) {
+        const int c = item % (D / 16), rowi = item / (D / 16), kvh = rowi % g.hkv, tl = rowi / g.hkv;
+        const uint32_t aw[4] = {xa[k].x, xa[k].y, xa[k].z, xa[k].w};
+        const uint32_t bw[4] = {xb[k].x, xb[k].y, xb[k].z, xb[k].w};
+        uint32_t y1[4], y2[4];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t ha = (e & 1) ? (aw[e >> 1] >> 16) : (aw[e >> 1] & 0xffffu);
+          const uint32_t hb = (e & 1) ? (bw[e >> 1] >> 16) : (bw[e >> 1] & 0xffffu);
+          const double x1 = (double)bf16_bits_to_f32((uint16_t)ha), x2 = (double)bf16_bits_to_f32((uint16_t)hb);
+          const double2 cs = tab[tl * HALF + 8 * c + e];
+          // plain rounded products and differences (no fused multiply-add)
+          const uint32_t r1 = f64_to_bf16_rne(__dsub_rn(__dmul_rn(x1, cs.x), __dmul_rn(x2, cs.y)));
+          const uint32_t r2 = f64_to_bf16_rne(__dadd_rn(__dmul_rn(x2, cs.x), __dmul_rn(x1, cs.y)));
+          if (e & 1) {
+            y1[e >> 1] |= r1 << 16;
+            y2[e >> 1] |= r2 << 16;
+          } else {
+            y1[e >> 1] = r1;
+            y2[e >> 1] = r2;
+          }
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(kc + cache_row(g, b, kvh, (long long)L + t0 + tl) * D);
+        dst[c] = make_uint4(y1[0], y1[1], y1[2], y1[3]);
+        dst[c + D / 16] = make_uint4(y2[0], y2[1], y2[2], y2[3]);
+      }
+    }
   }
-  for (int idx = threadIdx.x; idx < nt * g.hkv * (D / 8); idx += THREADS) {
-    const int ch = idx % (D / 8), rowi = idx / (D / 8), kvh = rowi % g.hkv, t = t0 + rowi / g.hkv;
-    const long long row = cache_row(g, b, kvh, (long long)L + t);
-    *reinterpret_cast<uint4 *>(vc + row * D + ch * 8) =
-        *reinterpret_cast<const uint4 *>(vb + (((long long)b * blk + t) * g.hkv + kvh) * D + ch * 8);
+  // V: bit-exact 16-byte copies, 8 loads in flight per thread
+  const int nv = nt * g.hkv * (D / 8);
+  for (int base = 0; base < nv; base += THREADS * 8) {
+    uint4 x[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int item = base + threadIdx.x + THREADS * k;
+      if (item < nv) {
+        const int ch = item % (D / 8), rowi = item / (D / 8), kvh = rowi % g.hkv, t = t0 + rowi / g.hkv;
+        x[k] = reinterpret_cast<const uint4 *>(vb + (((long long)b * blk + t) * g.hkv + kvh) * D)[ch];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int item = base + threadIdx.x + THREADS * k;
+      if (item < nv) {
+        const int ch = item % (D / 8), rowi = item / (D / 8), kvh = rowi % g.hkv, t = t0 + rowi / g.hkv;
+        reinterpret_cast<uint4 *>(vc + cache_row(g, b, kvh, (long long)L + t) * D)[ch] = x[k];
+      }
+    }
   }
 }
 

@@ -22,7 +22,8 @@ constexpr int KV_TILE = 64;
 struct Geometry {
   int batch, hq, hkv, group, d, blk, rows;  // rows = group * blk (query rows per kv-head)
   float tau;                                // softmax scale
-  double inv_freq_over_pi[64];              // base^(-2i/d) / pi, i < d/2
+  double log2_base;                         // log2(rope base)
+  double inv_freq_over_pi[64];              // base^(-2i/d) / pi, i < d/2 (host pow())
   // cache
   const __nv_bfloat16 *kc, *vc;
   int paged, page_size, page_shift, max_pages;
@@ -143,6 +144,14 @@ __device__ __forceinline__ long long cache_row(const Geometry &g, int b, int kvh
 // formed in fp64 as a multiple of pi, reduced to [-1, 1] exactly in fp64, and
 // only then handed to CUDA's sincospi, so positions near 1.3e5 keep full
 // fp32 accuracy.
+// theta_i / pi computed in registers (no divergent parameter-space reads):
+// exp2(-(2i/d) log2(base)) in fp64, relative error ~2e-15, i.e. < 3e-10 rad at
+// position 1.3e5. The commit kernel, whose rounded output is compared bit for
+// bit, reads the host-computed pow() table instead.
+__device__ __forceinline__ double freq_over_pi(int i, int d, double log2_base) {
+  return exp2(-2.0 * i / d * log2_base) * (1.0 / CUDART_PI);
+}
+
 __device__ __forceinline__ double rope_turns(int pos, double inv_freq_over_pi) {
   double t = (double)pos * inv_freq_over_pi;
   return t - 2.0 * rint(0.5 * t);

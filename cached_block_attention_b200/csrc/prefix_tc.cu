@@ -59,10 +59,8 @@ struct Cfg {
   static constexpr int B_OFREE = B_ODONE + MT;
   static constexpr int B_DRAIN = B_OFREE + MT;
   static constexpr int NBAR = B_DRAIN + 1;
-  // per softmax warp: cos/sin(L theta_i) (float2) and theta_i (float), i < D/2
-  static constexpr int CS_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int TH_OFF = CS_OFF + 4 * MT * (D / 2) * 8;
-  static constexpr int MISC_OFF = TH_OFF + 4 * MT * (D / 2) * 4;
+  static constexpr int TH_OFF = BAR_OFF + NBAR * 8;  // [D/2] double: theta_i / pi
+  static constexpr int MISC_OFF = TH_OFF + (D / 2) * 8;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;   // + slack to align the base to 1024
   static constexpr int THREADS = 128 + 128 * MT;
   static constexpr int TMEM_S = 0;                    // S[mt][buf] at (2*mt + buf) * 64
@@ -167,6 +165,8 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
   }
+  double *theta_tab = reinterpret_cast<double *>(smem + C::TH_OFF);
+  if (threadIdx.x < D / 2) theta_tab[threadIdx.x] = freq_over_pi(threadIdx.x, D, g.log2_base);
   fence_proxy_async();
   fence_before_sync();
   __syncthreads();
@@ -283,12 +283,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     const bool wact = mt * 128 + wq * 32 < g.rows;  // warp holds at least one real row
     const uint32_t tl = (uint32_t)(wq * 32) << 16;
     const float sl2 = g.tau * 1.4426950408889634f;  // scores in log2 units
-    // Per-warp RoPE tables, so the warps of a warpgroup never wait on each other
-    // (only bounded mbarrier waits cross warps).
-    const int wid = warp - 4;
-    float2 *csL = reinterpret_cast<float2 *>(smem + C::CS_OFF) + wid * (D / 2);
-    float *thf = reinterpret_cast<float *>(smem + C::TH_OFF) + wid * (D / 2);
-    for (int ii = lane; ii < D / 2; ii += 32) thf[ii] = (float)(g.inv_freq_over_pi[ii] * CUDART_PI);
+    const int wg_tid = threadIdx.x - 128 - 128 * mt;  // 0..127 inside the warpgroup
     // waits are made warp-uniform so that warp-collective TMEM accesses never diverge
     auto wwait = [&](uint32_t b, uint32_t ph) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(b, ph, abort_flag));
@@ -299,45 +294,59 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     int i = 0;
     bool ok = true;
     while (ok && walk.next(g, p)) {
-      // cos/sin(L theta_i) for this piece; row t adds t theta_i by angle addition
-      __syncwarp();
-      for (int ii = lane; ii < D / 2; ii += 32) csL[ii] = rope_cs_f32(p.L, g.inv_freq_over_pi[ii]);
-      __syncwarp();
-      if (wact) {
+      // ---- Q^ of this unit: RoPE at position L + t, bf16, 128B-swizzled K-major.
+      // All 128 threads of the warpgroup share the rows; item = (row, 8-pair chunk).
+      {
+        constexpr int CHUNKS = D / 16, MAXIT = CHUNKS, KB = MT == 2 ? MAXIT / 2 : MAXIT;
+        const int real_rows = min(128, g.rows - mt * 128);
         const uint32_t qbase = sb + C::Q_OFF + mt * C::Q_BYTES;
-        const bool real = r < g.rows;
-        const int hl = real ? r / g.blk : 0, t = real ? r % g.blk : 0;
-        const uint4 *src = reinterpret_cast<const uint4 *>(
-            q + (((long long)p.b * g.blk + t) * g.hq + p.kvh * g.group + hl) * D);
-        uint4 raw[D / 8];  // the whole bf16 row, requested before any use
+#pragma unroll 1
+        for (int pass = 0; pass < MAXIT / KB; ++pass) {  // (two passes bound the registers at MT = 2)
+        uint4 xa[KB], xb[KB];
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) raw[c] = real ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          const uint32_t aw[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-          const uint32_t bw[4] = {raw[c + D / 16].x, raw[c + D / 16].y, raw[c + D / 16].z, raw[c + D / 16].w};
-          uint32_t y1w[4], y2w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float y1[2], y2[2];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int ii = 8 * c + 2 * e + h2;
-              const float x1 = __uint_as_float(h2 ? (aw[e] & 0xffff0000u) : (aw[e] << 16));
-              const float x2 = __uint_as_float(h2 ? (bw[e] & 0xffff0000u) : (bw[e] << 16));
-              float st_, ct_;
-              __sincosf((float)t * thf[ii], &st_, &ct_);
-              const float2 cl = csL[ii];
-              const float cs = cl.x * ct_ - cl.y * st_, sn = cl.y * ct_ + cl.x * st_;
-              y1[h2] = x1 * cs - x2 * sn;
-              y2[h2] = x2 * cs + x1 * sn;
-            }
-            y1w[e] = pack_bf16(y1[0], y1[1]);
-            y2w[e] = pack_bf16(y2[0], y2[1]);
+        for (int k = 0; k < KB; ++k) {  // every load of the pass first
+          const int item = wg_tid + 128 * (pass * KB + k), rr = item / CHUNKS, c = item % CHUNKS;
+          xa[k] = xb[k] = make_uint4(0, 0, 0, 0);
+          if (rr < real_rows) {
+            const int r2 = mt * 128 + rr, t = r2 % g.blk, hl = r2 / g.blk;
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                q + (((long long)p.b * g.blk + t) * g.hq + p.kvh * g.group + hl) * D);
+            xa[k] = __ldg(src + c);
+            xb[k] = __ldg(src + c + D / 16);
           }
-          const int e1 = 8 * c, e2 = D / 2 + 8 * c;  // first element of each chunk
-          st_shared_v4(qbase + (e1 / 64) * 16384 + sw128(row, (e1 % 64) / 8), y1w[0], y1w[1], y1w[2], y1w[3]);
-          st_shared_v4(qbase + (e2 / 64) * 16384 + sw128(row, (e2 % 64) / 8), y2w[0], y2w[1], y2w[2], y2w[3]);
+        }
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+          const int item = wg_tid + 128 * (pass * KB + k), rr = item / CHUNKS, c = item % CHUNKS;
+          if (rr >= real_rows) {  // padding rows of the M-tile are zeros
+            const int e1 = 8 * c, e2 = D / 2 + 8 * c;
+            st_shared_v4(qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8), 0, 0, 0, 0);
+            st_shared_v4(qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8), 0, 0, 0, 0);
+          } else {
+            const int t = (mt * 128 + rr) % g.blk;
+            const uint32_t aw[4] = {xa[k].x, xa[k].y, xa[k].z, xa[k].w};
+            const uint32_t bw[4] = {xb[k].x, xb[k].y, xb[k].z, xb[k].w};
+            uint32_t y1w[4], y2w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float y1[2], y2[2];
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const int ii = 8 * c + 2 * e + h2;
+                const float x1 = __uint_as_float(h2 ? (aw[e] & 0xffff0000u) : (aw[e] << 16));
+                const float x2 = __uint_as_float(h2 ? (bw[e] & 0xffff0000u) : (bw[e] << 16));
+                const float2 cs = rope_cs_fast(p.L + t, theta_tab[ii]);
+                y1[h2] = x1 * cs.x - x2 * cs.y;
+                y2[h2] = x2 * cs.x + x1 * cs.y;
+              }
+              y1w[e] = pack_bf16(y1[0], y1[1]);
+              y2w[e] = pack_bf16(y2[0], y2[1]);
+            }
+            const int e1 = 8 * c, e2 = D / 2 + 8 * c;  // first element of each chunk
+            st_shared_v4(qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8), y1w[0], y1w[1], y1w[2], y1w[3]);
+            st_shared_v4(qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8), y2w[0], y2w[1], y2w[2], y2w[3]);
+          }
+        }
         }
       }
       fence_proxy_async();
@@ -358,17 +367,22 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
         }
         fence_before_sync();
         mbar_arrive(bar(C::B_SEMPTY + 2 * mt + buf));
-        uint32_t pk[32];
         if (wact) {
           const int j = p.tile_begin + jj;
-          const int nval = min(KV_TILE, p.L - j * KV_TILE);
-          float tmax = -CUDART_INF_F;  // S is scaled to log2 units in place
+          const int nval = p.L - j * KV_TILE;
+          if (nval < KV_TILE) {  // the unit's partial last tile (warp-uniform)
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float v = c < nval ? __uint_as_float(sr[c]) * sl2 : -CUDART_INF_F;
-            sr[c] = __float_as_uint(v);
-            tmax = fmaxf(tmax, v);
+            for (int c = 0; c < 64; ++c)
+              if (c >= nval) sr[c] = __float_as_uint(-CUDART_INF_F);
           }
+          // tile max of the raw scores (tau > 0): 8 independent chains, then a tree
+          float mx[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
+#pragma unroll
+          for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
+          const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
           m_true = fmaxf(m_true, tmax);
           const bool need = jj > 0 && tmax > m_ref + 8.f;
           if (jj == 0) m_ref = tmax;
@@ -395,22 +409,30 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
               m_ref = tmax;
             }
           }
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const uint32_t w = pack_bf16(exp2f(__uint_as_float(sr[2 * c]) - m_ref),
-                                         exp2f(__uint_as_float(sr[2 * c + 1]) - m_ref));
-            lsum += __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
-            pk[c] = w;
-          }
         }
         if (!ok) break;
-        // P~ buffer is free once the previous tile's PV has completed
+        // the P~ buffer is free once the previous tile's PV has completed
         if (i > 0 && !wwait(bar(C::B_ODONE + mt), (i - 1) & 1)) { ok = false; break; }
         if (wact) {
+          // P~ = 2^(s*tau*log2(e) - m_ref): one FFMA and one exp2 per element,
+          // written to the swizzled P~ tile 8 keys (16 bytes) at a time
+          const float neg = -m_ref;
           const uint32_t pbase = sb + C::P_OFF + mt * C::P_BYTES;
+          float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            st_shared_v4(pbase + sw128(row, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int c8 = 0; c8 < 8; ++c8) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 8 * c8 + 2 * e;
+              const float p0 = exp2f(fmaf(__uint_as_float(sr[c]), sl2, neg));
+              const float p1 = exp2f(fmaf(__uint_as_float(sr[c + 1]), sl2, neg));
+              w4[e] = pack_bf16(p0, p1);
+              ps[e] += p0 + p1;
+            }
+            st_shared_v4(pbase + sw128(row, c8), w4[0], w4[1], w4[2], w4[3]);
+          }
+          lsum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         }
         fence_proxy_async();
         fence_before_sync();

@@ -72,7 +72,7 @@ typedef struct fbk_shape {
   int32_t n_kv_heads;  /* Hkv >= 1, Hq % Hkv == 0 */
   int32_t head_dim;    /* d in {64, 128} */
   int32_t block_len;   /* B in [1, 64]; G*B <= 256 */
-  float softmax_scale; /* tau: scores are tau * <RoPE(q), k> (the pages write S = Q K^T: tau = 1) */
+  float softmax_scale; /* tau > 0: scores are tau * <RoPE(q), k> (the pages write S = Q K^T: tau = 1) */
   double rope_base;    /* theta_i = rope_base^(-2i/d), rotate-half pairs (i, i + d/2) */
   int32_t mode;        /* fbk_mode */
 } fbk_shape;

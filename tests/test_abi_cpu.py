@@ -55,7 +55,8 @@ def _cache(fbk, **kw):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(batch=0), -1), (dict(n_q_heads=0), -1), (dict(block_len=0), -1), (dict(mode=3), -1),
-    (dict(rope_base=-1.0), -1), (dict(softmax_scale=float("nan")), -1),
+    (dict(rope_base=-1.0), -1), (dict(softmax_scale=float("nan")), -1), (dict(softmax_scale=0.0), -1),
+    (dict(softmax_scale=-0.5), -1),
     (dict(head_dim=96), -2), (dict(n_q_heads=6, n_kv_heads=4), -2), (dict(block_len=65), -2),
     (dict(n_q_heads=16, n_kv_heads=2, block_len=64), -2),
 ])
