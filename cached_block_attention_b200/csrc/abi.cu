@@ -23,6 +23,7 @@ fbk_status check_shape(const fbk_shape *s) {
   if (s->n_q_heads % s->n_kv_heads != 0) return FBK_ERR_UNSUPPORTED;
   if (s->block_len > 64) return FBK_ERR_UNSUPPORTED;
   if ((long long)(s->n_q_heads / s->n_kv_heads) * s->block_len > 256) return FBK_ERR_UNSUPPORTED;
+  if (s->batch > MAX_BATCH) return FBK_ERR_UNSUPPORTED;
   return FBK_OK;
 }
 
@@ -42,6 +43,10 @@ fbk_status check_cache(const fbk_shape *s, const fbk_kv_cache *c) {
     rows = (long long)s->batch * s->n_kv_heads * c->capacity_tokens;
   }
   if (rows > 0x7fffffffll) return FBK_ERR_CAPACITY;  // TMA row coordinates are int32
+  // the prefix kernels' tile list must stay below 2^31 entries
+  const long long per_seq = c->paged ? (long long)c->max_pages_per_seq * c->page_size : c->capacity_tokens;
+  if ((long long)s->batch * s->n_kv_heads * ((per_seq + KV_TILE - 1) / KV_TILE) > 0x7fffffffll)
+    return FBK_ERR_CAPACITY;
   return FBK_OK;
 }
 

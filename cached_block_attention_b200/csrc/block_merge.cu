@@ -26,6 +26,7 @@
 //  * FBK_FP32_CHECK: the same steps on CUDA cores in fp32 (no bf16 rounding of
 //    Q^, K^ or P~): lane j scores keys j and j + 32, warp-shuffle row max/sum.
 #include "launch.h"
+#include "tc.cuh"
 
 namespace fbk {
 namespace {
@@ -141,25 +142,45 @@ __global__ void __launch_bounds__(256) block_merge_mma_kernel(
   if (va) { m1a = __ldg(pfx.m + pa); l1a = __ldg(pfx.l + pa); }
   if (vbr) { m1b = __ldg(pfx.m + pb); l1b = __ldg(pfx.l + pb); }
 
-  // ---- 2. RoPE cos/sin of positions L .. L+B-1 (thread count is a multiple of d/2)
+  // ---- 2. RoPE cos/sin of positions L .. L+B-1 while the copies fly: each
+  // thread keeps one frequency i; cos/sin(L theta_i) is fp64-reduced, and the
+  // offset t theta_i (t < 64) is added by angle addition in fp32 (abs error
+  // ~1e-5, far below the bf16 rounding of Q^ and K^ that follows).
   {
     const int i = tid % HALF;
     const double f = freq_over_pi(i, D, g.log2_base);
-    for (int t = tid / HALF; t < blk; t += nthreads / HALF) cs[t * HALF + i] = rope_cs_fast(L + t, f);
+    const float2 cl = rope_cs_fast(L, f);
+    const float th = (float)(f * CUDART_PI);
+    for (int t = tid / HALF; t < blk; t += nthreads / HALF) {
+      float st, ct;
+      __sincosf((float)t * th, &st, &ct);
+      cs[t * HALF + i] = make_float2(cl.x * ct - cl.y * st, cl.y * ct + cl.x * st);
+    }
   }
   cp_async_wait_all();
   __syncthreads();
 
-  // ---- 3. rotate block K and the query rows in place (bf16)
-  for (int idx = tid; idx < (blk + rows_cta) * HALF; idx += nthreads) {
-    const int rowi = idx / HALF, i = idx % HALF;
+  // ---- 3. rotate block K and the query rows in place (bf16), 8 pairs per item
+  for (int idx = tid; idx < (blk + rows_cta) * (D / 16); idx += nthreads) {
+    const int rowi = idx / (D / 16), c = idx % (D / 16);
     const bool is_k = rowi < blk;
     const int t = is_k ? rowi : (r0 + rowi - blk) % blk;
-    __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(is_k ? Ks + rowi * RS : Qs + (rowi - blk) * RS);
-    const float x1 = __bfloat162float(row[i]), x2 = __bfloat162float(row[i + HALF]);
-    const float2 c = cs[t * HALF + i];
-    row[i] = __float2bfloat16_rn(x1 * c.x - x2 * c.y);
-    row[i + HALF] = __float2bfloat16_rn(x2 * c.x + x1 * c.y);
+    uint8_t *row = is_k ? Ks + rowi * RS : Qs + (rowi - blk) * RS;
+    uint4 *p1 = reinterpret_cast<uint4 *>(row + c * 16), *p2 = reinterpret_cast<uint4 *>(row + D + c * 16);
+    const uint4 a = *p1, bq = *p2;
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {bq.x, bq.y, bq.z, bq.w};
+    const float4 *cp = reinterpret_cast<const float4 *>(cs + t * HALF + 8 * c);
+    uint32_t y1[4], y2[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float4 c2 = cp[e];  // (cos, sin) of pairs 8c + 2e and 8c + 2e + 1
+      const float x1l = __uint_as_float(aw[e] << 16), x1h = __uint_as_float(aw[e] & 0xffff0000u);
+      const float x2l = __uint_as_float(bw[e] << 16), x2h = __uint_as_float(bw[e] & 0xffff0000u);
+      y1[e] = pack2(x1l * c2.x - x2l * c2.y, x1h * c2.z - x2h * c2.w);
+      y2[e] = pack2(x2l * c2.x + x1l * c2.y, x2h * c2.z + x1h * c2.w);
+    }
+    *p1 = make_uint4(y1[0], y1[1], y1[2], y1[3]);
+    *p2 = make_uint4(y2[0], y2[1], y2[2], y2[3]);
   }
   __syncthreads();
   if (warp >= nw_rows) return;
@@ -209,8 +230,8 @@ __global__ void __launch_bounds__(256) block_merge_mma_kernel(
   uint32_t pa_frag[8], pb_frag[8];  // P~ as bf16 pairs: [n-tile] for rows lr and lr + 8
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    const float p0 = exp2f(sacc[j][0] - mxa), p1 = exp2f(sacc[j][1] - mxa);
-    const float p2 = exp2f(sacc[j][2] - mxb), p3 = exp2f(sacc[j][3] - mxb);
+    const float p0 = tc::ex2(sacc[j][0] - mxa), p1 = tc::ex2(sacc[j][1] - mxa);
+    const float p2 = tc::ex2(sacc[j][2] - mxb), p3 = tc::ex2(sacc[j][3] - mxb);
     sa += p0 + p1;
     sbs += p2 + p3;
     pa_frag[j] = pack2(p0, p1);
@@ -275,11 +296,10 @@ cudaError_t launch_mma(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfl
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.bytes);
     if (e != cudaSuccess) return e;
   }
-  const int rows_cta = g.rows < MMA_MAX_ROWS ? g.rows : MMA_MAX_ROWS;
-  int warps = (rows_cta + 15) / 16;
-  if (warps * 32 % (D / 2)) ++warps;  // the RoPE table loop needs a multiple of d/2 threads
+  // 8 warps always: all of them load, build the RoPE table and rotate; only
+  // those that own query rows go on to the tensor-core part.
   dim3 grid((g.rows + MMA_MAX_ROWS - 1) / MMA_MAX_ROWS, g.batch * g.hkv);
-  kern<<<grid, warps * 32, lay.bytes, st>>>(g, q, kb, vb, pfx, static_cast<__nv_bfloat16 *>(out), lse);
+  kern<<<grid, 256, lay.bytes, st>>>(g, q, kb, vb, pfx, static_cast<__nv_bfloat16 *>(out), lse);
   return cudaGetLastError();
 }
 

@@ -56,13 +56,6 @@ __device__ __forceinline__ int prefix_len(const Geometry &g, int b) {
 
 __device__ __forceinline__ int tiles_of(int L) { return (L + KV_TILE - 1) / KV_TILE; }
 
-// Total tiles over all (sequence, kv-head) pairs.
-__device__ __forceinline__ long long total_tiles(const Geometry &g) {
-  long long t = 0;
-  for (int b = 0; b < g.batch; ++b) t += (long long)g.hkv * tiles_of(prefix_len(g, b));
-  return t;
-}
-
 // Share c of P covers list positions [c*T/P, (c+1)*T/P).
 __host__ __device__ __forceinline__ long long share_begin(long long c, long long T, long long P) {
   return (c * T) / P;
@@ -71,6 +64,33 @@ __host__ __device__ __forceinline__ long long share_begin(long long c, long long
 // The share that holds list position x (largest c with share_begin(c) <= x).
 __device__ __forceinline__ long long share_of(long long x, long long T, long long P) {
   return ((x + 1) * P - 1) / T;
+}
+
+// Per-sequence tile counts, loaded once per CTA: s_len[b] = validated L_b,
+// s_scan[b] = Hkv * sum_{b' <= b} ceil(L_b' / KV_TILE) (inclusive scan; the
+// host keeps the total below 2^31). All threads call it; the loads are issued
+// in parallel, one per thread. Returns T, the total tile count.
+constexpr int MAX_BATCH = 1024;  // sequences per call (shared-memory scan)
+
+__device__ __forceinline__ int load_tile_scan(const Geometry &g, int *s_len, int *s_scan) {
+  for (int b = threadIdx.x; b < g.batch; b += blockDim.x) s_len[b] = prefix_len(g, b);
+  __syncthreads();
+  if (threadIdx.x < 32) {  // one warp scans 32 sequences per round
+    int carry = 0;
+    for (int b0 = 0; b0 < g.batch; b0 += 32) {
+      const int b = b0 + (int)threadIdx.x;
+      int v = b < g.batch ? g.hkv * tiles_of(s_len[b]) : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if ((int)threadIdx.x >= o) v += n;
+      }
+      if (b < g.batch) s_scan[b] = carry + v;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+  }
+  __syncthreads();
+  return g.batch > 0 ? s_scan[g.batch - 1] : 0;
 }
 
 // A piece: the intersection of one share with one (sequence, kv-head) unit.
@@ -82,39 +102,45 @@ struct Piece {
   int tile_begin, tile_end;  // tile indices inside the unit
 };
 
-// Walks the pieces of one share in list order. Every warp role of a kernel
-// runs its own copy; the walk is deterministic, so all copies agree.
+// Walks the pieces of one share in list order, reading the shared-memory
+// scan. Every warp role of a kernel runs its own copy; the walk is
+// deterministic, so all copies agree.
 struct PieceWalker {
   long long pos, end;  // list positions still to cover
-  long long acc;       // list position where sequence b starts
-  int b, L, tb;        // current sequence, its length and tiles per kv-head
+  int b;               // current sequence
+  const int *len;
+  const int *scan;
 
-  __device__ __forceinline__ void init(const Geometry &g, long long share, long long T,
-                                       long long P) {
+  __device__ __forceinline__ void init(const Geometry &g, const int *s_len, const int *s_scan,
+                                       long long share, long long T, long long P) {
     pos = share_begin(share, T, P);
     end = share_begin(share + 1, T, P);
-    acc = 0;
-    b = 0;
-    L = g.batch > 0 ? prefix_len(g, 0) : 0;
-    tb = tiles_of(L);
+    len = s_len;
+    scan = s_scan;
+    // first sequence whose scan passes pos (binary search; scan is non-decreasing)
+    int lo = 0, hi = g.batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (scan[mid] > pos) hi = mid; else lo = mid + 1;
+    }
+    b = lo;
   }
 
   __device__ __forceinline__ bool next(const Geometry &g, Piece &p) {
     if (pos >= end) return false;
-    while (pos >= acc + (long long)g.hkv * tb) {
-      acc += (long long)g.hkv * tb;
-      if (++b >= g.batch) {  // only if the lengths changed under a running kernel
+    while (pos >= scan[b]) {
+      if (++b >= g.batch) {  // unreachable while the scan is consistent
         pos = end;
         return false;
       }
-      L = prefix_len(g, b);
-      tb = tiles_of(L);
     }
-    long long off = pos - acc;
-    int kvh = (int)(off / tb);
-    int j0 = (int)(off - (long long)kvh * tb);
-    long long unit_end = acc + (long long)(kvh + 1) * tb;
-    long long stop = unit_end < end ? unit_end : end;
+    const int L = len[b], tb = tiles_of(L);
+    const long long acc = scan[b] - (long long)g.hkv * tb;  // list position where sequence b starts
+    const long long off = pos - acc;
+    const int kvh = (int)(off / tb);
+    const int j0 = (int)(off - (long long)kvh * tb);
+    const long long unit_end = acc + (long long)(kvh + 1) * tb;
+    const long long stop = unit_end < end ? unit_end : end;
     p.b = b;
     p.kvh = kvh;
     p.u = b * g.hkv + kvh;

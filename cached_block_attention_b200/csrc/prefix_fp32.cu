@@ -22,7 +22,9 @@ struct Smem {
   static constexpr int V_OFF = K_OFF + KV_TILE * KP;
   static constexpr int Q_OFF = V_OFF + KV_TILE * D;
   static constexpr int P_OFF = Q_OFF + ROWS_PER_PASS * D;
-  static constexpr int FLOATS = P_OFF + ROWS_PER_PASS * KV_TILE;
+  static constexpr int LEN_OFF = P_OFF + ROWS_PER_PASS * KV_TILE;  // [MAX_BATCH] int
+  static constexpr int SCAN_OFF = LEN_OFF + MAX_BATCH;               // [MAX_BATCH] int
+  static constexpr int FLOATS = SCAN_OFF + MAX_BATCH;
 };
 
 template <int D>
@@ -39,10 +41,12 @@ __global__ void __launch_bounds__(THREADS) prefix_fp32_kernel(Geometry g,
   constexpr int CPL = D / 32;  // output columns per lane
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const long long T = total_tiles(g);
+  int *s_len = reinterpret_cast<int *>(sm + S::LEN_OFF);
+  int *s_scan = reinterpret_cast<int *>(sm + S::SCAN_OFF);
+  const long long T = load_tile_scan(g, s_len, s_scan);
   if (T == 0) return;
   PieceWalker walk;
-  walk.init(g, blockIdx.x, T, shares);
+  walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
   Piece p;
   while (walk.next(g, p)) {
     const long long slot = (long long)blockIdx.x + p.u;
@@ -55,7 +59,7 @@ __global__ void __launch_bounds__(THREADS) prefix_fp32_kernel(Geometry g,
           const int hl = r / g.blk, t = r % g.blk, h = p.kvh * g.group + hl;
           const __nv_bfloat16 *src = q + (((long long)p.b * g.blk + t) * g.hq + h) * D;
           const float x1 = __bfloat162float(src[i]), x2 = __bfloat162float(src[i + D / 2]);
-          const float2 cs = rope_cs_f32(p.L + t, g.inv_freq_over_pi[i]);
+          const float2 cs = rope_cs_f32(p.L + t, freq_over_pi(i, D, g.log2_base));
           y1 = x1 * cs.x - x2 * cs.y;
           y2 = x2 * cs.x + x1 * cs.y;
         }

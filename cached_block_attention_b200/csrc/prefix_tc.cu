@@ -60,7 +60,9 @@ struct Cfg {
   static constexpr int B_DRAIN = B_OFREE + MT;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int TH_OFF = BAR_OFF + NBAR * 8;  // [D/2] double: theta_i / pi
-  static constexpr int MISC_OFF = TH_OFF + (D / 2) * 8;
+  static constexpr int LEN_OFF = TH_OFF + (D / 2) * 8;  // [MAX_BATCH] int: validated L_b
+  static constexpr int SCAN_OFF = LEN_OFF + MAX_BATCH * 4;  // [MAX_BATCH] int: tile scan
+  static constexpr int MISC_OFF = SCAN_OFF + MAX_BATCH * 4;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;   // + slack to align the base to 1024
   static constexpr int THREADS = 128 + 128 * MT;
   static constexpr int TMEM_S = 0;                    // S[mt][buf] at (2*mt + buf) * 64
@@ -125,7 +127,9 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
   const uint32_t sb = raw_addr + pad;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const long long T = total_tiles(g);
+  int *s_len = reinterpret_cast<int *>(smem + C::LEN_OFF);
+  int *s_scan = reinterpret_cast<int *>(smem + C::SCAN_OFF);
+  const long long T = load_tile_scan(g, s_len, s_scan);
   if (T == 0) return;
   if (share_begin(blockIdx.x, T, shares) == share_begin(blockIdx.x + 1, T, shares)) return;
 
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       PieceWalker walk;
-      walk.init(g, blockIdx.x, T, shares);
+      walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
       Piece p;
       int i = 0, k_issued = 0, v_issued = 0;
       bool ok = true;
@@ -211,7 +215,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, KV_TILE, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
       PieceWalker walk;
-      walk.init(g, blockIdx.x, T, shares);
+      walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
       Piece p;
       int i = 0, pi = 0;
       bool ok = true;
@@ -289,7 +293,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
       return __all_sync(0xffffffffu, mbar_wait(b, ph, abort_flag));
     };
     PieceWalker walk;
-    walk.init(g, blockIdx.x, T, shares);
+    walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
     Piece p;
     int i = 0;
     bool ok = true;
@@ -425,8 +429,8 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int c = 8 * c8 + 2 * e;
-              const float p0 = exp2f(fmaf(__uint_as_float(sr[c]), sl2, neg));
-              const float p1 = exp2f(fmaf(__uint_as_float(sr[c + 1]), sl2, neg));
+              const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl2, neg));
+              const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl2, neg));
               w4[e] = pack_bf16(p0, p1);
               ps[e] += p0 + p1;
             }

@@ -16,20 +16,38 @@ namespace {
 constexpr int WARPS = 8;
 
 template <int D>
-__global__ void __launch_bounds__(WARPS * 32, 2) split_reduce_kernel(Geometry g, Workspace ws,
+__global__ void __launch_bounds__(WARPS * 32, 1) split_reduce_kernel(Geometry g, Workspace ws,
                                                                    int shares, fbk_partial out) {
   constexpr int CPL = D / 32;
   const int u = blockIdx.x, b = u / g.hkv, kvh = u % g.hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.y * WARPS + warp;
-  if (r >= g.rows) return;
 
+  // tiles before sequence b and in total: parallel loads, block reduction
+  __shared__ long long red[2][WARPS];
   long long before = 0, T = 0;
-  for (int bb = 0; bb < g.batch; ++bb) {
+  for (int bb = threadIdx.x; bb < g.batch; bb += WARPS * 32) {
     const long long n = (long long)g.hkv * tiles_of(prefix_len(g, bb));
     if (bb < b) before += n;
     T += n;
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+    T += __shfl_xor_sync(0xffffffffu, T, o);
+  }
+  if (lane == 0) {
+    red[0][warp] = before;
+    red[1][warp] = T;
+  }
+  __syncthreads();
+  before = T = 0;
+#pragma unroll
+  for (int w = 0; w < WARPS; ++w) {
+    before += red[0][w];
+    T += red[1][w];
+  }
+  if (r >= g.rows) return;
   const int tb = tiles_of(prefix_len(g, b));
   const long long A = before + (long long)kvh * tb, E = A + tb;
 

@@ -47,7 +47,7 @@ extern "C" {
 typedef enum fbk_status {
   FBK_OK = 0,
   FBK_ERR_INVALID_ARG = -1,  /* NULL pointer, non-positive size, bad struct field */
-  FBK_ERR_UNSUPPORTED = -2,  /* d not in {64,128}, Hq % Hkv != 0, G*B > 256, B > 64 ... */
+  FBK_ERR_UNSUPPORTED = -2,  /* d not in {64,128}, Hq % Hkv != 0, G*B > 256, B > 64, b > 1024 ... */
   FBK_ERR_CAPACITY = -3,     /* cache geometry cannot hold the request */
   FBK_ERR_WORKSPACE = -4,    /* workspace NULL or smaller than fbk_prefix_workspace_bytes */
   FBK_ERR_CUDA = -5          /* a CUDA runtime call or launch failed */
@@ -67,7 +67,7 @@ typedef enum fbk_mode { FBK_BF16 = 0, FBK_FP32_CHECK = 1 } fbk_mode;
 #define FBK_DEVERR_TIMEOUT 8u    /* a bounded device-side wait gave up (kernel returned early) */
 
 typedef struct fbk_shape {
-  int32_t batch;       /* b >= 1 */
+  int32_t batch;       /* 1 <= b <= 1024 */
   int32_t n_q_heads;   /* Hq >= 1 */
   int32_t n_kv_heads;  /* Hkv >= 1, Hq % Hkv == 0 */
   int32_t head_dim;    /* d in {64, 128} */

@@ -58,7 +58,7 @@ def _cache(fbk, **kw):
     (dict(rope_base=-1.0), -1), (dict(softmax_scale=float("nan")), -1), (dict(softmax_scale=0.0), -1),
     (dict(softmax_scale=-0.5), -1),
     (dict(head_dim=96), -2), (dict(n_q_heads=6, n_kv_heads=4), -2), (dict(block_len=65), -2),
-    (dict(n_q_heads=16, n_kv_heads=2, block_len=64), -2),
+    (dict(n_q_heads=16, n_kv_heads=2, block_len=64), -2), (dict(batch=1025), -2),
 ])
 def test_shape_validation(fbk, kw, code):
     s = _shape(fbk, **kw)

@@ -98,12 +98,17 @@ def test_stress_logits_and_rescale(mode, mname):
     """Growing logits: key tile t is scaled so the score spread rises from ~0.1
     to ~4 along the prefix, and the running max climbs by more than 8 log2
     units after the first tile, which drives the tensor-core kernel's rescale
-    of the TMEM accumulator."""
+    of the TMEM accumulator. The block keys are scaled down to keep the block
+    logits O(0.1) like the workloads': with unit-scale block Q and K (logits up
+    to ~30) the bf16 rounding of Q^ and K^ alone moves a logit by ~0.06, which
+    no bf16 tolerance can absorb."""
     from cached_block_attention_b200 import synth
     case = H.make_case(1, 8, 2, 128, 32, (700,), 0, 1.0, scale=1.0, seed=21, mode=mode)
     k = orc.bits_to_f64(case.k_pfx_bits[0])
     ramp = 0.01 + 0.034 * (np.arange(k.shape[1]) // 64)
     case.k_pfx_bits[0] = synth.bf16_bits(k * ramp[None, :, None])
+    qb, kb, vb = case.steps_bits[0]
+    case.steps_bits[0] = (qb, synth.bf16_bits(orc.bits_to_f64(kb) * 0.01), vb)
     case.upload()
     pfx = H.run_prefix(case, case.dev["steps"][0][0])
     ref = orc.prefix_partial(case.step_f64(0)[0], case.k_pfx(), case.v_pfx(), case.lens, 2, 1.0, case.base)
