@@ -6,20 +6,23 @@
 // (Eq. 2-6) whose result FACache keeps in HBM, here for the block's own query
 // rows (FlashBlock, Abstract: cached block-external attention).
 //
-// How (one CTA per SM-sized share of the flattened (unit, 64-key tile) list):
-//  * warp 0, one lane: TMA producer. Streams 64-key K and V tiles of the bf16
-//    cache (contiguous rows or pages) into an NS-stage ring, 128-byte swizzled,
-//    with an L2 evict-first policy (each KV byte is read once).
-//  * warp 1, one lane: MMA issuer. S = Q K^T (M=128 query rows, N=64 keys,
-//    K=d) into TMEM, then O += P V (M=128, N=d, K=64 keys) into a TMEM
-//    accumulator, all tcgen05.mma kind::f16 with fp32 accumulation. S of tile
-//    i+1 is issued before PV of tile i, and S is double-buffered in TMEM, so
-//    the tensor core works on the next tile while softmax runs.
+// How (one CTA per SM-sized share of the flattened (unit, 64-key tile) list),
+// warp-specialised, each role one elected lane or one warpgroup:
+//  * warps 0 and 3: TMA producers of 64-key K and V tiles of the bf16 cache
+//    (contiguous rows or pages) into NS-stage rings, 128-byte swizzled, L2
+//    evict-first (each KV byte is read once). K and V have separate rings and
+//    producers: a K stage frees as soon as S = Q K^T is done, a V stage only
+//    after O += P~ V, so K runs ahead of V.
+//  * warp 1: issues S = Q K^T (M = 128 query rows, N = 64 keys, K = d) into
+//    a double-buffered TMEM S; warp 2: issues O += P~ V (M = 128, N = d,
+//    K = 64 keys) into a TMEM accumulator. Both are tcgen05.mma kind::f16 with
+//    fp32 accumulation; two issuers keep a late K tile from holding back a
+//    ready PV product.
 //  * warps 4..4+4*MT-1: one warpgroup per 128-row M-tile (MT = ceil(G*B/128)).
 //    GQA packing: all G query heads of a kv-head share each staged K/V tile,
-//    so every KV byte is read from HBM once per unit. Each thread owns one
-//    query row = one TMEM lane: it rotates and writes its Q row (bf16,
-//    swizzled) at the start of a piece, reads its S row from TMEM, applies
+//    so every KV byte is read from HBM once per unit. The warpgroup rotates
+//    and writes Q (bf16, swizzled) at the start of a piece; then each thread
+//    owns one query row = one TMEM lane: it reads its S row from TMEM, applies
 //    the recurrence in the log2 domain and writes P~ (bf16) for the PV MMA.
 //    The O accumulator stays in TMEM; it is rescaled only when the running
 //    max grows by more than 2^8 over the reference max, which leaves the
@@ -57,8 +60,8 @@ struct Cfg {
   static constexpr int B_PFULL = B_SEMPTY + 2 * MT;
   static constexpr int B_ODONE = B_PFULL + MT;
   static constexpr int B_OFREE = B_ODONE + MT;
-  static constexpr int B_DRAIN = B_OFREE + MT;
-  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int B_DRAIN = B_OFREE + MT;  // [2]: S issuer, PV issuer
+  static constexpr int NBAR = B_DRAIN + 2;
   static constexpr int TH_OFF = BAR_OFF + NBAR * 8;  // [D/2] double: theta_i / pi
   static constexpr int LEN_OFF = TH_OFF + (D / 2) * 8;  // [MAX_BATCH] int: validated L_b
   static constexpr int SCAN_OFF = LEN_OFF + MAX_BATCH * 4;  // [MAX_BATCH] int: tile scan
@@ -84,6 +87,17 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
+}
+
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async16_s(uint32_t smem_addr, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr), "l"(gsrc) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -155,6 +169,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
       mbar_init(bar(C::B_OFREE + mt), 128);
     }
     mbar_init(bar(C::B_DRAIN), 1);
+    mbar_init(bar(C::B_DRAIN + 1), 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -177,86 +192,53 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
+  if (warp == 0 || warp == 3) {
+    // ---------------------------------------------------------------- producers
+    // warp 0 streams K tiles, warp 3 streams V tiles: K stages are released as
+    // soon as S = Q K^T is done, V stages only after O += P~ V, so separate
+    // producers let the K stream run ahead of the V stream.
     if (lane == 0) {
+      const bool is_k = warp == 0;
+      const CUtensorMap *map = is_k ? &tmk : &tmv;
+      const int b_full = is_k ? C::B_KFULL : C::B_VFULL, b_empty = is_k ? C::B_KEMPTY : C::B_VEMPTY;
+      const uint32_t ring = sb + (is_k ? C::K_OFF : C::V_OFF);
       const uint64_t pol = policy_evict_first();
       PieceWalker walk;
       walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
       Piece p;
-      int i = 0, k_issued = 0, v_issued = 0;
+      int i = 0;
       bool ok = true;
       while (ok && walk.next(g, p)) {
         for (int j = p.tile_begin; j < p.tile_end; ++j, ++i) {
           const int st = i % C::NS;
-          const uint32_t ph = ((i / C::NS) & 1) ^ 1;
-          if (!mbar_wait(bar(C::B_KEMPTY + st), ph, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(bar(C::B_KFULL + st), C::KV_BYTES);
-          load_kv_tile<D>(g, &tmk, sb + C::K_OFF + st * C::KV_BYTES, p, j, boxh,
-                          bar(C::B_KFULL + st), pol);
-          ++k_issued;
-          if (!mbar_wait(bar(C::B_VEMPTY + st), ph, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(bar(C::B_VFULL + st), C::KV_BYTES);
-          load_kv_tile<D>(g, &tmv, sb + C::V_OFF + st * C::KV_BYTES, p, j, boxh,
-                          bar(C::B_VFULL + st), pol);
-          ++v_issued;
+          if (!mbar_wait(bar(b_empty + st), ((i / C::NS) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(bar(b_full + st), C::KV_BYTES);
+          load_kv_tile<D>(g, map, ring + st * C::KV_BYTES, p, j, boxh, bar(b_full + st), pol);
         }
       }
       // no TMA write may be in flight when the CTA leaves
-      for (int n = max(0, k_issued - C::NS); n < k_issued; ++n)
-        mbar_wait_drain(bar(C::B_KFULL + n % C::NS), (n / C::NS) & 1);
-      for (int n = max(0, v_issued - C::NS); n < v_issued; ++n)
-        mbar_wait_drain(bar(C::B_VFULL + n % C::NS), (n / C::NS) & 1);
+      for (int n = max(0, i - C::NS); n < i; ++n) mbar_wait_drain(bar(b_full + n % C::NS), (n / C::NS) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
+    // ---------------------------------------------------------------- S = Q K^T issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, KV_TILE, false);
-      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
       PieceWalker walk;
       walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
       Piece p;
       int i = 0, pi = 0;
       bool ok = true;
-      // O[mt] += P~[mt] V for tile ii (the piece's first tile overwrites O)
-      auto issue_pv = [&](int ii, bool first) -> bool {
-        const int st = ii % C::NS;
-        if (!mbar_wait(bar(C::B_VFULL + st), (ii / C::NS) & 1, abort_flag)) return false;
-        if (first && pi > 0)
-          for (int mt = 0; mt < MT; ++mt)
-            if (!mbar_wait(bar(C::B_OFREE + mt), (pi - 1) & 1, abort_flag)) return false;
-        for (int mt = 0; mt < MT; ++mt) {
-          if (!mbar_wait(bar(C::B_PFULL + mt), ii & 1, abort_flag)) return false;
-          fence_after_sync();
-          const uint32_t d_tmem = tmem + C::TMEM_O + mt * D;
-#pragma unroll
-          for (int kk = 0; kk < KV_TILE / 16; ++kk) {
-            const uint64_t a = sdesc_sw128(sb + C::P_OFF + mt * C::P_BYTES + kk * 32, 16, 1024);
-            const uint64_t b = sdesc_sw128(sb + C::V_OFF + st * C::KV_BYTES + kk * 2048,
-                                           KV_TILE * 128, 1024);
-            mma_bf16(d_tmem, a, b, IDESC_PV, (first && kk == 0) ? 0u : 1u);
-          }
-          mma_commit(bar(C::B_ODONE + mt));
-        }
-        mma_commit(bar(C::B_VEMPTY + st));
-        return true;
-      };
       while (ok && walk.next(g, p)) {
-        for (int mt = 0; mt < MT && ok; ++mt)
-          ok = mbar_wait(bar(C::B_QFULL + mt), pi & 1, abort_flag);
+        for (int mt = 0; mt < MT && ok; ++mt) ok = mbar_wait(bar(C::B_QFULL + mt), pi & 1, abort_flag);
         if (!ok) break;
         fence_after_sync();
-        const int n = p.tile_end - p.tile_begin;
-        for (int jj = 0; jj < n && ok; ++jj, ++i) {
+        for (int j = p.tile_begin; j < p.tile_end && ok; ++j, ++i) {
           const int st = i % C::NS, buf = i & 1;
           if (!mbar_wait(bar(C::B_KFULL + st), (i / C::NS) & 1, abort_flag)) { ok = false; break; }
           fence_after_sync();
           for (int mt = 0; mt < MT && ok; ++mt) {
-            if (!mbar_wait(bar(C::B_SEMPTY + 2 * mt + buf), ((i >> 1) & 1) ^ 1, abort_flag)) {
-              ok = false;
-              break;
-            }
+            if (!mbar_wait(bar(C::B_SEMPTY + 2 * mt + buf), ((i >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
             fence_after_sync();
             const uint32_t d_tmem = tmem + C::TMEM_S + (2 * mt + buf) * KV_TILE;
 #pragma unroll
@@ -268,15 +250,48 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
             }
             mma_commit(bar(C::B_SFULL + 2 * mt + buf));
           }
-          if (!ok) break;
-          mma_commit(bar(C::B_KEMPTY + st));
-          if (jj > 0 && !issue_pv(i - 1, jj == 1)) { ok = false; break; }
+          if (ok) mma_commit(bar(C::B_KEMPTY + st));
         }
-        if (ok && !issue_pv(i - 1, n == 1)) ok = false;
         ++pi;
       }
       mma_commit(bar(C::B_DRAIN));
       mbar_wait_drain(bar(C::B_DRAIN), 0);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ---------------------------------------------------------------- O += P~ V issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
+      PieceWalker walk;
+      walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
+      Piece p;
+      int i = 0, pi = 0;
+      bool ok = true;
+      while (ok && walk.next(g, p)) {
+        for (int j = p.tile_begin; j < p.tile_end && ok; ++j, ++i) {
+          const bool first = j == p.tile_begin;  // the piece's first tile overwrites O
+          const int st = i % C::NS;
+          if (!mbar_wait(bar(C::B_VFULL + st), (i / C::NS) & 1, abort_flag)) { ok = false; break; }
+          if (first && pi > 0)  // the previous piece's epilogue has read O
+            for (int mt = 0; mt < MT && ok; ++mt) ok = mbar_wait(bar(C::B_OFREE + mt), (pi - 1) & 1, abort_flag);
+          for (int mt = 0; mt < MT && ok; ++mt) {
+            if (!mbar_wait(bar(C::B_PFULL + mt), i & 1, abort_flag)) { ok = false; break; }
+            fence_after_sync();
+            const uint32_t d_tmem = tmem + C::TMEM_O + mt * D;
+#pragma unroll
+            for (int kk = 0; kk < KV_TILE / 16; ++kk) {
+              const uint64_t a = sdesc_sw128(sb + C::P_OFF + mt * C::P_BYTES + kk * 32, 16, 1024);
+              const uint64_t b = sdesc_sw128(sb + C::V_OFF + st * C::KV_BYTES + kk * 2048, KV_TILE * 128, 1024);
+              mma_bf16(d_tmem, a, b, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+            }
+            mma_commit(bar(C::B_ODONE + mt));
+          }
+          if (ok) mma_commit(bar(C::B_VEMPTY + st));
+        }
+        ++pi;
+      }
+      mma_commit(bar(C::B_DRAIN + 1));
+      mbar_wait_drain(bar(C::B_DRAIN + 1), 0);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -299,44 +314,48 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     bool ok = true;
     while (ok && walk.next(g, p)) {
       // ---- Q^ of this unit: RoPE at position L + t, bf16, 128B-swizzled K-major.
-      // All 128 threads of the warpgroup share the rows; item = (row, 8-pair chunk).
+      // An item is 8 rotation pairs of one row (chunk c of each half). Each
+      // thread copies its items' raw bf16 chunks straight into their swizzled
+      // slots (all copies in flight at once), waits for its own copies, then
+      // rotates them in place; no other thread touches those bytes.
       {
-        constexpr int CHUNKS = D / 16, MAXIT = CHUNKS, KB = MT == 2 ? MAXIT / 2 : MAXIT;
+        constexpr int CHUNKS = D / 16;
         const int real_rows = min(128, g.rows - mt * 128);
         const uint32_t qbase = sb + C::Q_OFF + mt * C::Q_BYTES;
-#pragma unroll 1
-        for (int pass = 0; pass < MAXIT / KB; ++pass) {  // (two passes bound the registers at MT = 2)
-        uint4 xa[KB], xb[KB];
 #pragma unroll
-        for (int k = 0; k < KB; ++k) {  // every load of the pass first
-          const int item = wg_tid + 128 * (pass * KB + k), rr = item / CHUNKS, c = item % CHUNKS;
-          xa[k] = xb[k] = make_uint4(0, 0, 0, 0);
+        for (int k = 0; k < CHUNKS; ++k) {
+          const int item = wg_tid + 128 * k, rr = item / CHUNKS, c = item % CHUNKS;
+          const int e1 = 8 * c, e2 = D / 2 + 8 * c;
+          const uint32_t a1 = qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8);
+          const uint32_t a2 = qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8);
           if (rr < real_rows) {
             const int r2 = mt * 128 + rr, t = r2 % g.blk, hl = r2 / g.blk;
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                q + (((long long)p.b * g.blk + t) * g.hq + p.kvh * g.group + hl) * D);
-            xa[k] = __ldg(src + c);
-            xb[k] = __ldg(src + c + D / 16);
+            const __nv_bfloat16 *src = q + (((long long)p.b * g.blk + t) * g.hq + p.kvh * g.group + hl) * D;
+            cp_async16_s(a1, src + e1);
+            cp_async16_s(a2, src + e2);
+          } else {  // padding rows of the M-tile are zeros
+            st_shared_v4(a1, 0, 0, 0, 0);
+            st_shared_v4(a2, 0, 0, 0, 0);
           }
         }
+        cp_async_wait_all();
 #pragma unroll
-        for (int k = 0; k < KB; ++k) {
-          const int item = wg_tid + 128 * (pass * KB + k), rr = item / CHUNKS, c = item % CHUNKS;
-          if (rr >= real_rows) {  // padding rows of the M-tile are zeros
-            const int e1 = 8 * c, e2 = D / 2 + 8 * c;
-            st_shared_v4(qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8), 0, 0, 0, 0);
-            st_shared_v4(qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8), 0, 0, 0, 0);
-          } else {
-            const int t = (mt * 128 + rr) % g.blk;
-            const uint32_t aw[4] = {xa[k].x, xa[k].y, xa[k].z, xa[k].w};
-            const uint32_t bw[4] = {xb[k].x, xb[k].y, xb[k].z, xb[k].w};
+        for (int k = 0; k < CHUNKS; ++k) {
+          const int item = wg_tid + 128 * k, rr = item / CHUNKS, c = item % CHUNKS;
+          if (rr < real_rows) {
+            const int e1 = 8 * c, e2 = D / 2 + 8 * c, t = (mt * 128 + rr) % g.blk;
+            const uint32_t a1 = qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8);
+            const uint32_t a2 = qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8);
+            uint32_t aw[4], bw[4];
+            ld_shared_v4(a1, aw);
+            ld_shared_v4(a2, bw);
             uint32_t y1w[4], y2w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               float y1[2], y2[2];
 #pragma unroll
               for (int h2 = 0; h2 < 2; ++h2) {
-                const int ii = 8 * c + 2 * e + h2;
+                const int ii = e1 + 2 * e + h2;
                 const float x1 = __uint_as_float(h2 ? (aw[e] & 0xffff0000u) : (aw[e] << 16));
                 const float x2 = __uint_as_float(h2 ? (bw[e] & 0xffff0000u) : (bw[e] << 16));
                 const float2 cs = rope_cs_fast(p.L + t, theta_tab[ii]);
@@ -346,11 +365,9 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
               y1w[e] = pack_bf16(y1[0], y1[1]);
               y2w[e] = pack_bf16(y2[0], y2[1]);
             }
-            const int e1 = 8 * c, e2 = D / 2 + 8 * c;  // first element of each chunk
-            st_shared_v4(qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8), y1w[0], y1w[1], y1w[2], y1w[3]);
-            st_shared_v4(qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8), y2w[0], y2w[1], y2w[2], y2w[3]);
+            st_shared_v4(a1, y1w[0], y1w[1], y1w[2], y1w[3]);
+            st_shared_v4(a2, y2w[0], y2w[1], y2w[2], y2w[3]);
           }
-        }
         }
       }
       fence_proxy_async();
