@@ -43,20 +43,18 @@ using namespace tc;
 
 template <int D, int MT>
 struct Cfg {
-  static constexpr int NS = (D == 128) ? (MT == 2 ? 3 : 4) : (MT == 2 ? 6 : 8);
+  static constexpr int NS = (D == 128) ? (MT == 2 ? 4 : 5) : 8;  // K and V ring depth
   static constexpr int Q_BYTES = 128 * D * 2;          // one M-tile of Q
   static constexpr int KV_BYTES = KV_TILE * D * 2;     // one K (or V) stage
-  static constexpr int P_BYTES = 128 * KV_TILE * 2;    // one M-tile of P~
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + MT * Q_BYTES;
   static constexpr int V_OFF = K_OFF + NS * KV_BYTES;
-  static constexpr int P_OFF = V_OFF + NS * KV_BYTES;
-  static constexpr int BAR_OFF = P_OFF + MT * P_BYTES;
+  static constexpr int BAR_OFF = V_OFF + NS * KV_BYTES;
   // barrier indices
   static constexpr int B_KFULL = 0, B_KEMPTY = NS, B_VFULL = 2 * NS, B_VEMPTY = 3 * NS;
   static constexpr int B_QFULL = 4 * NS;
   static constexpr int B_SFULL = B_QFULL + MT;        // [MT][2]
-  static constexpr int B_SEMPTY = B_SFULL + 2 * MT;   // [MT][2]
+  static constexpr int B_SEMPTY = B_SFULL + 2 * MT;   // [MT][2]: S buffer (and the P~ in it) free
   static constexpr int B_PFULL = B_SEMPTY + 2 * MT;
   static constexpr int B_ODONE = B_PFULL + MT;
   static constexpr int B_OFREE = B_ODONE + MT;
@@ -128,6 +126,74 @@ __device__ __forceinline__ void load_kv_tile(const Geometry &g, const CUtensorMa
   }
 }
 
+// Query rows of one unit for M-tile mt, in two halves so the copies can be
+// requested early. An item is 8 rotation pairs of one row (chunk c of each
+// half of the row); thread wg_tid of the warpgroup owns items wg_tid + 128k.
+// issue_q_rows copies the raw bf16 chunks straight into their 128B-swizzled
+// slots of the Q tile (padding rows get zeros); rotate_q_rows waits for this
+// thread's own copies and rotates them in place (RoPE at L + t), so no other
+// thread ever touches those bytes.
+template <int D, int MT>
+__device__ __forceinline__ void issue_q_rows(const Geometry &g, const __nv_bfloat16 *__restrict__ q,
+                                             const Piece &p, uint32_t qbase, int mt, int wg_tid) {
+  constexpr int CHUNKS = D / 16;
+  const int real_rows = min(128, g.rows - mt * 128);
+#pragma unroll
+  for (int k = 0; k < CHUNKS; ++k) {
+    const int item = wg_tid + 128 * k, rr = item / CHUNKS, c = item % CHUNKS;
+    const int e1 = 8 * c, e2 = D / 2 + 8 * c;
+    const uint32_t a1 = qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8);
+    const uint32_t a2 = qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8);
+    if (rr < real_rows) {
+      const int r2 = mt * 128 + rr, t = r2 % g.blk, hl = r2 / g.blk;
+      const __nv_bfloat16 *src = q + (((long long)p.b * g.blk + t) * g.hq + p.kvh * g.group + hl) * D;
+      cp_async16_s(a1, src + e1);
+      cp_async16_s(a2, src + e2);
+    } else {
+      st_shared_v4(a1, 0, 0, 0, 0);
+      st_shared_v4(a2, 0, 0, 0, 0);
+    }
+  }
+}
+
+template <int D, int MT>
+__device__ __forceinline__ void rotate_q_rows(const Geometry &g, const Piece &p, uint32_t qbase, int mt,
+                                              int wg_tid, const double *theta_tab) {
+  constexpr int CHUNKS = D / 16;
+  const int real_rows = min(128, g.rows - mt * 128);
+  cp_async_wait_all();
+#pragma unroll
+  for (int k = 0; k < CHUNKS; ++k) {
+    const int item = wg_tid + 128 * k, rr = item / CHUNKS, c = item % CHUNKS;
+    if (rr < real_rows) {
+      const int e1 = 8 * c, e2 = D / 2 + 8 * c, t = (mt * 128 + rr) % g.blk;
+      const uint32_t a1 = qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8);
+      const uint32_t a2 = qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8);
+      uint32_t aw[4], bw[4];
+      ld_shared_v4(a1, aw);
+      ld_shared_v4(a2, bw);
+      uint32_t y1w[4], y2w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float y1[2], y2[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int ii = e1 + 2 * e + h2;
+          const float x1 = __uint_as_float(h2 ? (aw[e] & 0xffff0000u) : (aw[e] << 16));
+          const float x2 = __uint_as_float(h2 ? (bw[e] & 0xffff0000u) : (bw[e] << 16));
+          const float2 cs = rope_cs_fast(p.L + t, theta_tab[ii]);
+          y1[h2] = x1 * cs.x - x2 * cs.y;
+          y2[h2] = x2 * cs.x + x1 * cs.y;
+        }
+        y1w[e] = pack_bf16(y1[0], y1[1]);
+        y2w[e] = pack_bf16(y2[0], y2[1]);
+      }
+      st_shared_v4(a1, y1w[0], y1w[1], y1w[2], y1w[3]);
+      st_shared_v4(a2, y2w[0], y2w[1], y2w[2], y2w[3]);
+    }
+  }
+}
+
 template <int D, int MT>
 __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     prefix_tc_kernel(const __grid_constant__ Geometry g, const __nv_bfloat16 *__restrict__ q,
@@ -162,8 +228,8 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
       mbar_init(bar(C::B_QFULL + mt), 128);
       mbar_init(bar(C::B_SFULL + 2 * mt), 1);
       mbar_init(bar(C::B_SFULL + 2 * mt + 1), 1);
-      mbar_init(bar(C::B_SEMPTY + 2 * mt), 128);
-      mbar_init(bar(C::B_SEMPTY + 2 * mt + 1), 128);
+      mbar_init(bar(C::B_SEMPTY + 2 * mt), 1);
+      mbar_init(bar(C::B_SEMPTY + 2 * mt + 1), 1);
       mbar_init(bar(C::B_PFULL + mt), 128);
       mbar_init(bar(C::B_ODONE + mt), 1);
       mbar_init(bar(C::B_OFREE + mt), 128);
@@ -173,9 +239,6 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     *abort_flag = 0;
     mbar_fence_init();
   }
-  // P~ rows of warps whose rows are all padding are never written: zero them once.
-  for (int i = threadIdx.x; i < MT * C::P_BYTES / 16; i += C::THREADS)
-    reinterpret_cast<uint4 *>(smem + C::P_OFF)[i] = make_uint4(0, 0, 0, 0);
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
@@ -186,6 +249,17 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
   }
   double *theta_tab = reinterpret_cast<double *>(smem + C::TH_OFF);
   if (threadIdx.x < D / 2) theta_tab[threadIdx.x] = freq_over_pi(threadIdx.x, D, g.log2_base);
+  // The softmax warpgroups request their first unit's query rows now, before
+  // the producers start the K/V stream, so those few KB do not queue behind it.
+  PieceWalker sm_walk;
+  Piece sm_piece;
+  bool sm_more = false;
+  if (warp >= 4) {
+    sm_walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
+    sm_more = sm_walk.next(g, sm_piece);
+    if (sm_more) issue_q_rows<D, MT>(g, q, sm_piece, sb + C::Q_OFF + ((warp - 4) >> 2) * C::Q_BYTES,
+                                     (warp - 4) >> 2, threadIdx.x & 127);
+  }
   fence_proxy_async();
   fence_before_sync();
   __syncthreads();
@@ -278,13 +352,14 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
             if (!mbar_wait(bar(C::B_PFULL + mt), i & 1, abort_flag)) { ok = false; break; }
             fence_after_sync();
             const uint32_t d_tmem = tmem + C::TMEM_O + mt * D;
+            const uint32_t p_tmem = tmem + C::TMEM_S + (2 * mt + (i & 1)) * KV_TILE;
 #pragma unroll
             for (int kk = 0; kk < KV_TILE / 16; ++kk) {
-              const uint64_t a = sdesc_sw128(sb + C::P_OFF + mt * C::P_BYTES + kk * 32, 16, 1024);
               const uint64_t b = sdesc_sw128(sb + C::V_OFF + st * C::KV_BYTES + kk * 2048, KV_TILE * 128, 1024);
-              mma_bf16(d_tmem, a, b, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+              mma_bf16_ts(d_tmem, p_tmem + kk * 8, b, IDESC_PV, (first && kk == 0) ? 0u : 1u);
             }
             mma_commit(bar(C::B_ODONE + mt));
+            mma_commit(bar(C::B_SEMPTY + 2 * mt + (i & 1)));  // S / P~ buffer reusable
           }
           if (ok) mma_commit(bar(C::B_VEMPTY + st));
         }
@@ -297,79 +372,24 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- softmax
     const int mt = (warp - 4) >> 2, wq = warp & 3;
-    const int row = wq * 32 + lane;              // row inside the M-tile = TMEM lane
-    const int r = mt * 128 + row;                // query row inside the unit
+    const int row = wq * 32 + lane;                 // row inside the M-tile = TMEM lane
+    const int r = mt * 128 + row;                   // query row inside the unit
     const bool wact = mt * 128 + wq * 32 < g.rows;  // warp holds at least one real row
     const uint32_t tl = (uint32_t)(wq * 32) << 16;
     const float sl2 = g.tau * 1.4426950408889634f;  // scores in log2 units
-    const int wg_tid = threadIdx.x - 128 - 128 * mt;  // 0..127 inside the warpgroup
+    const int wg_tid = threadIdx.x & 127;           // 0..127 inside the warpgroup
+    const uint32_t qbase = sb + C::Q_OFF + mt * C::Q_BYTES;
     // waits are made warp-uniform so that warp-collective TMEM accesses never diverge
     auto wwait = [&](uint32_t b, uint32_t ph) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(b, ph, abort_flag));
     };
-    PieceWalker walk;
-    walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
-    Piece p;
+    Piece& p = sm_piece;
     int i = 0;
-    bool ok = true;
-    while (ok && walk.next(g, p)) {
-      // ---- Q^ of this unit: RoPE at position L + t, bf16, 128B-swizzled K-major.
-      // An item is 8 rotation pairs of one row (chunk c of each half). Each
-      // thread copies its items' raw bf16 chunks straight into their swizzled
-      // slots (all copies in flight at once), waits for its own copies, then
-      // rotates them in place; no other thread touches those bytes.
-      {
-        constexpr int CHUNKS = D / 16;
-        const int real_rows = min(128, g.rows - mt * 128);
-        const uint32_t qbase = sb + C::Q_OFF + mt * C::Q_BYTES;
-#pragma unroll
-        for (int k = 0; k < CHUNKS; ++k) {
-          const int item = wg_tid + 128 * k, rr = item / CHUNKS, c = item % CHUNKS;
-          const int e1 = 8 * c, e2 = D / 2 + 8 * c;
-          const uint32_t a1 = qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8);
-          const uint32_t a2 = qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8);
-          if (rr < real_rows) {
-            const int r2 = mt * 128 + rr, t = r2 % g.blk, hl = r2 / g.blk;
-            const __nv_bfloat16 *src = q + (((long long)p.b * g.blk + t) * g.hq + p.kvh * g.group + hl) * D;
-            cp_async16_s(a1, src + e1);
-            cp_async16_s(a2, src + e2);
-          } else {  // padding rows of the M-tile are zeros
-            st_shared_v4(a1, 0, 0, 0, 0);
-            st_shared_v4(a2, 0, 0, 0, 0);
-          }
-        }
-        cp_async_wait_all();
-#pragma unroll
-        for (int k = 0; k < CHUNKS; ++k) {
-          const int item = wg_tid + 128 * k, rr = item / CHUNKS, c = item % CHUNKS;
-          if (rr < real_rows) {
-            const int e1 = 8 * c, e2 = D / 2 + 8 * c, t = (mt * 128 + rr) % g.blk;
-            const uint32_t a1 = qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8);
-            const uint32_t a2 = qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8);
-            uint32_t aw[4], bw[4];
-            ld_shared_v4(a1, aw);
-            ld_shared_v4(a2, bw);
-            uint32_t y1w[4], y2w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float y1[2], y2[2];
-#pragma unroll
-              for (int h2 = 0; h2 < 2; ++h2) {
-                const int ii = e1 + 2 * e + h2;
-                const float x1 = __uint_as_float(h2 ? (aw[e] & 0xffff0000u) : (aw[e] << 16));
-                const float x2 = __uint_as_float(h2 ? (bw[e] & 0xffff0000u) : (bw[e] << 16));
-                const float2 cs = rope_cs_fast(p.L + t, theta_tab[ii]);
-                y1[h2] = x1 * cs.x - x2 * cs.y;
-                y2[h2] = x2 * cs.x + x1 * cs.y;
-              }
-              y1w[e] = pack_bf16(y1[0], y1[1]);
-              y2w[e] = pack_bf16(y2[0], y2[1]);
-            }
-            st_shared_v4(a1, y1w[0], y1w[1], y1w[2], y1w[3]);
-            st_shared_v4(a2, y2w[0], y2w[1], y2w[2], y2w[3]);
-          }
-        }
-      }
+    bool ok = true, first_piece = true;
+    while (ok && sm_more) {
+      if (!first_piece) issue_q_rows<D, MT>(g, q, p, qbase, mt, wg_tid);
+      first_piece = false;
+      rotate_q_rows<D, MT>(g, p, qbase, mt, wg_tid, theta_tab);
       fence_proxy_async();
       mbar_arrive(bar(C::B_QFULL + mt));
 
@@ -379,16 +399,12 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
         const int buf = i & 1;
         if (!wwait(bar(C::B_SFULL + 2 * mt + buf), (i >> 1) & 1)) { ok = false; break; }
         fence_after_sync();
-        uint32_t sr[64];
         if (wact) {
-          const uint32_t ta = tmem + tl + C::TMEM_S + (2 * mt + buf) * KV_TILE;
-          tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(sr));
-          tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+          const uint32_t ts = tmem + tl + C::TMEM_S + (2 * mt + buf) * KV_TILE;
+          uint32_t sr[64];
+          tmem_ld32(ts, *reinterpret_cast<uint32_t(*)[32]>(sr));
+          tmem_ld32(ts + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
           tmem_wait_ld();
-        }
-        fence_before_sync();
-        mbar_arrive(bar(C::B_SEMPTY + 2 * mt + buf));
-        if (wact) {
           const int j = p.tile_begin + jj;
           const int nval = p.L - j * KV_TILE;
           if (nval < KV_TILE) {  // the unit's partial last tile (warp-uniform)
@@ -408,7 +424,8 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
           const bool need = jj > 0 && tmax > m_ref + 8.f;
           if (jj == 0) m_ref = tmax;
           if (__any_sync(0xffffffffu, need)) {
-            // rescale this row's O~ (and l) to the new reference max
+            // rescale this row's O~ (and l) to the new reference max, once every
+            // PV product issued so far has landed
             if (!wwait(bar(C::B_ODONE + mt), (i - 1) & 1)) ok = false;
             fence_after_sync();
             const float f = need ? exp2f(m_ref - tmax) : 1.f;
@@ -430,32 +447,26 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
               m_ref = tmax;
             }
           }
+          if (ok) {
+            // P~ = 2^(s*tau*log2(e) - m_ref) (one FFMA and one exp2 per element),
+            // packed to bf16 pairs in place (pair c overwrites sr[c] after sr[2c],
+            // sr[2c+1] are read) and stored over the first 32 columns of this
+            // S buffer, where the PV issuer reads it as the A operand
+            const float neg = -m_ref;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, neg));
+              const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, neg));
+              sr[c] = pack_bf16(p0, p1);
+              ps[c & 3] += p0 + p1;
+            }
+            lsum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+            tmem_st32(ts, *reinterpret_cast<uint32_t(*)[32]>(sr));
+            tmem_wait_st();
+          }
         }
         if (!ok) break;
-        // the P~ buffer is free once the previous tile's PV has completed
-        if (i > 0 && !wwait(bar(C::B_ODONE + mt), (i - 1) & 1)) { ok = false; break; }
-        if (wact) {
-          // P~ = 2^(s*tau*log2(e) - m_ref): one FFMA and one exp2 per element,
-          // written to the swizzled P~ tile 8 keys (16 bytes) at a time
-          const float neg = -m_ref;
-          const uint32_t pbase = sb + C::P_OFF + mt * C::P_BYTES;
-          float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 8 * c8 + 2 * e;
-              const float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl2, neg));
-              const float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl2, neg));
-              w4[e] = pack_bf16(p0, p1);
-              ps[e] += p0 + p1;
-            }
-            st_shared_v4(pbase + sw128(row, c8), w4[0], w4[1], w4[2], w4[3]);
-          }
-          lsum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-        }
-        fence_proxy_async();
         fence_before_sync();
         mbar_arrive(bar(C::B_PFULL + mt));
       }
@@ -487,6 +498,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
       }
       fence_before_sync();
       mbar_arrive(bar(C::B_OFREE + mt));
+      sm_more = sm_walk.next(g, p);
     }
   }
 
