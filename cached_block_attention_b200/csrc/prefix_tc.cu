@@ -55,8 +55,10 @@ struct Cfg {
   static constexpr int B_QFULL = 4 * NS;
   static constexpr int B_SFULL = B_QFULL + MT;        // [MT][2]
   static constexpr int B_SEMPTY = B_SFULL + 2 * MT;   // [MT][2]: S buffer (and the P~ in it) free
+  // [MT][2]: P~ of the tile in S buffer `buf` is written. One barrier per S
+  // buffer, so an arrival for tile i+1 can never count toward tile i.
   static constexpr int B_PFULL = B_SEMPTY + 2 * MT;
-  static constexpr int B_ODONE = B_PFULL + MT;
+  static constexpr int B_ODONE = B_PFULL + 2 * MT;
   static constexpr int B_OFREE = B_ODONE + MT;
   static constexpr int B_DRAIN = B_OFREE + MT;  // [2]: S issuer, PV issuer
   static constexpr int NBAR = B_DRAIN + 2;
@@ -230,7 +232,8 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
       mbar_init(bar(C::B_SFULL + 2 * mt + 1), 1);
       mbar_init(bar(C::B_SEMPTY + 2 * mt), 1);
       mbar_init(bar(C::B_SEMPTY + 2 * mt + 1), 1);
-      mbar_init(bar(C::B_PFULL + mt), 128);
+      mbar_init(bar(C::B_PFULL + 2 * mt), 128);
+      mbar_init(bar(C::B_PFULL + 2 * mt + 1), 128);
       mbar_init(bar(C::B_ODONE + mt), 1);
       mbar_init(bar(C::B_OFREE + mt), 128);
     }
@@ -349,7 +352,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
           if (first && pi > 0)  // the previous piece's epilogue has read O
             for (int mt = 0; mt < MT && ok; ++mt) ok = mbar_wait(bar(C::B_OFREE + mt), (pi - 1) & 1, abort_flag);
           for (int mt = 0; mt < MT && ok; ++mt) {
-            if (!mbar_wait(bar(C::B_PFULL + mt), i & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(bar(C::B_PFULL + 2 * mt + (i & 1)), (i >> 1) & 1, abort_flag)) { ok = false; break; }
             fence_after_sync();
             const uint32_t d_tmem = tmem + C::TMEM_O + mt * D;
             const uint32_t p_tmem = tmem + C::TMEM_S + (2 * mt + (i & 1)) * KV_TILE;
@@ -468,7 +471,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
         }
         if (!ok) break;
         fence_before_sync();
-        mbar_arrive(bar(C::B_PFULL + mt));
+        mbar_arrive(bar(C::B_PFULL + 2 * mt + buf));
       }
       if (!ok) break;
       // epilogue: rebase to the true max and store this piece's state
