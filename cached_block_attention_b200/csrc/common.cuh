@@ -10,7 +10,7 @@
 #include <math_constants.h>
 #include <stdint.h>
 
-#include "../../include/fbk.h"
+#include "fbk.h"
 
 namespace fbk {
 

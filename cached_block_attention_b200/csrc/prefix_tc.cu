@@ -470,6 +470,11 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
           }
         }
         if (!ok) break;
+        // Track every phase of O_DONE in order: a parity wait is only exact when
+        // the barrier is at most one phase away, so each tile waits for the
+        // previous tile's PV here (normally long done), which keeps the rescale
+        // and epilogue waits below unambiguous.
+        if (i > 0 && !wwait(bar(C::B_ODONE + mt), (i - 1) & 1)) { ok = false; break; }
         fence_before_sync();
         mbar_arrive(bar(C::B_PFULL + 2 * mt + buf));
       }
