@@ -4,6 +4,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "launch.h"
 
 namespace fbk {
@@ -99,6 +101,30 @@ void ws_sizes(const fbk_shape *s, int shares, size_t *o_bytes, size_t *ml_bytes,
 }
 
 fbk_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FBK_OK : FBK_ERR_CUDA; }
+
+// Built-in scratch of fbk_prefix_partial_static_scratch: one array per device,
+// part of this file's device image, so using it allocates nothing.
+static __device__ __align__(256) unsigned char g_static_scratch[FBK_STATIC_SCRATCH_BYTES];
+
+constexpr int MAX_DEVICES = 64;
+std::mutex g_static_scratch_mu;
+void *g_static_scratch_addr[MAX_DEVICES];  // per device, looked up on first use
+
+// Device address of g_static_scratch on the current device. The first call
+// on a device asks the runtime (with that device current) and caches it.
+fbk_status static_scratch_address(void **ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FBK_ERR_CUDA;
+  if (dev < 0 || dev >= MAX_DEVICES) return FBK_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return FBK_ERR_CUDA;
+    g_static_scratch_addr[dev] = p;
+  }
+  *ptr = g_static_scratch_addr[dev];
+  return FBK_OK;
+}
 
 }  // namespace
 }  // namespace fbk
@@ -201,6 +227,36 @@ fbk_status fbk_full_ref_attn(const fbk_shape *shape, const void *q_blk, const vo
                                    shape->mode == FBK_FP32_CHECK, static_cast<cudaStream_t>(cuda_stream)));
 }
 
+fbk_status fbk_prefix_partial_static_scratch(const fbk_shape *shape, const void *q_blk,
+                                             const fbk_kv_cache *cache, const fbk_partial *out,
+                                             int32_t num_splits, void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if ((st = check_cache(shape, cache)) != FBK_OK) return st;
+  if (!q_blk || !out || !out->o_unnorm || !out->m || !out->l || num_splits < 0) return FBK_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(q_blk) & 15u) return FBK_ERR_UNSUPPORTED;
+  const int shares = num_splits ? num_splits : default_shares();
+  if (shares < 1) return FBK_ERR_CUDA;
+  size_t ob, mlb;
+  long long slots;
+  ws_sizes(shape, shares, &ob, &mlb, &slots);
+  if (ob + 2 * mlb > (size_t)FBK_STATIC_SCRATCH_BYTES) return FBK_ERR_SCRATCH_LIMIT;
+  void *scratch = nullptr;
+  if ((st = static_scratch_address(&scratch)) != FBK_OK) return st;
+  Workspace w;
+  w.o = static_cast<float *>(scratch);
+  w.m = reinterpret_cast<float *>(static_cast<char *>(scratch) + ob);
+  w.l = reinterpret_cast<float *>(static_cast<char *>(scratch) + ob + mlb);
+  w.slots = slots;
+  const Geometry g = make_geometry(shape, cache);
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_blk);
+  cudaError_t e = shape->mode == FBK_BF16 ? launch_prefix_tc(g, q, w, shares, s)
+                                          : launch_prefix_fp32(g, q, w, shares, s);
+  if (e != cudaSuccess) return FBK_ERR_CUDA;
+  return from_cuda(launch_split_reduce(g, w, shares, *out, s));
+}
+
 const char *fbk_status_string(fbk_status status) {
   switch (status) {
     case FBK_OK: return "ok";
@@ -209,6 +265,7 @@ const char *fbk_status_string(fbk_status status) {
     case FBK_ERR_CAPACITY: return "cache geometry exceeds the supported size";
     case FBK_ERR_WORKSPACE: return "workspace missing or too small";
     case FBK_ERR_CUDA: return "CUDA error";
+    case FBK_ERR_SCRATCH_LIMIT: return "call needs more scratch than the built-in 32 MiB array";
   }
   return "unknown status";
 }

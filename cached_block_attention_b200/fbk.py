@@ -33,7 +33,9 @@ DEVERR_TIMEOUT = 8
 
 EXPORTS = ("fbk_prefix_workspace_bytes", "fbk_default_num_splits", "fbk_prefix_partial",
            "fbk_block_attn_merge", "fbk_commit_block_rope_append", "fbk_full_ref_attn",
-           "fbk_status_string")
+           "fbk_status_string", "fbk_prefix_partial_static_scratch")
+
+STATIC_SCRATCH_BYTES = 32 << 20  # FBK_STATIC_SCRATCH_BYTES
 
 
 class _Shape(ctypes.Structure):
@@ -70,6 +72,9 @@ _lib.fbk_commit_block_rope_append.argtypes = [_P(_Shape), _vp, _vp, _P(_Cache), 
 _lib.fbk_commit_block_rope_append.restype = ctypes.c_int
 _lib.fbk_full_ref_attn.argtypes = [_P(_Shape), _vp, _vp, _vp, _P(_Cache), _vp, _vp, _vp]
 _lib.fbk_full_ref_attn.restype = ctypes.c_int
+_lib.fbk_prefix_partial_static_scratch.argtypes = [_P(_Shape), _vp, _P(_Cache), _P(_Partial),
+                                                   ctypes.c_int32, _vp]
+_lib.fbk_prefix_partial_static_scratch.restype = ctypes.c_int
 _lib.fbk_status_string.argtypes = [ctypes.c_int]
 _lib.fbk_status_string.restype = ctypes.c_char_p
 
@@ -176,6 +181,16 @@ def prefix_partial(shape: Shape, q_blk: torch.Tensor, cache: KVCache, out: Parti
     _check(_lib.fbk_prefix_partial(ctypes.byref(cs), _ptr(q_blk), ctypes.byref(cc), ctypes.byref(po),
                                    _ptr(ws), ws.numel() * ws.element_size(), num_splits,
                                    _stream(stream)), "fbk_prefix_partial")
+
+
+def prefix_partial_static_scratch(shape: Shape, q_blk: torch.Tensor, cache: KVCache, out: Partial,
+                                  num_splits: int = 0, stream=None) -> None:
+    """prefix_partial using the library's built-in per-device scratch array
+    (no workspace argument; calls on one device must not overlap)."""
+    cs, cc, po = shape.c(), cache.c(), out.c()
+    _check(_lib.fbk_prefix_partial_static_scratch(ctypes.byref(cs), _ptr(q_blk), ctypes.byref(cc),
+                                                  ctypes.byref(po), num_splits, _stream(stream)),
+           "fbk_prefix_partial_static_scratch")
 
 
 def block_attn_merge(shape: Shape, q_blk, k_blk, v_blk, prefix_lens, prefix: Partial, out,

@@ -19,7 +19,8 @@
  *  - Memory. Every pointer argument is DEVICE memory owned by the caller,
  *    except the structs themselves (fbk_shape, fbk_kv_cache, fbk_partial),
  *    which are host structs read during the call only. The library allocates
- *    nothing, keeps no state between calls and never synchronises.
+ *    nothing and never synchronises. Apart from fbk_prefix_partial_static_scratch
+ *    (last below), it keeps no state between calls.
  *  - Streams. `cuda_stream` is a cudaStream_t (NULL = legacy default stream).
  *    Every call only enqueues work on it and returns.
  *  - Errors. Argument errors are detected on the host and returned before any
@@ -50,7 +51,9 @@ typedef enum fbk_status {
   FBK_ERR_UNSUPPORTED = -2,  /* d not in {64,128}, Hq % Hkv != 0, G*B > 256, B > 64, b > 1024 ... */
   FBK_ERR_CAPACITY = -3,     /* cache geometry cannot hold the request */
   FBK_ERR_WORKSPACE = -4,    /* workspace NULL or smaller than fbk_prefix_workspace_bytes */
-  FBK_ERR_CUDA = -5          /* a CUDA runtime call or launch failed */
+  FBK_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed */
+  FBK_ERR_SCRATCH_LIMIT = -6 /* fbk_prefix_partial_static_scratch: the call needs more than
+                                FBK_STATIC_SCRATCH_BYTES of scratch */
 } fbk_status;
 
 /* Arithmetic of a call.
@@ -167,6 +170,48 @@ fbk_status fbk_commit_block_rope_append(const fbk_shape *shape, const void *k_bl
 fbk_status fbk_full_ref_attn(const fbk_shape *shape, const void *q_blk, const void *k_blk,
                              const void *v_blk, const fbk_kv_cache *cache, void *out,
                              float *lse, void *cuda_stream);
+
+/* Size of the library's built-in scratch array (per device) used by
+ * fbk_prefix_partial_static_scratch: 32 MiB. */
+#define FBK_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* fbk_prefix_partial without a caller-supplied workspace. The pages have no
+ * counterpart to this call: it is an interface convenience only, and it
+ * computes exactly what fbk_prefix_partial computes, with the same two
+ * kernels and the same results.
+ *
+ * Who it is for. Some callers cannot hand over scratch memory. Examples are a
+ * plain C host with no device allocator of its own, or a plug-in inside another
+ * runtime whose memory pool owns the device and forbids outside allocations.
+ * Another is code that must not call cudaMalloc/cudaFree, because those
+ * calls can synchronise the device and stall other streams. This entry point
+ * allocates nothing either: its scratch is a fixed array of
+ * FBK_STATIC_SCRATCH_BYTES bytes in the library's own device image, one per
+ * device, created when the CUDA module is loaded.
+ *
+ * Arguments are those of fbk_prefix_partial minus ws and ws_bytes.
+ *
+ * Set-up. The first call on each device looks up the array's address with
+ * cudaGetSymbolAddress, with that device current, and caches it for the rest of
+ * the process. Make that first call before any stream capture begins on that
+ * device. The cached address does not survive cudaDeviceReset.
+ *
+ * Limit. A call whose workspace, fbk_prefix_workspace_bytes(shape, cache,
+ * num_splits), exceeds FBK_STATIC_SCRATCH_BYTES returns FBK_ERR_SCRATCH_LIMIT
+ * before any launch. Lower num_splits, or use fbk_prefix_partial.
+ *
+ * Zeroing. No part of the array has to start at zero. Every scratch slot the
+ * reduction reads is written by the share kernel of the same call.
+ *
+ * Concurrency. There is one array per device, shared by every caller. Calls
+ * that overlap on one device race on it and corrupt each other's results:
+ * calls from different streams or host threads must be ordered (one stream, or
+ * events).
+ *
+ * Errors are otherwise those of fbk_prefix_partial. */
+fbk_status fbk_prefix_partial_static_scratch(const fbk_shape *shape, const void *q_blk,
+                                             const fbk_kv_cache *cache, const fbk_partial *out,
+                                             int32_t num_splits, void *cuda_stream);
 
 /* Static text for a status code. */
 const char *fbk_status_string(fbk_status status);
