@@ -421,7 +421,7 @@ def run_ours(args, wl, rank, world, local):
                    "schedule": "reuse (prefix state computed once per block)"},
         "roofline": roofline,
         "prefix_partial": {"us": pfx_ms * 1e3, "kv_gbs": pfx_gbs, "tflops": pfx_tfs,
-                           "hbm_frac": pfx_gbs / hbm_gbs, "tensor_frac": pfx_tfs * 1e3 / tflops,
+                           "hbm_frac": pfx_gbs / hbm_gbs, "tensor_frac": pfx_tfs / tflops,
                            "kv_bytes": kv_bytes, "flops": pfx_flops},
         "step_us": step_launch_ms * 1e3, "commit_us": commit_ms * 1e3,
         "recompute_schedule": {"value": world * S / (rec_ms * 1e-3), "unit": "denoising steps/s",

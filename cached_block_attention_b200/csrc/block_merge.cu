@@ -95,6 +95,10 @@ __global__ void __launch_bounds__(256) block_merge_mma_kernel(
   const int r0 = blockIdx.x * MMA_MAX_ROWS;
   const int rows_cta = min(MMA_MAX_ROWS, g.rows - r0);
   const int nthreads = blockDim.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // this thread's RoPE frequency (kernel parameters only: before the wait)
+  const double rope_f = freq_over_pi(tid % HALF, D, g.log2_base);
+  pdl_release();
+  pdl_wait();
   int L = g.lens[b];
   if (L < 0) {
     raise_flag(g, FBK_DEVERR_PREFIX_LEN);
@@ -148,7 +152,7 @@ __global__ void __launch_bounds__(256) block_merge_mma_kernel(
   // ~1e-5, far below the bf16 rounding of Q^ and K^ that follows).
   {
     const int i = tid % HALF;
-    const double f = freq_over_pi(i, D, g.log2_base);
+    const double f = rope_f;
     const float2 cl = rope_cs_fast(L, f);
     const float th = (float)(f * CUDART_PI);
     for (int t = tid / HALF; t < blk; t += nthreads / HALF) {
@@ -299,8 +303,8 @@ cudaError_t launch_mma(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfl
   // 8 warps always: all of them load, build the RoPE table and rotate; only
   // those that own query rows go on to the tensor-core part.
   dim3 grid((g.rows + MMA_MAX_ROWS - 1) / MMA_MAX_ROWS, g.batch * g.hkv);
-  kern<<<grid, 256, lay.bytes, st>>>(g, q, kb, vb, pfx, static_cast<__nv_bfloat16 *>(out), lse);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(256), lay.bytes, st, g, q, kb, vb, pfx,
+                    static_cast<__nv_bfloat16 *>(out), lse);
 }
 
 // ====================================================================== fp32 check (CUDA cores)
@@ -349,6 +353,9 @@ __global__ void __launch_bounds__(THREADS) block_merge_f32_kernel(
   const int u = blockIdx.y, b = u / g.hkv, kvh = u % g.hkv;
   const int r0 = blockIdx.x * RC;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const double rope_f = freq_over_pi(tid % HALF, D, g.log2_base);
+  pdl_release();
+  pdl_wait();
   int L = g.lens[b];
   if (L < 0) {
     raise_flag(g, FBK_DEVERR_PREFIX_LEN);
@@ -387,8 +394,7 @@ __global__ void __launch_bounds__(THREADS) block_merge_f32_kernel(
   }
   {  // RoPE table, accurate sincospi (check mode); each thread keeps one frequency
     const int i = tid % HALF;
-    const double f = freq_over_pi(i, D, g.log2_base);
-    for (int t = tid / HALF; t < blk; t += THREADS / HALF) cs[t * HALF + i] = rope_cs_f32(L + t, f);
+    for (int t = tid / HALF; t < blk; t += THREADS / HALF) cs[t * HALF + i] = rope_cs_f32(L + t, rope_f);
   }
   cp_async_wait_all();
   __syncthreads();
@@ -475,8 +481,8 @@ cudaError_t launch_f32_cfg(const Geometry &g, const __nv_bfloat16 *q, const __nv
     if (e != cudaSuccess) return e;
   }
   dim3 grid((g.rows + RC - 1) / RC, g.batch * g.hkv);
-  kern<<<grid, THREADS, lay.bytes, st>>>(g, q, kb, vb, pfx, static_cast<float *>(out), lse);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(THREADS), lay.bytes, st, g, q, kb, vb, pfx,
+                    static_cast<float *>(out), lse);
 }
 
 template <int D>

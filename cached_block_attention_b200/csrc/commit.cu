@@ -32,6 +32,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(THREADS)
   __shared__ double2 tab[MAX_TOK * HALF];
   const int b = blockIdx.y, crank = blockIdx.x, blk = g.blk;
   const int t0 = crank * blk / CLUSTER, t1 = (crank + 1) * blk / CLUSTER, nt = t1 - t0;
+  pdl_release();
+  pdl_wait();
   if (threadIdx.x == 0) {
     const int L = lens[b];
     bool ok = L >= 0 && (long long)L + blk <= seq_capacity(g);
@@ -133,11 +135,8 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(THREADS)
 cudaError_t launch_commit(const Geometry &g, const __nv_bfloat16 *kb, const __nv_bfloat16 *vb,
                           __nv_bfloat16 *kc, __nv_bfloat16 *vc, int *lens, cudaStream_t st) {
   dim3 grid(CLUSTER, g.batch);
-  if (g.d == 128)
-    commit_kernel<128><<<grid, THREADS, 0, st>>>(g, kb, vb, kc, vc, lens);
-  else
-    commit_kernel<64><<<grid, THREADS, 0, st>>>(g, kb, vb, kc, vc, lens);
-  return cudaGetLastError();
+  if (g.d == 128) return launch_pdl(commit_kernel<128>, grid, dim3(THREADS), 0, st, g, kb, vb, kc, vc, lens);
+  return launch_pdl(commit_kernel<64>, grid, dim3(THREADS), 0, st, g, kb, vb, kc, vc, lens);
 }
 
 }  // namespace fbk

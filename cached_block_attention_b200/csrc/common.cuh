@@ -259,6 +259,21 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
+// Programmatic dependent launch. Every kernel of the library is launched with
+// programmatic stream serialization, so it may become resident while the
+// kernel before it in the stream is still running. pdl_wait() returns once
+// that predecessor has completed and its writes are visible: each kernel calls
+// it before its first read of anything another kernel may have written
+// (inputs, prefix lengths, states), and before its first global write. Only
+// work on kernel parameters and shared memory comes before it. pdl_release()
+// lets the next kernel in the stream start launching; each kernel calls it
+// once all of its CTAs are running, i.e. at its top. Both are no-ops for a
+// kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Workspace view of the per-share states written by the prefix kernels.
 struct Workspace {
   float *o;  // [slots, rows, d]

@@ -7,6 +7,25 @@
 
 namespace fbk {
 
+// Launch with programmatic stream serialization (see pdl_wait / pdl_release):
+// the kernel may start while its stream predecessor finishes, and waits for it
+// on the device before touching its results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 struct TmaMaps;  // defined in prefix_tc.cu
 
 // fp32 CUDA-core prefix kernel (FBK_FP32_CHECK): one CTA per share.

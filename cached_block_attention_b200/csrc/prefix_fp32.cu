@@ -43,6 +43,8 @@ __global__ void __launch_bounds__(THREADS) prefix_fp32_kernel(Geometry g,
 
   int *s_len = reinterpret_cast<int *>(sm + S::LEN_OFF);
   int *s_scan = reinterpret_cast<int *>(sm + S::SCAN_OFF);
+  pdl_release();
+  pdl_wait();
   const long long T = load_tile_scan(g, s_len, s_scan);
   if (T == 0) return;
   PieceWalker walk;
@@ -156,8 +158,7 @@ cudaError_t launch_d(const Geometry &g, const __nv_bfloat16 *q, const Workspace 
   cudaError_t e = cudaFuncSetAttribute(prefix_fp32_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
-  prefix_fp32_kernel<D><<<shares, THREADS, bytes, st>>>(g, q, ws, shares);
-  return cudaGetLastError();
+  return launch_pdl(prefix_fp32_kernel<D>, dim3(shares), dim3(THREADS), bytes, st, g, q, ws, shares);
 }
 
 }  // namespace

@@ -211,6 +211,15 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
 
   int *s_len = reinterpret_cast<int *>(smem + C::LEN_OFF);
   int *s_scan = reinterpret_cast<int *>(smem + C::SCAN_OFF);
+  // kernel parameters only before the wait: tensor maps and the RoPE table
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+  }
+  double *theta_tab = reinterpret_cast<double *>(smem + C::TH_OFF);
+  if (threadIdx.x < D / 2) theta_tab[threadIdx.x] = freq_over_pi(threadIdx.x, D, g.log2_base);
+  pdl_release();
+  pdl_wait();
   const long long T = load_tile_scan(g, s_len, s_scan);
   if (T == 0) return;
   if (share_begin(blockIdx.x, T, shares) == share_begin(blockIdx.x + 1, T, shares)) return;
@@ -246,12 +255,6 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
-  }
-  double *theta_tab = reinterpret_cast<double *>(smem + C::TH_OFF);
-  if (threadIdx.x < D / 2) theta_tab[threadIdx.x] = freq_over_pi(threadIdx.x, D, g.log2_base);
   // The softmax warpgroups request their first unit's query rows now, before
   // the producers start the K/V stream, so those few KB do not queue behind it.
   PieceWalker sm_walk;
@@ -557,8 +560,7 @@ cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const Workspac
   auto kern = prefix_tc_kernel<D, MT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<shares, C::THREADS, C::SMEM, st>>>(g, q, ws, shares, mk, mv, boxh);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(shares), dim3(C::THREADS), C::SMEM, st, g, q, ws, shares, mk, mv, boxh);
 }
 
 }  // namespace

@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) split_reduce_kernel(Geometry g,
   const int u = blockIdx.x, b = u / g.hkv, kvh = u % g.hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.y * WARPS + warp;
+  pdl_release();
+  pdl_wait();
 
   // tiles before sequence b and in total: parallel loads, block reduction
   __shared__ long long red[2][WARPS];
@@ -103,11 +105,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) split_reduce_kernel(Geometry g,
 cudaError_t launch_split_reduce(const Geometry &g, const Workspace &ws, int shares,
                                 const fbk_partial &out, cudaStream_t st) {
   dim3 grid(g.batch * g.hkv, (g.rows + WARPS - 1) / WARPS);
-  if (g.d == 128)
-    split_reduce_kernel<128><<<grid, WARPS * 32, 0, st>>>(g, ws, shares, out);
-  else
-    split_reduce_kernel<64><<<grid, WARPS * 32, 0, st>>>(g, ws, shares, out);
-  return cudaGetLastError();
+  if (g.d == 128) return launch_pdl(split_reduce_kernel<128>, grid, dim3(WARPS * 32), 0, st, g, ws, shares, out);
+  return launch_pdl(split_reduce_kernel<64>, grid, dim3(WARPS * 32), 0, st, g, ws, shares, out);
 }
 
 }  // namespace fbk
