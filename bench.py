@@ -45,6 +45,38 @@ def parse():
     return ap.parse_args()
 
 
+# DRAM traffic per launch of the dominant kernels, from ncu captures
+# (dram__bytes_read.sum + dram__bytes_write.sum). An entry counts only while the
+# kernel's sources hash to the value recorded with it; otherwise traffic is null.
+TRAFFIC_FILE = os.path.join(ROOT, "cached_block_attention_b200", "ncu_traffic.json")
+KERNEL_SOURCES = {
+    "block_merge_mma_kernel": ["block_merge.cu", "common.cuh", "tc.cuh", "launch.h"],
+    "prefix_tc_kernel": ["prefix_tc.cu", "common.cuh", "tc.cuh", "launch.h"],
+}
+API_KERNEL = {"fbk_block_attn_merge": "block_merge_mma_kernel", "fbk_prefix_partial": "prefix_tc_kernel"}
+
+
+def sources_hash(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "cached_block_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel, workload):
+    try:
+        with open(TRAFFIC_FILE) as f:
+            entries = json.load(f)
+    except (OSError, ValueError):
+        return None
+    for e in entries:
+        if e.get("kernel") == kernel and e.get("workload") == workload and e.get("sources") == sources_hash(kernel):
+            return e
+    return None
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -294,20 +326,36 @@ def run_ours(args, wl, rank, world, local):
     torch.cuda.synchronize()
     assert int(err.item()) == 0, f"device error flags {int(err.item())}"
 
+    def seg_block():
+        seg_prefix(); seg_steps(); seg_commit()
+
     st = torch.cuda.Stream(dev)
     st.wait_stream(torch.cuda.current_stream(dev))
     graphs = []
     with torch.cuda.stream(st):
-        for fn in (seg_prefix, seg_steps, seg_commit, seg_recompute):
+        for fn in (seg_block, seg_prefix, seg_steps, seg_commit, seg_recompute):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=st, capture_error_mode="thread_local"):
                 fn()
             graphs.append(g)
     torch.cuda.synchronize()
-    g_pfx, g_steps, g_commit, g_recomp = graphs
+    g_block, g_pfx, g_steps, g_commit, g_recomp = graphs
 
-    def timed_blocks(n, record):
-        """n blocks, each after an L2 flush; events bracket the three segments."""
+    def timed_blocks(n):
+        """n blocks, each after an L2 flush; one graph per block between two events."""
+        evs = []
+        with torch.cuda.stream(st):
+            for _ in range(n):
+                flush.zero_()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e[0].record(st)
+                g_block.replay()
+                e[1].record(st)
+                evs.append(e)
+        return evs
+
+    def segment_blocks(n):
+        """Per-segment breakdown: the same block as three graphs with events between."""
         evs = []
         with torch.cuda.stream(st):
             for _ in range(n):
@@ -323,20 +371,22 @@ def run_ours(args, wl, rank, world, local):
                 evs.append(e)
         return evs
 
-    timed_blocks(args.warmup, False)
+    timed_blocks(args.warmup)
     barrier(world)
     clocks = ClockSampler(local)
     clocks.start()
     barrier(world)
-    evs = timed_blocks(args.steps, True)
+    evs = timed_blocks(args.steps)
     barrier(world)
     clock_info = clocks.stop()
-    t_blocks = [e[0].elapsed_time(e[3]) for e in evs]
-    t_pfx = [e[0].elapsed_time(e[1]) for e in evs]
-    t_steps = [e[1].elapsed_time(e[2]) for e in evs]
-    t_commit = [e[2].elapsed_time(e[3]) for e in evs]
+    t_blocks = [e[0].elapsed_time(e[1]) for e in evs]
     total_ms = max_over_ranks(sum(t_blocks), world)
     assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+    sevs = segment_blocks(max(3, args.steps))
+    torch.cuda.synchronize()
+    t_pfx = [e[0].elapsed_time(e[1]) for e in sevs]
+    t_steps = [e[1].elapsed_time(e[2]) for e in sevs]
+    t_commit = [e[2].elapsed_time(e[3]) for e in sevs]
 
     # recompute-every-step schedule, same flush discipline
     rec = []
@@ -400,8 +450,11 @@ def run_ours(args, wl, rank, world, local):
     dom = max(units, key=lambda k: units[k][0])
     _, dom_bytes, dom_launch_ms, _ = units[dom]
     achieved = dom_bytes / (dom_launch_ms * 1e-3) / 1e9
+    tr = measured_traffic(API_KERNEL[dom], wl.name)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
-                "frac": achieved / hbm_gbs, "traffic": None, "kernel": dom,
+                "frac": achieved / hbm_gbs, "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                "traffic_source": tr["profile"] if tr else "no ncu capture of the current kernel source",
+                "kernel": dom,
                 "peak_kind": f"{peak_kind} hbm_gbs",
                 "algorithmic_bytes_per_launch": dom_bytes, "launch_us": dom_launch_ms * 1e3}
     pfx_gbs = kv_bytes / (pfx_ms * 1e-3) / 1e9
@@ -415,7 +468,10 @@ def run_ours(args, wl, rank, world, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": wl.name, "description": wl.description,
-                   "bench_step": f"one block: prefix state once + {S} denoising steps + commit",
+                   "bench_step": f"one block: prefix state once + {S} denoising steps + commit, "
+                                 "one CUDA graph per block",
+                   "breakdown": "prefix_partial.us / step_us / commit_us from the same block run as three "
+                                "graphs with events between (includes graph-launch gaps)",
                    "l2": "flushed (2x L2 memset) before every timed block, outside the events",
                    "parallelism": "replicas" if world > 1 else "single GPU",
                    "schedule": "reuse (prefix state computed once per block)"},
@@ -436,7 +492,7 @@ def run_ours(args, wl, rank, world, local):
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graphs, g_pfx, g_steps, g_commit, g_recomp
+    del graphs, g_block, g_pfx, g_steps, g_commit, g_recomp
 
 
 def main():

@@ -16,13 +16,13 @@
 // (cp.async for block K/V and query rows, register loads for the prefix
 // state), the RoPE cos/sin table is computed while those requests fly, and
 // the rest runs from shared memory and registers.
-//  * FBK_BF16: a CTA holds one (sequence, kv-head) unit, up to 128 query rows
-//    (all G heads of the group share the staged K/V), and each warp owns 16
-//    rows: S = Q^ K^T and O = P~ V are warp-level bf16 tensor-core MMAs
-//    (mma.sync m16n8k16, fp32 accumulation; at 16 x B x d per warp these
-//    products are far too small for the TMEM/tcgen05 machinery to pay off),
-//    the softmax runs on the accumulator fragments with quad shuffles, and P~
-//    is re-packed in registers as the A operand of the second MMA.
+//  * FBK_BF16: a CTA holds 16 query rows of one (sequence, kv-head) unit and
+//    that unit's block K/V; its 4 warps split the keys of S = Q^ K^T and the
+//    columns of O = P~ V, which are warp-level bf16 tensor-core MMAs
+//    (mma.sync m16n8k16, fp32 accumulation; at 16 x B x d these products are
+//    far too small for the TMEM/tcgen05 machinery to pay off). Many small
+//    CTAs keep the per-warp chain of dependent steps short, which is what a
+//    step's latency is made of.
 //  * FBK_FP32_CHECK: the same steps on CUDA cores in fp32 (no bf16 rounding of
 //    Q^, K^ or P~): lane j scores keys j and j + 32, warp-shuffle row max/sum.
 #include "launch.h"
@@ -32,8 +32,6 @@ namespace fbk {
 namespace {
 
 // ====================================================================== bf16 (tensor cores)
-
-constexpr int MMA_MAX_ROWS = 128;  // query rows per CTA (8 warps x 16)
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
                                         uint32_t &r3) {
@@ -64,108 +62,134 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-template <int D>
-struct MmaLayout {  // byte offsets in shared memory
-  static constexpr int RS = D * 2 + 16;  // padded bf16 row: ldmatrix rows hit distinct banks
-  int ks, vs, qs, cs, bytes;
-  __host__ __device__ MmaLayout(int blk) {
-    const int bpad = (blk + 15) & ~15;
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t &r0, uint32_t &r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
+constexpr int STEP_ROWS = 16;   // query rows of one row tile: one m16 MMA tile
+constexpr int STEP_WARPS = 4;   // warps per row tile: they split the keys of S and the columns of O
+
+template <int D, int RT>
+struct StepLayout {  // byte offsets in shared memory, all 16-byte aligned; RT row tiles per CTA
+  static constexpr int RS = D * 2 + 16;  // padded bf16 row: the 8 rows of an ldmatrix hit distinct banks
+  int bpad, ps_stride, ks, vs, qs, ps, red, cs, bytes;
+  __host__ __device__ StepLayout(int blk) {
+    bpad = (blk + 15) & ~15;
+    ps_stride = bpad * 2 + 16;
     ks = 0;
     vs = ks + bpad * RS;
     qs = vs + bpad * RS;
-    cs = qs + MMA_MAX_ROWS * RS;
+    ps = qs + RT * STEP_ROWS * RS;
+    red = ps + RT * STEP_ROWS * ps_stride;               // [2][RT][STEP_WARPS][STEP_ROWS] fp32
+    cs = red + 2 * RT * STEP_WARPS * STEP_ROWS * 4;      // [blk][D/2] (cos, sin)
     bytes = cs + blk * (D / 2) * 8;
   }
 };
 
-template <int D>
-__global__ void __launch_bounds__(256) block_merge_mma_kernel(
+// bf16 step kernel: one CTA per (unit, RT tiles of 16 query rows), 4 warps
+// per row tile; the CTA stages the unit's block K/V and RoPE table once for
+// all its row tiles.
+//
+// RoPE at block offsets. The block's queries and keys sit at L_b + t. A score
+// depends on the two positions only through their difference (RoPE's
+// rotation matrices compose: R(a)^T R(b) = R(b - a)), so rotating Q and K at t
+// alone gives the same scores exactly in real arithmetic; only the rounding
+// of the rotated bf16 operands differs. The cos/sin table then depends on the
+// kernel parameters only and is built before the kernel waits for its
+// predecessor; prefix_lens is not needed on this path.
+//
+// Warp w of a row tile computes S for the key n-tiles w and w + 4 (8 keys
+// each), the row max and sum are combined across the tile's warps through
+// shared memory, P~ goes to shared memory as bf16, and warp w then forms
+// O~2 = P~ V and the merged, normalised output for its D/4 columns.
+template <int D, int RT>
+__global__ void __launch_bounds__(RT * STEP_WARPS * 32) block_merge_mma_kernel(
     Geometry g, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kb,
     const __nv_bfloat16 *__restrict__ vb, fbk_partial pfx, __nv_bfloat16 *__restrict__ out,
-    float *__restrict__ lse) {
-  constexpr int HALF = D / 2, CH = D / 8, NTO = D / 8, RS = MmaLayout<D>::RS;
+    float *__restrict__ lse, int tiles) {
+  constexpr int CTA_ROWS = RT * STEP_ROWS, NTHREADS = RT * STEP_WARPS * 32;
+  constexpr int HALF = D / 2, CH = D / 8, RS = StepLayout<D, RT>::RS;
+  constexpr int COLS_W = D / STEP_WARPS, NTW = COLS_W / 8;  // output columns (n-tiles) per warp
   extern __shared__ float4 smem_f4[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(smem_f4);
-  const int blk = g.blk, bpad = (blk + 15) & ~15;
-  const MmaLayout<D> lay(blk);
-  uint8_t *Ks = sm + lay.ks, *Vs = sm + lay.vs, *Qs = sm + lay.qs;
+  const int blk = g.blk;
+  const StepLayout<D, RT> lay(blk);
+  const int bpad = lay.bpad, NT = bpad / 8, PSS = lay.ps_stride;
+  uint8_t *Ks = sm + lay.ks, *Vs = sm + lay.vs, *Qs = sm + lay.qs, *Ps = sm + lay.ps;
+  float *red_max = reinterpret_cast<float *>(sm + lay.red);
+  float *red_sum = red_max + RT * STEP_WARPS * STEP_ROWS;
   float2 *cs = reinterpret_cast<float2 *>(sm + lay.cs);
 
-  const int u = blockIdx.y, b = u / g.hkv, kvh = u % g.hkv;
-  const int r0 = blockIdx.x * MMA_MAX_ROWS;
-  const int rows_cta = min(MMA_MAX_ROWS, g.rows - r0);
-  const int nthreads = blockDim.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // this thread's RoPE frequency (kernel parameters only: before the wait)
-  const double rope_f = freq_over_pi(tid % HALF, D, g.log2_base);
+  const int u = blockIdx.x / tiles, r0 = (blockIdx.x % tiles) * CTA_ROWS;
+  const int b = u / g.hkv, kvh = u % g.hkv;
+  const int rows_cta = min(CTA_ROWS, g.rows - r0);
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int grp = tid >> 7, warp = (tid >> 5) & 3;  // row tile of the CTA, warp inside the tile
+
+  // ---- 0. cos/sin of t * theta_i, t < B (kernel parameters only), in fp32:
+  // the angle in turns, reduced to [-1, 1], then the fast sine/cosine. At
+  // t <= 63 the absolute error stays near 1e-5 rad, far below the bf16
+  // rounding of the rotated operands.
+  {
+    const int i = tid % HALF;
+    const float f = exp2f(-2.0f * (float)i / (float)D * (float)g.log2_base) * (float)(1.0 / CUDART_PI);
+    for (int t = tid / HALF; t < blk; t += NTHREADS / HALF) {
+      float x = (float)t * f;
+      x -= 2.0f * rintf(0.5f * x);
+      float sn, c;
+      __sincosf(x * (float)CUDART_PI, &sn, &c);
+      cs[t * HALF + i] = make_float2(c, sn);
+    }
+  }
   pdl_release();
   pdl_wait();
-  int L = g.lens[b];
-  if (L < 0) {
-    raise_flag(g, FBK_DEVERR_PREFIX_LEN);
-    L = 0;
-  }
 
   // ---- 1. every global read of the CTA, issued at once
   const long long kv_row0 = (long long)b * blk * g.hkv + kvh;  // token t: row kv_row0 + t*hkv
-  for (int idx = tid; idx < blk * CH; idx += nthreads) {
+  for (int idx = tid; idx < blk * CH; idx += NTHREADS) {
     const int t = idx / CH, c = idx % CH;
     const long long src = (kv_row0 + (long long)t * g.hkv) * D + c * 8;
     cp_async16(Ks + t * RS + c * 16, kb + src);
     cp_async16(Vs + t * RS + c * 16, vb + src);
   }
-  for (int idx = tid; idx < rows_cta * CH; idx += nthreads) {
+  for (int idx = tid; idx < rows_cta * CH; idx += NTHREADS) {
     const int rr = idx / CH, c = idx % CH, r = r0 + rr;
     const int t = r % blk, h = kvh * g.group + r / blk;
     cp_async16(Qs + rr * RS + c * 16, q + (((long long)b * blk + t) * g.hq + h) * D + c * 8);
   }
-  // padding key rows must be finite zeros (they meet P~ = 0 in the PV product)
-  for (int idx = tid; idx < (bpad - blk) * CH; idx += nthreads) {
+  // padding key rows and query rows must be finite zeros
+  for (int idx = tid; idx < (bpad - blk) * CH; idx += NTHREADS) {
     const int t = blk + idx / CH, c = idx % CH;
     *reinterpret_cast<uint4 *>(Ks + t * RS + c * 16) = make_uint4(0, 0, 0, 0);
     *reinterpret_cast<uint4 *>(Vs + t * RS + c * 16) = make_uint4(0, 0, 0, 0);
   }
-  const int nw_rows = (rows_cta + 15) / 16;
-  for (int idx = tid; idx < (nw_rows * 16 - rows_cta) * CH; idx += nthreads) {
+  for (int idx = tid; idx < (CTA_ROWS - rows_cta) * CH; idx += NTHREADS) {
     const int rr = rows_cta + idx / CH, c = idx % CH;
     *reinterpret_cast<uint4 *>(Qs + rr * RS + c * 16) = make_uint4(0, 0, 0, 0);
   }
-  // this thread's two accumulator rows and their prefix state (registers)
-  const int lr = lane >> 2, lc = (lane & 3) * 2;
-  const int ra = r0 + warp * 16 + lr, rb = ra + 8;
-  const bool va = warp < nw_rows && ra < g.rows, vbr = warp < nw_rows && rb < g.rows;
+  // this thread's outputs: rows lr and lr + 8 of its row tile, columns col0 + 8j + lc (+1)
+  const int lr = lane >> 2, lc = (lane & 3) * 2, col0 = warp * COLS_W, tr0 = grp * STEP_ROWS;
+  const int ra = r0 + tr0 + lr, rb = ra + 8;
+  const bool va = tr0 + lr < rows_cta, vbr = tr0 + lr + 8 < rows_cta;
   const int ta = va ? ra % blk : 0, ha = va ? kvh * g.group + ra / blk : 0;
   const int tb_ = vbr ? rb % blk : 0, hb = vbr ? kvh * g.group + rb / blk : 0;
   const long long pa = ((long long)b * g.hq + ha) * blk + ta, pb = ((long long)b * g.hq + hb) * blk + tb_;
-  float2 o1a[NTO], o1b[NTO];
+  float2 o1a[NTW], o1b[NTW];
   float m1a = -CUDART_INF_F, l1a = 0.f, m1b = -CUDART_INF_F, l1b = 0.f;
 #pragma unroll
-  for (int j = 0; j < NTO; ++j) {
-    o1a[j] = va ? __ldg(reinterpret_cast<const float2 *>(pfx.o_unnorm + pa * D + 8 * j + lc)) : make_float2(0.f, 0.f);
-    o1b[j] = vbr ? __ldg(reinterpret_cast<const float2 *>(pfx.o_unnorm + pb * D + 8 * j + lc)) : make_float2(0.f, 0.f);
+  for (int j = 0; j < NTW; ++j) {
+    o1a[j] = va ? __ldg(reinterpret_cast<const float2 *>(pfx.o_unnorm + pa * D + col0 + 8 * j + lc))
+                : make_float2(0.f, 0.f);
+    o1b[j] = vbr ? __ldg(reinterpret_cast<const float2 *>(pfx.o_unnorm + pb * D + col0 + 8 * j + lc))
+                 : make_float2(0.f, 0.f);
   }
   if (va) { m1a = __ldg(pfx.m + pa); l1a = __ldg(pfx.l + pa); }
   if (vbr) { m1b = __ldg(pfx.m + pb); l1b = __ldg(pfx.l + pb); }
-
-  // ---- 2. RoPE cos/sin of positions L .. L+B-1 while the copies fly: each
-  // thread keeps one frequency i; cos/sin(L theta_i) is fp64-reduced, and the
-  // offset t theta_i (t < 64) is added by angle addition in fp32 (abs error
-  // ~1e-5, far below the bf16 rounding of Q^ and K^ that follows).
-  {
-    const int i = tid % HALF;
-    const double f = rope_f;
-    const float2 cl = rope_cs_fast(L, f);
-    const float th = (float)(f * CUDART_PI);
-    for (int t = tid / HALF; t < blk; t += nthreads / HALF) {
-      float st, ct;
-      __sincosf((float)t * th, &st, &ct);
-      cs[t * HALF + i] = make_float2(cl.x * ct - cl.y * st, cl.y * ct + cl.x * st);
-    }
-  }
   cp_async_wait_all();
   __syncthreads();
 
-  // ---- 3. rotate block K and the query rows in place (bf16), 8 pairs per item
-  for (int idx = tid; idx < (blk + rows_cta) * (D / 16); idx += nthreads) {
+  // ---- 2. rotate block K and the query rows in place at their block offsets, 8 pairs per item
+  for (int idx = tid; idx < (blk + rows_cta) * (D / 16); idx += NTHREADS) {
     const int rowi = idx / (D / 16), c = idx % (D / 16);
     const bool is_k = rowi < blk;
     const int t = is_k ? rowi : (r0 + rowi - blk) % blk;
@@ -187,85 +211,113 @@ __global__ void __launch_bounds__(256) block_merge_mma_kernel(
     *p2 = make_uint4(y2[0], y2[1], y2[2], y2[3]);
   }
   __syncthreads();
-  if (warp >= nw_rows) return;
 
-  // ---- 4. S = Q^ K^T for this warp's 16 rows (up to 64 keys: 8 n-tiles)
-  const uint32_t qs_a = (uint32_t)__cvta_generic_to_shared(Qs), ks_a = (uint32_t)__cvta_generic_to_shared(Ks),
-                 vs_a = (uint32_t)__cvta_generic_to_shared(Vs);
-  float sacc[8][4];
+  // ---- 3. S = Q^ K^T for key n-tiles warp and warp + 4 (16 rows x 8 keys each)
+  const uint32_t qs_a = (uint32_t)__cvta_generic_to_shared(Qs + tr0 * RS),
+                 ks_a = (uint32_t)__cvta_generic_to_shared(Ks), vs_a = (uint32_t)__cvta_generic_to_shared(Vs),
+                 ps_a = (uint32_t)__cvta_generic_to_shared(Ps + tr0 * PSS);
+  uint8_t *Pt = Ps + tr0 * PSS;  // this row tile's P~
+  float *rmax = red_max + grp * STEP_WARPS * STEP_ROWS, *rsum = red_sum + grp * STEP_WARPS * STEP_ROWS;
+  const int a_row = (lane & 7) + 8 * ((lane >> 3) & 1), a_col = 8 * (lane >> 4);  // A fragments (16x16)
+  const int b_row = lane & 7, b_col = 8 * ((lane >> 3) & 1);                      // B fragment (k16 x n8)
+  float sacc[2][4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
-  const int a_row = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1), a_col = 8 * (lane >> 4);
-  const int b_row = (lane & 7) + 8 * (lane >> 4), b_col = 8 * ((lane >> 3) & 1);
+  for (int e = 0; e < 2; ++e) sacc[e][0] = sacc[e][1] = sacc[e][2] = sacc[e][3] = 0.f;
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     uint32_t a0, a1, a2, a3;
     ldsm_x4(qs_a + a_row * RS + (16 * kk + a_col) * 2, a0, a1, a2, a3);
 #pragma unroll
-    for (int jp = 0; jp < 4; ++jp) {
-      if (16 * jp < bpad) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(ks_a + (16 * jp + b_row) * RS + (16 * kk + b_col) * 2, b0, b1, b2, b3);
-        mma16816(sacc[2 * jp], a0, a1, a2, a3, b0, b1);
-        mma16816(sacc[2 * jp + 1], a0, a1, a2, a3, b2, b3);
+    for (int e = 0; e < 2; ++e) {
+      const int nt = warp + STEP_WARPS * e;
+      if (nt < NT) {
+        uint32_t b0, b1;
+        ldsm_x2(ks_a + (8 * nt + b_row) * RS + (16 * kk + b_col) * 2, b0, b1);
+        mma16816(sacc[e], a0, a1, a2, a3, b0, b1);
       }
     }
   }
 
-  // ---- 5. block softmax on the fragments (rows lr and lr + 8 of the warp tile)
+  // ---- 4. block softmax across the 4 warps (log2 units)
   const float sl2 = g.tau * 1.4426950408889634f;
   float mxa = -CUDART_INF_F, mxb = -CUDART_INF_F;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int e = 0; e < 2; ++e) {
+    const int nt = warp + STEP_WARPS * e;
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const bool ok = 8 * j + lc + e < blk;
-      sacc[j][e] = ok ? sacc[j][e] * sl2 : -CUDART_INF_F;
-      sacc[j][2 + e] = ok ? sacc[j][2 + e] * sl2 : -CUDART_INF_F;
-      mxa = fmaxf(mxa, sacc[j][e]);
-      mxb = fmaxf(mxb, sacc[j][2 + e]);
+    for (int c = 0; c < 2; ++c) {
+      const bool ok = nt < NT && 8 * nt + lc + c < blk;
+      sacc[e][c] = ok ? sacc[e][c] * sl2 : -CUDART_INF_F;
+      sacc[e][2 + c] = ok ? sacc[e][2 + c] * sl2 : -CUDART_INF_F;
+      mxa = fmaxf(mxa, sacc[e][c]);
+      mxb = fmaxf(mxb, sacc[e][2 + c]);
     }
   }
   mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
   mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
   mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
   mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
-  float sa = 0.f, sbs = 0.f;
-  uint32_t pa_frag[8], pb_frag[8];  // P~ as bf16 pairs: [n-tile] for rows lr and lr + 8
+  if ((lane & 3) == 0) {
+    rmax[warp * STEP_ROWS + lr] = mxa;
+    rmax[warp * STEP_ROWS + lr + 8] = mxb;
+  }
+  __syncthreads();
+  mxa = mxb = -CUDART_INF_F;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float p0 = tc::ex2(sacc[j][0] - mxa), p1 = tc::ex2(sacc[j][1] - mxa);
-    const float p2 = tc::ex2(sacc[j][2] - mxb), p3 = tc::ex2(sacc[j][3] - mxb);
-    sa += p0 + p1;
-    sbs += p2 + p3;
-    pa_frag[j] = pack2(p0, p1);
-    pb_frag[j] = pack2(p2, p3);
+  for (int w = 0; w < STEP_WARPS; ++w) {
+    mxa = fmaxf(mxa, rmax[w * STEP_ROWS + lr]);
+    mxb = fmaxf(mxb, rmax[w * STEP_ROWS + lr + 8]);
+  }
+  float sa = 0.f, sbs = 0.f;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int nt = warp + STEP_WARPS * e;
+    if (nt < NT) {
+      const float p0 = tc::ex2(sacc[e][0] - mxa), p1 = tc::ex2(sacc[e][1] - mxa);
+      const float p2 = tc::ex2(sacc[e][2] - mxb), p3 = tc::ex2(sacc[e][3] - mxb);
+      sa += p0 + p1;
+      sbs += p2 + p3;
+      *reinterpret_cast<uint32_t *>(Pt + lr * PSS + (8 * nt + lc) * 2) = pack2(p0, p1);
+      *reinterpret_cast<uint32_t *>(Pt + (lr + 8) * PSS + (8 * nt + lc) * 2) = pack2(p2, p3);
+    }
   }
   sa += __shfl_xor_sync(0xffffffffu, sa, 1);
   sa += __shfl_xor_sync(0xffffffffu, sa, 2);
   sbs += __shfl_xor_sync(0xffffffffu, sbs, 1);
   sbs += __shfl_xor_sync(0xffffffffu, sbs, 2);
-
-  // ---- 6. O~2 = P~ V
-  float oacc[NTO][4];
+  if ((lane & 3) == 0) {
+    rsum[warp * STEP_ROWS + lr] = sa;
+    rsum[warp * STEP_ROWS + lr + 8] = sbs;
+  }
+  __syncthreads();
+  sa = sbs = 0.f;
 #pragma unroll
-  for (int j = 0; j < NTO; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
+  for (int w = 0; w < STEP_WARPS; ++w) {
+    sa += rsum[w * STEP_ROWS + lr];
+    sbs += rsum[w * STEP_ROWS + lr + 8];
+  }
+
+  // ---- 5. O~2 = P~ V for this warp's columns
+  float oacc[NTW][4];
+#pragma unroll
+  for (int j = 0; j < NTW; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
   const int v_row = (lane & 7) + 8 * ((lane >> 3) & 1), v_col = 8 * (lane >> 4);
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk) {
     if (16 * kk < bpad) {
-      const uint32_t a0 = pa_frag[2 * kk], a1 = pb_frag[2 * kk], a2 = pa_frag[2 * kk + 1], a3 = pb_frag[2 * kk + 1];
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(ps_a + a_row * PSS + (16 * kk + a_col) * 2, a0, a1, a2, a3);
 #pragma unroll
-      for (int jp = 0; jp < D / 16; ++jp) {
+      for (int jp = 0; jp < NTW / 2; ++jp) {
         uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vs_a + (16 * kk + v_row) * RS + (16 * jp + v_col) * 2, b0, b1, b2, b3);
+        ldsm_x4_t(vs_a + (16 * kk + v_row) * RS + (col0 + 16 * jp + v_col) * 2, b0, b1, b2, b3);
         mma16816(oacc[2 * jp], a0, a1, a2, a3, b0, b1);
         mma16816(oacc[2 * jp + 1], a0, a1, a2, a3, b2, b3);
       }
     }
   }
 
-  // ---- 7. merge with the prefix state, normalise, store
+  // ---- 6. merge with the prefix state, normalise, store
   const float LN2 = 0.6931471805599453f;
   const float m2a = mxa * LN2, m2b = mxb * LN2;
   const float Ma = fmaxf(m1a, m2a), Mb = fmaxf(m1b, m2b);
@@ -273,10 +325,10 @@ __global__ void __launch_bounds__(256) block_merge_mma_kernel(
   const float w1b = lse_weight(m1b, Mb), w2b = expf(m2b - Mb);
   const float lta = w1a * l1a + w2a * sa, ltb = w1b * l1b + w2b * sbs;
   const float ia = 1.f / lta, ib = 1.f / ltb;
-  __nv_bfloat16 *da = out + (((long long)b * blk + ta) * g.hq + ha) * D + lc;
-  __nv_bfloat16 *db = out + (((long long)b * blk + tb_) * g.hq + hb) * D + lc;
+  __nv_bfloat16 *da = out + (((long long)b * blk + ta) * g.hq + ha) * D + col0 + lc;
+  __nv_bfloat16 *db = out + (((long long)b * blk + tb_) * g.hq + hb) * D + col0 + lc;
 #pragma unroll
-  for (int j = 0; j < NTO; ++j) {
+  for (int j = 0; j < NTW; ++j) {
     if (va)
       *reinterpret_cast<uint32_t *>(da + 8 * j) = pack2((w1a * o1a[j].x + w2a * oacc[j][0]) * ia,
                                                         (w1a * o1a[j].y + w2a * oacc[j][1]) * ia);
@@ -284,27 +336,47 @@ __global__ void __launch_bounds__(256) block_merge_mma_kernel(
       *reinterpret_cast<uint32_t *>(db + 8 * j) = pack2((w1b * o1b[j].x + w2b * oacc[j][2]) * ib,
                                                         (w1b * o1b[j].y + w2b * oacc[j][3]) * ib);
   }
-  if (lse && (lane & 3) == 0) {
+  if (lse && warp == 0 && (lane & 3) == 0) {
     if (va) lse[pa] = Ma + logf(lta);
     if (vbr) lse[pb] = Mb + logf(ltb);
   }
 }
 
-template <int D>
-cudaError_t launch_mma(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
-                       const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
-                       cudaStream_t st) {
-  const MmaLayout<D> lay(g.blk);
-  auto kern = block_merge_mma_kernel<D>;
+template <int D, int RT>
+cudaError_t launch_mma_rt(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
+                          const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
+                          cudaStream_t st) {
+  const StepLayout<D, RT> lay(g.blk);
+  auto kern = block_merge_mma_kernel<D, RT>;
   if (lay.bytes > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.bytes);
     if (e != cudaSuccess) return e;
   }
-  // 8 warps always: all of them load, build the RoPE table and rotate; only
-  // those that own query rows go on to the tensor-core part.
-  dim3 grid((g.rows + MMA_MAX_ROWS - 1) / MMA_MAX_ROWS, g.batch * g.hkv);
-  return launch_pdl(kern, grid, dim3(256), lay.bytes, st, g, q, kb, vb, pfx,
-                    static_cast<__nv_bfloat16 *>(out), lse);
+  const int tiles = (g.rows + RT * STEP_ROWS - 1) / (RT * STEP_ROWS);
+  const long long ctas = (long long)g.batch * g.hkv * tiles;
+  if (ctas > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+  return launch_pdl(kern, dim3((unsigned)ctas), dim3(RT * STEP_WARPS * 32), lay.bytes, st, g, q, kb, vb, pfx,
+                    static_cast<__nv_bfloat16 *>(out), lse, tiles);
+}
+
+// Row tiles per CTA: the largest RT in {1, 2, 4} that still gives at least
+// one CTA per SM, so that big batches share each staged K/V and RoPE table
+// among more rows while small ones keep the most CTAs (and the shortest chain).
+template <int D>
+cudaError_t launch_mma(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
+                       const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
+                       cudaStream_t st) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long units = (long long)g.batch * g.hkv, t16 = (g.rows + STEP_ROWS - 1) / STEP_ROWS;
+  int rt = 1;
+  for (int c = 4; c > 1; c >>= 1)
+    if (c <= t16 && units * ((t16 + c - 1) / c) >= sms) { rt = c; break; }
+  switch (rt) {
+    case 4: return launch_mma_rt<D, 4>(g, q, kb, vb, pfx, out, lse, st);
+    case 2: return launch_mma_rt<D, 2>(g, q, kb, vb, pfx, out, lse, st);
+    default: return launch_mma_rt<D, 1>(g, q, kb, vb, pfx, out, lse, st);
+  }
 }
 
 // ====================================================================== fp32 check (CUDA cores)

@@ -10,6 +10,8 @@
 // (hardware, no spinning) guarantees all reads happened, and only then does
 // CTA 0 advance prefix_lens[b]. The fp64 cos/sin of each (position, pair)
 // are computed once per CTA into shared memory and reused by all kv-heads.
+// The block K/V loads of the first batch are issued before the length is
+// read, so the two memory round trips overlap.
 #include <cooperative_groups.h>
 
 #include "launch.h"
@@ -19,68 +21,86 @@ namespace {
 
 namespace cg = cooperative_groups;
 
-constexpr int THREADS = 256;
+constexpr int THREADS = 512;
 constexpr int CLUSTER = 8;
 constexpr int MAX_TOK = 64 / CLUSTER;  // block_len <= 64
+constexpr int KB = 2;                  // K items (8 rotation pairs) per thread per batch
+constexpr int VB = 4;                  // V 16-byte chunks per thread per batch
 
 template <int D>
 __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(THREADS)
     commit_kernel(Geometry g, const __nv_bfloat16 *__restrict__ kb, const __nv_bfloat16 *__restrict__ vb,
                   __nv_bfloat16 *__restrict__ kc, __nv_bfloat16 *__restrict__ vc, int *lens) {
-  constexpr int HALF = D / 2;
+  constexpr int HALF = D / 2, KI = D / 16, VI = D / 8;
   __shared__ int s_ok, s_L;
   __shared__ double2 tab[MAX_TOK * HALF];
   const int b = blockIdx.y, crank = blockIdx.x, blk = g.blk;
   const int t0 = crank * blk / CLUSTER, t1 = (crank + 1) * blk / CLUSTER, nt = t1 - t0;
+  const int nk = nt * g.hkv * KI, nv = nt * g.hkv * VI;
   pdl_release();
   pdl_wait();
-  if (threadIdx.x == 0) {
-    const int L = lens[b];
-    bool ok = L >= 0 && (long long)L + blk <= seq_capacity(g);
-    if (ok && g.paged) {
-      for (long long pg = (long long)L >> g.page_shift; pg <= ((long long)L + blk - 1) >> g.page_shift; ++pg) {
-        const int id = g.page_table[(long long)b * g.max_pages + pg];
-        if (id < 0 || (long long)id >= g.num_pages) ok = false;
-      }
-      if (!ok && crank == 0) raise_flag(g, FBK_DEVERR_PAGE_ID);
-    }
-    if (!ok && crank == 0) raise_flag(g, FBK_DEVERR_COMMIT);
-    s_ok = ok;
-    s_L = L;
-  }
-  cg::this_cluster().sync();  // every CTA of this sequence has read prefix_lens[b]
-  const bool ok = s_ok;
-  const int L = s_L;
-  if (ok && crank == 0 && threadIdx.x == 0) lens[b] = L + blk;
-  if (!ok || nt == 0) return;
 
-  for (int idx = threadIdx.x; idx < nt * HALF; idx += THREADS) {
-    double c, s;
-    rope_cs_f64(L + t0 + idx / HALF, g.inv_freq_over_pi[idx % HALF], &c, &s);
-    tab[idx] = make_double2(c, s);
-  }
-  __syncthreads();
-
-  // K: an item is 8 rotation pairs, i.e. the 16-byte chunk c of each half of a
-  // row; every load of a batch is issued before the first use.
-  const int nk = nt * g.hkv * (D / 16);
-  for (int base = 0; base < nk; base += THREADS * 4) {
-    uint4 xa[4], xb[4];
+  int L = 0;
+  bool first = true;
+  for (int kbase = 0, vbase = 0; first || kbase < nk || vbase < nv; kbase += THREADS * KB, vbase += THREADS * VB) {
+    // block K and V do not depend on L: the first batch is requested before the
+    // length is known, so both round trips overlap
+    uint4 xa[KB], xb[KB], xv[VB];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int item = base + threadIdx.x + THREADS * k;
+    for (int k = 0; k < KB; ++k) {
+      const int item = kbase + threadIdx.x + THREADS * k;
       if (item < nk) {
-        const int c = item % (D / 16), rowi = item / (D / 16), kvh = rowi % g.hkv, t = t0 + rowi / g.hkv;
+        const int c = item % KI, rowi = item / KI, kvh = rowi % g.hkv, t = t0 + rowi / g.hkv;
         const uint4 *src = reinterpret_cast<const uint4 *>(kb + (((long long)b * blk + t) * g.hkv + kvh) * D);
         xa[k] = src[c];
-        xb[k] = src[c + D / 16];
+        xb[k] = src[c + KI];
       }
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int item = base + threadIdx.x + THREADS * k;
+    for (int k = 0; k < VB; ++k) {
+      const int item = vbase + threadIdx.x + THREADS * k;
+      if (item < nv) {
+        const int ch = item % VI, rowi = item / VI, kvh = rowi % g.hkv, t = t0 + rowi / g.hkv;
+        xv[k] = reinterpret_cast<const uint4 *>(vb + (((long long)b * blk + t) * g.hkv + kvh) * D)[ch];
+      }
+    }
+    if (first) {
+      first = false;
+      if (threadIdx.x == 0) {
+        const int Lb = lens[b];
+        bool ok = Lb >= 0 && (long long)Lb + blk <= seq_capacity(g);
+        if (ok && g.paged) {
+          for (long long pg = (long long)Lb >> g.page_shift; pg <= ((long long)Lb + blk - 1) >> g.page_shift; ++pg) {
+            const int id = g.page_table[(long long)b * g.max_pages + pg];
+            if (id < 0 || (long long)id >= g.num_pages) ok = false;
+          }
+          if (!ok && crank == 0) raise_flag(g, FBK_DEVERR_PAGE_ID);
+        }
+        if (!ok && crank == 0) raise_flag(g, FBK_DEVERR_COMMIT);
+        s_ok = ok;
+        s_L = Lb;
+      }
+      cg::this_cluster().sync();  // every CTA of this sequence has read prefix_lens[b]
+      L = s_L;
+      if (!s_ok) return;
+      if (crank == 0 && threadIdx.x == 0) lens[b] = L + blk;
+      if (nt == 0) return;
+      // entry of pair i = 8c + e sits at e * KI + c: the 8 lanes that rotate
+      // chunks c = 0..7 of one row read 8 consecutive entries (no bank conflict)
+      for (int idx = threadIdx.x; idx < nt * HALF; idx += THREADS) {
+        const int tl = idx / HALF, i = idx % HALF;
+        double c, sn;
+        rope_cs_f64(L + t0 + tl, g.inv_freq_over_pi[i], &c, &sn);
+        tab[tl * HALF + (i & 7) * KI + (i >> 3)] = make_double2(c, sn);
+      }
+      __syncthreads();
+    }
+    // K: an item is 8 rotation pairs, the 16-byte chunk c of each half of a row
+#pragma unroll
+    for (int k = 0; k < KB; ++k) {
+      const int item = kbase + threadIdx.x + THREADS * k;
       if (item < nk) {
-        const int c = item % (D / 16), rowi = item / (D / 16), kvh = rowi % g.hkv, tl = rowi / g.hkv;
+        const int c = item % KI, rowi = item / KI, kvh = rowi % g.hkv, tl = rowi / g.hkv;
         const uint32_t aw[4] = {xa[k].x, xa[k].y, xa[k].z, xa[k].w};
         const uint32_t bw[4] = {xb[k].x, xb[k].y, xb[k].z, xb[k].w};
         uint32_t y1[4], y2[4];
@@ -89,7 +109,7 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(THREADS)
           const uint32_t ha = (e & 1) ? (aw[e >> 1] >> 16) : (aw[e >> 1] & 0xffffu);
           const uint32_t hb = (e & 1) ? (bw[e >> 1] >> 16) : (bw[e >> 1] & 0xffffu);
           const double x1 = (double)bf16_bits_to_f32((uint16_t)ha), x2 = (double)bf16_bits_to_f32((uint16_t)hb);
-          const double2 cs = tab[tl * HALF + 8 * c + e];
+          const double2 cs = tab[tl * HALF + e * KI + c];
           // plain rounded products and differences (no fused multiply-add)
           const uint32_t r1 = f64_to_bf16_rne(__dsub_rn(__dmul_rn(x1, cs.x), __dmul_rn(x2, cs.y)));
           const uint32_t r2 = f64_to_bf16_rne(__dadd_rn(__dmul_rn(x2, cs.x), __dmul_rn(x1, cs.y)));
@@ -103,28 +123,16 @@ __global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(THREADS)
         }
         uint4 *dst = reinterpret_cast<uint4 *>(kc + cache_row(g, b, kvh, (long long)L + t0 + tl) * D);
         dst[c] = make_uint4(y1[0], y1[1], y1[2], y1[3]);
-        dst[c + D / 16] = make_uint4(y2[0], y2[1], y2[2], y2[3]);
+        dst[c + KI] = make_uint4(y2[0], y2[1], y2[2], y2[3]);
       }
     }
-  }
-  // V: bit-exact 16-byte copies, 8 loads in flight per thread
-  const int nv = nt * g.hkv * (D / 8);
-  for (int base = 0; base < nv; base += THREADS * 8) {
-    uint4 x[8];
+    // V: bit-exact 16-byte copies
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int item = base + threadIdx.x + THREADS * k;
+    for (int k = 0; k < VB; ++k) {
+      const int item = vbase + threadIdx.x + THREADS * k;
       if (item < nv) {
-        const int ch = item % (D / 8), rowi = item / (D / 8), kvh = rowi % g.hkv, t = t0 + rowi / g.hkv;
-        x[k] = reinterpret_cast<const uint4 *>(vb + (((long long)b * blk + t) * g.hkv + kvh) * D)[ch];
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int item = base + threadIdx.x + THREADS * k;
-      if (item < nv) {
-        const int ch = item % (D / 8), rowi = item / (D / 8), kvh = rowi % g.hkv, t = t0 + rowi / g.hkv;
-        reinterpret_cast<uint4 *>(vc + cache_row(g, b, kvh, (long long)L + t) * D)[ch] = x[k];
+        const int ch = item % VI, rowi = item / VI, kvh = rowi % g.hkv, t = t0 + rowi / g.hkv;
+        reinterpret_cast<uint4 *>(vc + cache_row(g, b, kvh, (long long)L + t) * D)[ch] = xv[k];
       }
     }
   }

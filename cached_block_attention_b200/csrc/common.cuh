@@ -207,21 +207,18 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
   return __uint_as_float(((uint32_t)h) << 16);
 }
 
-// fp64 -> bf16, one rounding to nearest even, from the IEEE encodings: keep the
-// exponent and the top 7 fraction bits of the fp64 pattern, round on the 45
-// dropped bits (a carry moves into the exponent by itself), then re-bias the
-// exponent from 1023 to 127. Values below bf16's normal range (|x| < 2^-126)
-// go through fp32.
+// fp64 -> bf16 with a single rounding to nearest even, through fp32 rounded
+// to odd (Boldo and Melquiond, "When double rounding is odd"): truncate to
+// fp32, set its last bit when the truncation was inexact, then round that fp32
+// value to nearest-even bf16. fp32 carries 16 more significand bits than bf16
+// (the method needs 2), in the normal and the subnormal range alike, since
+// both formats share the 8-bit exponent, so the two roundings give the result
+// of one.
 __device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
-  unsigned long long u = (unsigned long long)__double_as_longlong(x);
-  unsigned long long sign = u >> 63;
-  unsigned long long a = u & 0x7FFFFFFFFFFFFFFFull;
-  if (a < 0x3810000000000000ull) return __bfloat16_as_ushort(__float2bfloat16_rn((float)x));
-  unsigned long long keep = a >> 45;
-  unsigned long long rem = a & ((1ull << 45) - 1);
-  const unsigned long long half = 1ull << 44;
-  keep += (rem > half || (rem == half && (keep & 1ull))) ? 1ull : 0ull;
-  return (uint16_t)((sign << 15) | (keep - (896ull << 7)));
+  const float f = __double2float_rz(x);
+  uint32_t u = __float_as_uint(f);
+  if ((double)f != x) u |= 1u;
+  return __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(u)));
 }
 
 __device__ __forceinline__ float warp_max(float v) {

@@ -63,7 +63,10 @@ struct Cfg {
   static constexpr int B_DRAIN = B_OFREE + MT;  // [2]: S issuer, PV issuer
   static constexpr int NBAR = B_DRAIN + 2;
   static constexpr int TH_OFF = BAR_OFF + NBAR * 8;  // [D/2] double: theta_i / pi
-  static constexpr int LEN_OFF = TH_OFF + (D / 2) * 8;  // [MAX_BATCH] int: validated L_b
+  // [2][8][D/2] float2: cos/sin of b*theta_i and of 8a*theta_i (a, b < 8), so
+  // that any block offset t = 8a + b < 64 is two complex products away
+  static constexpr int TT_OFF = TH_OFF + (D / 2) * 8;
+  static constexpr int LEN_OFF = TT_OFF + 2 * 8 * (D / 2) * 8;  // [MAX_BATCH] int: validated L_b
   static constexpr int SCAN_OFF = LEN_OFF + MAX_BATCH * 4;  // [MAX_BATCH] int: tile scan
   static constexpr int MISC_OFF = SCAN_OFF + MAX_BATCH * 4;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;   // + slack to align the base to 1024
@@ -158,19 +161,29 @@ __device__ __forceinline__ void issue_q_rows(const Geometry &g, const __nv_bfloa
   }
 }
 
+// Rotates this thread's own copies in place (RoPE at L + t). Every item of a
+// thread has the same chunk c (8 pairs i = 8c + m), so the thread forms
+// cos/sin(L theta_i) for its 8 pairs once per piece, fp64-reduced, while its
+// copies are in flight; the block offset t = 8a + b then enters through two
+// complex products with the tables of b*theta_i and 8a*theta_i.
 template <int D, int MT>
 __device__ __forceinline__ void rotate_q_rows(const Geometry &g, const Piece &p, uint32_t qbase, int mt,
-                                              int wg_tid, const double *theta_tab) {
-  constexpr int CHUNKS = D / 16;
+                                              int wg_tid, const double *theta_tab, const float2 *tt) {
+  constexpr int CHUNKS = D / 16, HALF = D / 2;
   const int real_rows = min(128, g.rows - mt * 128);
+  const int c = wg_tid % CHUNKS;
+  float2 cl[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) cl[m] = rope_cs_fast(p.L, theta_tab[8 * c + m]);
   cp_async_wait_all();
 #pragma unroll
   for (int k = 0; k < CHUNKS; ++k) {
-    const int item = wg_tid + 128 * k, rr = item / CHUNKS, c = item % CHUNKS;
+    const int item = wg_tid + 128 * k, rr = item / CHUNKS;
     if (rr < real_rows) {
-      const int e1 = 8 * c, e2 = D / 2 + 8 * c, t = (mt * 128 + rr) % g.blk;
+      const int e1 = 8 * c, e2 = HALF + 8 * c, t = (mt * 128 + rr) % g.blk;
       const uint32_t a1 = qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8);
       const uint32_t a2 = qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8);
+      const float2 *t1 = tt + (t & 7) * HALF + e1, *t8 = tt + (8 + (t >> 3)) * HALF + e1;
       uint32_t aw[4], bw[4];
       ld_shared_v4(a1, aw);
       ld_shared_v4(a2, bw);
@@ -180,12 +193,14 @@ __device__ __forceinline__ void rotate_q_rows(const Geometry &g, const Piece &p,
         float y1[2], y2[2];
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
-          const int ii = e1 + 2 * e + h2;
+          const int m = 2 * e + h2;
+          const float2 u = t1[m], v = t8[m];
+          const float uc = u.x * v.x - u.y * v.y, us = u.x * v.y + u.y * v.x;  // t * theta
+          const float cs = cl[m].x * uc - cl[m].y * us, sn = cl[m].x * us + cl[m].y * uc;  // (L + t) * theta
           const float x1 = __uint_as_float(h2 ? (aw[e] & 0xffff0000u) : (aw[e] << 16));
           const float x2 = __uint_as_float(h2 ? (bw[e] & 0xffff0000u) : (bw[e] << 16));
-          const float2 cs = rope_cs_fast(p.L + t, theta_tab[ii]);
-          y1[h2] = x1 * cs.x - x2 * cs.y;
-          y2[h2] = x2 * cs.x + x1 * cs.y;
+          y1[h2] = x1 * cs - x2 * sn;
+          y2[h2] = x2 * cs + x1 * sn;
         }
         y1w[e] = pack_bf16(y1[0], y1[1]);
         y2w[e] = pack_bf16(y2[0], y2[1]);
@@ -211,23 +226,11 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
 
   int *s_len = reinterpret_cast<int *>(smem + C::LEN_OFF);
   int *s_scan = reinterpret_cast<int *>(smem + C::SCAN_OFF);
-  // kernel parameters only before the wait: tensor maps and the RoPE table
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
-  }
-  double *theta_tab = reinterpret_cast<double *>(smem + C::TH_OFF);
-  if (threadIdx.x < D / 2) theta_tab[threadIdx.x] = freq_over_pi(threadIdx.x, D, g.log2_base);
-  pdl_release();
-  pdl_wait();
-  const long long T = load_tile_scan(g, s_len, s_scan);
-  if (T == 0) return;
-  if (share_begin(blockIdx.x, T, shares) == share_begin(blockIdx.x + 1, T, shares)) return;
-
   auto bar = [&](int idx) -> uint32_t { return sb + C::BAR_OFF + 8 * idx; };
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::MISC_OFF + 4);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF);
 
+  // ---- before the wait: nothing another kernel writes is touched here
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar(C::B_KFULL + s), 1);
@@ -250,13 +253,34 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     mbar_init(bar(C::B_DRAIN + 1), 1);
     *abort_flag = 0;
     mbar_fence_init();
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  // The softmax warpgroups request their first unit's query rows now, before
-  // the producers start the K/V stream, so those few KB do not queue behind it.
+  double *theta_tab = reinterpret_cast<double *>(smem + C::TH_OFF);
+  float2 *tt = reinterpret_cast<float2 *>(smem + C::TT_OFF);
+  for (int idx = threadIdx.x; idx < 2 * 8 * (D / 2); idx += C::THREADS) {
+    const int i = idx % (D / 2), k = idx / (D / 2);  // k < 8: b = k; k >= 8: 8a with a = k - 8
+    const double f = freq_over_pi(i, D, g.log2_base);
+    if (k == 0) theta_tab[i] = f;
+    tt[idx] = rope_cs_f32(k < 8 ? k : 8 * (k - 8), f);
+  }
+  pdl_release();
+  pdl_wait();
+  fence_before_sync();
+  const long long T = load_tile_scan(g, s_len, s_scan);  // reads prefix_lens; two CTA barriers
+  fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  if (T == 0 || share_begin(blockIdx.x, T, shares) == share_begin(blockIdx.x + 1, T, shares)) {
+    if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);  // nothing was issued on it
+    return;
+  }
+
+  // The softmax warpgroups request their first unit's query rows right away;
+  // the producers start the K/V stream at the same time.
   PieceWalker sm_walk;
   Piece sm_piece;
   bool sm_more = false;
@@ -266,11 +290,6 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     if (sm_more) issue_q_rows<D, MT>(g, q, sm_piece, sb + C::Q_OFF + ((warp - 4) >> 2) * C::Q_BYTES,
                                      (warp - 4) >> 2, threadIdx.x & 127);
   }
-  fence_proxy_async();
-  fence_before_sync();
-  __syncthreads();
-  fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 || warp == 3) {
     // ---------------------------------------------------------------- producers
@@ -395,7 +414,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     while (ok && sm_more) {
       if (!first_piece) issue_q_rows<D, MT>(g, q, p, qbase, mt, wg_tid);
       first_piece = false;
-      rotate_q_rows<D, MT>(g, p, qbase, mt, wg_tid, theta_tab);
+      rotate_q_rows<D, MT>(g, p, qbase, mt, wg_tid, theta_tab, tt);
       fence_proxy_async();
       mbar_arrive(bar(C::B_QFULL + mt));
 

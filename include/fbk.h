@@ -144,7 +144,10 @@ fbk_status fbk_prefix_partial(const fbk_shape *shape, const void *q_blk, const f
  * m = max(m1, m2), lse = m + log l (LaCache App. J, initialise with cache,
  * final normalisation and logsumexp).
  *  q_blk: bf16 [b, B, Hq, d] pre-RoPE; k_blk, v_blk: bf16 [b, B, Hkv, d], K pre-RoPE.
- *  prefix_lens: int32 [b] device (positions are prefix_lens[b] + t).
+ *  prefix_lens: int32 [b] device (positions are prefix_lens[b] + t). In
+ *         FBK_BF16 mode the in-block scores depend on positions only through
+ *         their differences (RoPE), so the kernel rotates at t and does not
+ *         read prefix_lens; FBK_FP32_CHECK rotates at prefix_lens[b] + t.
  *  prefix: a state from fbk_prefix_partial (read only).
  *  out: [b, B, Hq, d], bf16 (FBK_BF16) or fp32 (FBK_FP32_CHECK).
  *  lse: fp32 [b, Hq, B] or NULL. */

@@ -236,6 +236,24 @@ def test_commit_capacity_overflow_is_flagged_and_skipped():
     assert torch.equal(cache.k[1], k_before[1])
 
 
+@pytest.mark.parametrize("mode,mname", MODES)
+def test_all_prefixes_empty(mode, mname):
+    """No sequence has a committed token: every row of the state is (0, -inf, 0),
+    the step output is plain in-block attention, and a normal call that follows
+    still works (the prefix kernels return before any tile work)."""
+    case = H.make_case(2, 8, 2, 128, 32, (0, 0), 0, 1.0, seed=90, mode=mode).upload()
+    pfx = H.run_prefix(case, case.dev["steps"][0][0])
+    torch.cuda.synchronize()
+    assert torch.isneginf(pfx.m).all() and (pfx.l == 0).all() and (pfx.o_unnorm == 0).all()
+    out, lse = H.run_step(case, pfx, 0)
+    H.assert_close(H.host_f64(out), oracle_full(case, 0)[0], mname, "empty-prefix step")
+    nxt = H.make_case(1, 4, 4, 128, 32, (300,), 0, 1.0, seed=91, mode=mode).upload()
+    got = H.partial_to_host(H.run_prefix(nxt, nxt.dev["steps"][0][0]))
+    ref = orc.prefix_partial(nxt.step_f64(0)[0], nxt.k_pfx(), nxt.v_pfx(), nxt.lens, 4, 1.0, nxt.base)
+    H.check_partial(got, ref, mname)
+    assert int(case.dev["cache"].error_flags.item()) == 0
+
+
 def test_bad_prefix_len_and_page_are_flagged_not_read():
     from cached_block_attention_b200 import fbk
     case = H.make_case(2, 4, 2, 128, 16, (100, 100), 64, 1.0, seed=81).upload()
