@@ -66,11 +66,12 @@ __device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t &r0, uint32_t &r
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
 }
 
-constexpr int STEP_ROWS = 16;   // query rows of one row tile: one m16 MMA tile
-constexpr int STEP_WARPS = 4;   // warps per row tile: they split the keys of S and the columns of O
+constexpr int STEP_ROWS = 16;  // query rows of one row tile: one m16 MMA tile
 
-template <int D, int RT>
-struct StepLayout {  // byte offsets in shared memory, all 16-byte aligned; RT row tiles per CTA
+// WPT warps per row tile (1: one warp does the whole tile; 4: the warps split
+// the keys of S and the columns of O), RT row tiles per CTA.
+template <int D, int WPT, int RT>
+struct StepLayout {  // byte offsets in shared memory, all 16-byte aligned
   static constexpr int RS = D * 2 + 16;  // padded bf16 row: the 8 rows of an ldmatrix hit distinct banks
   int bpad, ps_stride, ks, vs, qs, ps, red, cs, bytes;
   __host__ __device__ StepLayout(int blk) {
@@ -80,15 +81,14 @@ struct StepLayout {  // byte offsets in shared memory, all 16-byte aligned; RT r
     vs = ks + bpad * RS;
     qs = vs + bpad * RS;
     ps = qs + RT * STEP_ROWS * RS;
-    red = ps + RT * STEP_ROWS * ps_stride;               // [2][RT][STEP_WARPS][STEP_ROWS] fp32
-    cs = red + 2 * RT * STEP_WARPS * STEP_ROWS * 4;      // [blk][D/2] (cos, sin)
-    bytes = cs + blk * (D / 2) * 8;
+    red = ps + (WPT > 1 ? RT * STEP_ROWS * ps_stride : 0);     // P~ of each row tile (bf16)
+    cs = red + (WPT > 1 ? 2 * RT * WPT * STEP_ROWS * 4 : 0);   // [2][RT][WPT][16] fp32 max, sum
+    bytes = cs + blk * (D / 2) * 8;                           // [blk][D/2] (cos, sin)
   }
 };
 
-// bf16 step kernel: one CTA per (unit, RT tiles of 16 query rows), 4 warps
-// per row tile; the CTA stages the unit's block K/V and RoPE table once for
-// all its row tiles.
+// bf16 step kernel: one CTA per (unit, RT tiles of 16 query rows); the CTA
+// stages the unit's block K/V and RoPE table once for all its row tiles.
 //
 // RoPE at block offsets. The block's queries and keys sit at L_b + t. A score
 // depends on the two positions only through their difference (RoPE's
@@ -98,48 +98,54 @@ struct StepLayout {  // byte offsets in shared memory, all 16-byte aligned; RT r
 // kernel parameters only and is built before the kernel waits for its
 // predecessor; prefix_lens is not needed on this path.
 //
-// Warp w of a row tile computes S for the key n-tiles w and w + 4 (8 keys
-// each), the row max and sum are combined across the tile's warps through
-// shared memory, P~ goes to shared memory as bf16, and warp w then forms
-// O~2 = P~ V and the merged, normalised output for its D/4 columns.
-template <int D, int RT>
-__global__ void __launch_bounds__(RT * STEP_WARPS * 32) block_merge_mma_kernel(
+// WPT = 4: warp w of a row tile computes S for the key n-tiles w and w + 4
+// (8 keys each), the row max and sum are combined across the tile's warps
+// through shared memory, P~ goes to shared memory as bf16, and warp w then
+// forms O~2 = P~ V and the merged output for its D/4 columns. Short chains
+// per warp: the choice when there are few row tiles.
+// WPT = 1: one warp computes all of S, the softmax on the accumulator
+// fragments (quad shuffles), O~2 = P~ V with P~ re-packed in registers as the
+// A operand, and all D columns. Fewest instructions per row: the choice when
+// there are many row tiles.
+template <int D, int WPT, int RT>
+__global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
     Geometry g, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kb,
     const __nv_bfloat16 *__restrict__ vb, fbk_partial pfx, __nv_bfloat16 *__restrict__ out,
     float *__restrict__ lse, int tiles) {
-  constexpr int CTA_ROWS = RT * STEP_ROWS, NTHREADS = RT * STEP_WARPS * 32;
-  constexpr int HALF = D / 2, CH = D / 8, RS = StepLayout<D, RT>::RS;
-  constexpr int COLS_W = D / STEP_WARPS, NTW = COLS_W / 8;  // output columns (n-tiles) per warp
+  using L = StepLayout<D, WPT, RT>;
+  constexpr int CTA_ROWS = RT * STEP_ROWS, NTHREADS = RT * WPT * 32;
+  constexpr int HALF = D / 2, CH = D / 8, RS = L::RS;
+  constexpr int COLS_W = D / WPT, NTW = COLS_W / 8;  // output columns (n-tiles) per warp
   extern __shared__ float4 smem_f4[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(smem_f4);
   const int blk = g.blk;
-  const StepLayout<D, RT> lay(blk);
+  const L lay(blk);
   const int bpad = lay.bpad, NT = bpad / 8, PSS = lay.ps_stride;
   uint8_t *Ks = sm + lay.ks, *Vs = sm + lay.vs, *Qs = sm + lay.qs, *Ps = sm + lay.ps;
   float *red_max = reinterpret_cast<float *>(sm + lay.red);
-  float *red_sum = red_max + RT * STEP_WARPS * STEP_ROWS;
+  float *red_sum = red_max + RT * WPT * STEP_ROWS;
   float2 *cs = reinterpret_cast<float2 *>(sm + lay.cs);
 
   const int u = blockIdx.x / tiles, r0 = (blockIdx.x % tiles) * CTA_ROWS;
   const int b = u / g.hkv, kvh = u % g.hkv;
   const int rows_cta = min(CTA_ROWS, g.rows - r0);
   const int tid = threadIdx.x, lane = tid & 31;
-  const int grp = tid >> 7, warp = (tid >> 5) & 3;  // row tile of the CTA, warp inside the tile
+  const int grp = tid / (WPT * 32), warp = (tid >> 5) % WPT;  // row tile of the CTA, warp inside the tile
 
   // ---- 0. cos/sin of t * theta_i, t < B (kernel parameters only), in fp32:
   // the angle in turns, reduced to [-1, 1], then the fast sine/cosine. At
   // t <= 63 the absolute error stays near 1e-5 rad, far below the bf16
   // rounding of the rotated operands.
-  {
-    const int i = tid % HALF;
+  for (int idx = tid; idx < blk * HALF; idx += NTHREADS) {
+    const int t = idx / HALF, i = idx % HALF;
     const float f = exp2f(-2.0f * (float)i / (float)D * (float)g.log2_base) * (float)(1.0 / CUDART_PI);
-    for (int t = tid / HALF; t < blk; t += NTHREADS / HALF) {
-      float x = (float)t * f;
-      x -= 2.0f * rintf(0.5f * x);
-      float sn, c;
-      __sincosf(x * (float)CUDART_PI, &sn, &c);
-      cs[t * HALF + i] = make_float2(c, sn);
-    }
+    float x = (float)t * f;
+    x -= 2.0f * rintf(0.5f * x);
+    float sn, c;
+    __sincosf(x * (float)CUDART_PI, &sn, &c);
+    // pair i = 8c + 2e + h sits at float2 (t, e, c, h): the 8 lanes that rotate
+    // chunks c = 0..7 of one row read 8 consecutive float4 (no bank conflict)
+    cs[t * HALF + ((i >> 1) & 3) * (D / 8) + (i >> 3) * 2 + (i & 1)] = make_float2(c, sn);
   }
   pdl_release();
   pdl_wait();
@@ -197,11 +203,11 @@ __global__ void __launch_bounds__(RT * STEP_WARPS * 32) block_merge_mma_kernel(
     uint4 *p1 = reinterpret_cast<uint4 *>(row + c * 16), *p2 = reinterpret_cast<uint4 *>(row + D + c * 16);
     const uint4 a = *p1, bq = *p2;
     const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {bq.x, bq.y, bq.z, bq.w};
-    const float4 *cp = reinterpret_cast<const float4 *>(cs + t * HALF + 8 * c);
+    const float4 *cp = reinterpret_cast<const float4 *>(cs + t * HALF + 2 * c);  // + e * (D / 8) float2
     uint32_t y1[4], y2[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float4 c2 = cp[e];  // (cos, sin) of pairs 8c + 2e and 8c + 2e + 1
+      const float4 c2 = cp[e * (D / 16)];  // (cos, sin) of pairs 8c + 2e and 8c + 2e + 1
       const float x1l = __uint_as_float(aw[e] << 16), x1h = __uint_as_float(aw[e] & 0xffff0000u);
       const float x2l = __uint_as_float(bw[e] << 16), x2h = __uint_as_float(bw[e] & 0xffff0000u);
       y1[e] = pack2(x1l * c2.x - x2l * c2.y, x1h * c2.z - x2h * c2.w);
@@ -212,107 +218,172 @@ __global__ void __launch_bounds__(RT * STEP_WARPS * 32) block_merge_mma_kernel(
   }
   __syncthreads();
 
-  // ---- 3. S = Q^ K^T for key n-tiles warp and warp + 4 (16 rows x 8 keys each)
   const uint32_t qs_a = (uint32_t)__cvta_generic_to_shared(Qs + tr0 * RS),
-                 ks_a = (uint32_t)__cvta_generic_to_shared(Ks), vs_a = (uint32_t)__cvta_generic_to_shared(Vs),
-                 ps_a = (uint32_t)__cvta_generic_to_shared(Ps + tr0 * PSS);
-  uint8_t *Pt = Ps + tr0 * PSS;  // this row tile's P~
-  float *rmax = red_max + grp * STEP_WARPS * STEP_ROWS, *rsum = red_sum + grp * STEP_WARPS * STEP_ROWS;
+                 ks_a = (uint32_t)__cvta_generic_to_shared(Ks), vs_a = (uint32_t)__cvta_generic_to_shared(Vs);
   const int a_row = (lane & 7) + 8 * ((lane >> 3) & 1), a_col = 8 * (lane >> 4);  // A fragments (16x16)
-  const int b_row = lane & 7, b_col = 8 * ((lane >> 3) & 1);                      // B fragment (k16 x n8)
-  float sacc[2][4];
-#pragma unroll
-  for (int e = 0; e < 2; ++e) sacc[e][0] = sacc[e][1] = sacc[e][2] = sacc[e][3] = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    uint32_t a0, a1, a2, a3;
-    ldsm_x4(qs_a + a_row * RS + (16 * kk + a_col) * 2, a0, a1, a2, a3);
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int nt = warp + STEP_WARPS * e;
-      if (nt < NT) {
-        uint32_t b0, b1;
-        ldsm_x2(ks_a + (8 * nt + b_row) * RS + (16 * kk + b_col) * 2, b0, b1);
-        mma16816(sacc[e], a0, a1, a2, a3, b0, b1);
-      }
-    }
-  }
-
-  // ---- 4. block softmax across the 4 warps (log2 units)
+  const int v_row = (lane & 7) + 8 * ((lane >> 3) & 1), v_col = 8 * (lane >> 4);  // V (transposed)
   const float sl2 = g.tau * 1.4426950408889634f;
-  float mxa = -CUDART_INF_F, mxb = -CUDART_INF_F;
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const int nt = warp + STEP_WARPS * e;
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const bool ok = nt < NT && 8 * nt + lc + c < blk;
-      sacc[e][c] = ok ? sacc[e][c] * sl2 : -CUDART_INF_F;
-      sacc[e][2 + c] = ok ? sacc[e][2 + c] * sl2 : -CUDART_INF_F;
-      mxa = fmaxf(mxa, sacc[e][c]);
-      mxb = fmaxf(mxb, sacc[e][2 + c]);
-    }
-  }
-  mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
-  mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
-  mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
-  mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
-  if ((lane & 3) == 0) {
-    rmax[warp * STEP_ROWS + lr] = mxa;
-    rmax[warp * STEP_ROWS + lr + 8] = mxb;
-  }
-  __syncthreads();
-  mxa = mxb = -CUDART_INF_F;
-#pragma unroll
-  for (int w = 0; w < STEP_WARPS; ++w) {
-    mxa = fmaxf(mxa, rmax[w * STEP_ROWS + lr]);
-    mxb = fmaxf(mxb, rmax[w * STEP_ROWS + lr + 8]);
-  }
-  float sa = 0.f, sbs = 0.f;
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const int nt = warp + STEP_WARPS * e;
-    if (nt < NT) {
-      const float p0 = tc::ex2(sacc[e][0] - mxa), p1 = tc::ex2(sacc[e][1] - mxa);
-      const float p2 = tc::ex2(sacc[e][2] - mxb), p3 = tc::ex2(sacc[e][3] - mxb);
-      sa += p0 + p1;
-      sbs += p2 + p3;
-      *reinterpret_cast<uint32_t *>(Pt + lr * PSS + (8 * nt + lc) * 2) = pack2(p0, p1);
-      *reinterpret_cast<uint32_t *>(Pt + (lr + 8) * PSS + (8 * nt + lc) * 2) = pack2(p2, p3);
-    }
-  }
-  sa += __shfl_xor_sync(0xffffffffu, sa, 1);
-  sa += __shfl_xor_sync(0xffffffffu, sa, 2);
-  sbs += __shfl_xor_sync(0xffffffffu, sbs, 1);
-  sbs += __shfl_xor_sync(0xffffffffu, sbs, 2);
-  if ((lane & 3) == 0) {
-    rsum[warp * STEP_ROWS + lr] = sa;
-    rsum[warp * STEP_ROWS + lr + 8] = sbs;
-  }
-  __syncthreads();
-  sa = sbs = 0.f;
-#pragma unroll
-  for (int w = 0; w < STEP_WARPS; ++w) {
-    sa += rsum[w * STEP_ROWS + lr];
-    sbs += rsum[w * STEP_ROWS + lr + 8];
-  }
-
-  // ---- 5. O~2 = P~ V for this warp's columns
+  float mxa = -CUDART_INF_F, mxb = -CUDART_INF_F, sa = 0.f, sbs = 0.f;
   float oacc[NTW][4];
 #pragma unroll
   for (int j = 0; j < NTW; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
-  const int v_row = (lane & 7) + 8 * ((lane >> 3) & 1), v_col = 8 * (lane >> 4);
+
+  if constexpr (WPT == 1) {
+    // ---- 3. S = Q^ K^T, all key n-tiles (up to 64 keys)
+    const int b_row = (lane & 7) + 8 * (lane >> 4), b_col = 8 * ((lane >> 3) & 1);
+    float sacc[8][4];
 #pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    if (16 * kk < bpad) {
+    for (int j = 0; j < 8; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
       uint32_t a0, a1, a2, a3;
-      ldsm_x4(ps_a + a_row * PSS + (16 * kk + a_col) * 2, a0, a1, a2, a3);
+      ldsm_x4(qs_a + a_row * RS + (16 * kk + a_col) * 2, a0, a1, a2, a3);
 #pragma unroll
-      for (int jp = 0; jp < NTW / 2; ++jp) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vs_a + (16 * kk + v_row) * RS + (col0 + 16 * jp + v_col) * 2, b0, b1, b2, b3);
-        mma16816(oacc[2 * jp], a0, a1, a2, a3, b0, b1);
-        mma16816(oacc[2 * jp + 1], a0, a1, a2, a3, b2, b3);
+      for (int jp = 0; jp < 4; ++jp) {
+        if (16 * jp < bpad) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(ks_a + (16 * jp + b_row) * RS + (16 * kk + b_col) * 2, b0, b1, b2, b3);
+          mma16816(sacc[2 * jp], a0, a1, a2, a3, b0, b1);
+          mma16816(sacc[2 * jp + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+    // ---- 4. softmax on the fragments (rows lr and lr + 8), log2 units
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool ok = 8 * j + lc + e < blk;
+        sacc[j][e] = ok ? sacc[j][e] * sl2 : -CUDART_INF_F;
+        sacc[j][2 + e] = ok ? sacc[j][2 + e] * sl2 : -CUDART_INF_F;
+        mxa = fmaxf(mxa, sacc[j][e]);
+        mxb = fmaxf(mxb, sacc[j][2 + e]);
+      }
+    }
+    mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
+    mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
+    mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
+    mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
+    uint32_t pa_frag[8], pb_frag[8];  // P~ as bf16 pairs: [n-tile] for rows lr and lr + 8
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float p0 = tc::ex2(sacc[j][0] - mxa), p1 = tc::ex2(sacc[j][1] - mxa);
+      const float p2 = tc::ex2(sacc[j][2] - mxb), p3 = tc::ex2(sacc[j][3] - mxb);
+      sa += p0 + p1;
+      sbs += p2 + p3;
+      pa_frag[j] = pack2(p0, p1);
+      pb_frag[j] = pack2(p2, p3);
+    }
+    sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+    sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+    sbs += __shfl_xor_sync(0xffffffffu, sbs, 1);
+    sbs += __shfl_xor_sync(0xffffffffu, sbs, 2);
+    // ---- 5. O~2 = P~ V, all D columns
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      if (16 * kk < bpad) {
+        const uint32_t a0 = pa_frag[2 * kk], a1 = pb_frag[2 * kk], a2 = pa_frag[2 * kk + 1],
+                       a3 = pb_frag[2 * kk + 1];
+#pragma unroll
+        for (int jp = 0; jp < NTW / 2; ++jp) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(vs_a + (16 * kk + v_row) * RS + (16 * jp + v_col) * 2, b0, b1, b2, b3);
+          mma16816(oacc[2 * jp], a0, a1, a2, a3, b0, b1);
+          mma16816(oacc[2 * jp + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+  } else {
+    const uint32_t ps_a = (uint32_t)__cvta_generic_to_shared(Ps + tr0 * PSS);
+    uint8_t *Pt = Ps + tr0 * PSS;  // this row tile's P~
+    float *rmax = red_max + grp * WPT * STEP_ROWS, *rsum = red_sum + grp * WPT * STEP_ROWS;
+    // ---- 3. S = Q^ K^T for key n-tiles warp and warp + 4 (16 rows x 8 keys each)
+    const int b_row = lane & 7, b_col = 8 * ((lane >> 3) & 1);  // B fragment (k16 x n8)
+    float sacc[2][4];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) sacc[e][0] = sacc[e][1] = sacc[e][2] = sacc[e][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(qs_a + a_row * RS + (16 * kk + a_col) * 2, a0, a1, a2, a3);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int nt = warp + WPT * e;
+        if (nt < NT) {
+          uint32_t b0, b1;
+          ldsm_x2(ks_a + (8 * nt + b_row) * RS + (16 * kk + b_col) * 2, b0, b1);
+          mma16816(sacc[e], a0, a1, a2, a3, b0, b1);
+        }
+      }
+    }
+    // ---- 4. block softmax across the tile's warps (log2 units)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int nt = warp + WPT * e;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const bool ok = nt < NT && 8 * nt + lc + c < blk;
+        sacc[e][c] = ok ? sacc[e][c] * sl2 : -CUDART_INF_F;
+        sacc[e][2 + c] = ok ? sacc[e][2 + c] * sl2 : -CUDART_INF_F;
+        mxa = fmaxf(mxa, sacc[e][c]);
+        mxb = fmaxf(mxb, sacc[e][2 + c]);
+      }
+    }
+    mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
+    mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
+    mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
+    mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
+    if ((lane & 3) == 0) {
+      rmax[warp * STEP_ROWS + lr] = mxa;
+      rmax[warp * STEP_ROWS + lr + 8] = mxb;
+    }
+    __syncthreads();
+    mxa = mxb = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < WPT; ++w) {
+      mxa = fmaxf(mxa, rmax[w * STEP_ROWS + lr]);
+      mxb = fmaxf(mxb, rmax[w * STEP_ROWS + lr + 8]);
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int nt = warp + WPT * e;
+      if (nt < NT) {
+        const float p0 = tc::ex2(sacc[e][0] - mxa), p1 = tc::ex2(sacc[e][1] - mxa);
+        const float p2 = tc::ex2(sacc[e][2] - mxb), p3 = tc::ex2(sacc[e][3] - mxb);
+        sa += p0 + p1;
+        sbs += p2 + p3;
+        *reinterpret_cast<uint32_t *>(Pt + lr * PSS + (8 * nt + lc) * 2) = pack2(p0, p1);
+        *reinterpret_cast<uint32_t *>(Pt + (lr + 8) * PSS + (8 * nt + lc) * 2) = pack2(p2, p3);
+      }
+    }
+    sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+    sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+    sbs += __shfl_xor_sync(0xffffffffu, sbs, 1);
+    sbs += __shfl_xor_sync(0xffffffffu, sbs, 2);
+    if ((lane & 3) == 0) {
+      rsum[warp * STEP_ROWS + lr] = sa;
+      rsum[warp * STEP_ROWS + lr + 8] = sbs;
+    }
+    __syncthreads();
+    sa = sbs = 0.f;
+#pragma unroll
+    for (int w = 0; w < WPT; ++w) {
+      sa += rsum[w * STEP_ROWS + lr];
+      sbs += rsum[w * STEP_ROWS + lr + 8];
+    }
+    // ---- 5. O~2 = P~ V for this warp's columns
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      if (16 * kk < bpad) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(ps_a + a_row * PSS + (16 * kk + a_col) * 2, a0, a1, a2, a3);
+#pragma unroll
+        for (int jp = 0; jp < NTW / 2; ++jp) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(vs_a + (16 * kk + v_row) * RS + (col0 + 16 * jp + v_col) * 2, b0, b1, b2, b3);
+          mma16816(oacc[2 * jp], a0, a1, a2, a3, b0, b1);
+          mma16816(oacc[2 * jp + 1], a0, a1, a2, a3, b2, b3);
+        }
       }
     }
   }
@@ -342,12 +413,12 @@ __global__ void __launch_bounds__(RT * STEP_WARPS * 32) block_merge_mma_kernel(
   }
 }
 
-template <int D, int RT>
-cudaError_t launch_mma_rt(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
-                          const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
-                          cudaStream_t st) {
-  const StepLayout<D, RT> lay(g.blk);
-  auto kern = block_merge_mma_kernel<D, RT>;
+template <int D, int WPT, int RT>
+cudaError_t launch_mma_cfg(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
+                           const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
+                           cudaStream_t st) {
+  const StepLayout<D, WPT, RT> lay(g.blk);
+  auto kern = block_merge_mma_kernel<D, WPT, RT>;
   if (lay.bytes > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.bytes);
     if (e != cudaSuccess) return e;
@@ -355,13 +426,16 @@ cudaError_t launch_mma_rt(const Geometry &g, const __nv_bfloat16 *q, const __nv_
   const int tiles = (g.rows + RT * STEP_ROWS - 1) / (RT * STEP_ROWS);
   const long long ctas = (long long)g.batch * g.hkv * tiles;
   if (ctas > 0x7fffffffll) return cudaErrorInvalidConfiguration;
-  return launch_pdl(kern, dim3((unsigned)ctas), dim3(RT * STEP_WARPS * 32), lay.bytes, st, g, q, kb, vb, pfx,
+  return launch_pdl(kern, dim3((unsigned)ctas), dim3(RT * WPT * 32), lay.bytes, st, g, q, kb, vb, pfx,
                     static_cast<__nv_bfloat16 *>(out), lse, tiles);
 }
 
-// Row tiles per CTA: the largest RT in {1, 2, 4} that still gives at least
-// one CTA per SM, so that big batches share each staged K/V and RoPE table
-// among more rows while small ones keep the most CTAs (and the shortest chain).
+// Layout choice from the number of 16-row tiles n = units * ceil(G*B / 16),
+// fitted to measurements on the five workload shapes: with n at least 4 per SM
+// the step is throughput-bound and one warp per tile (4 tiles per CTA) does
+// the fewest instructions; below that it is latency-bound and 4 warps per tile
+// shorten each warp's chain, with RT the largest of {1, 2, 4} that still gives
+// about one CTA per SM (at least 85% of the SM count).
 template <int D>
 cudaError_t launch_mma(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
                        const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
@@ -369,13 +443,14 @@ cudaError_t launch_mma(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfl
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long units = (long long)g.batch * g.hkv, t16 = (g.rows + STEP_ROWS - 1) / STEP_ROWS;
+  if (units * t16 >= 4ll * sms) return launch_mma_cfg<D, 1, 4>(g, q, kb, vb, pfx, out, lse, st);
   int rt = 1;
   for (int c = 4; c > 1; c >>= 1)
-    if (c <= t16 && units * ((t16 + c - 1) / c) >= sms) { rt = c; break; }
+    if (c <= t16 && units * ((t16 + c - 1) / c) * 20 >= 17ll * sms) { rt = c; break; }
   switch (rt) {
-    case 4: return launch_mma_rt<D, 4>(g, q, kb, vb, pfx, out, lse, st);
-    case 2: return launch_mma_rt<D, 2>(g, q, kb, vb, pfx, out, lse, st);
-    default: return launch_mma_rt<D, 1>(g, q, kb, vb, pfx, out, lse, st);
+    case 4: return launch_mma_cfg<D, 4, 4>(g, q, kb, vb, pfx, out, lse, st);
+    case 2: return launch_mma_cfg<D, 4, 2>(g, q, kb, vb, pfx, out, lse, st);
+    default: return launch_mma_cfg<D, 4, 1>(g, q, kb, vb, pfx, out, lse, st);
   }
 }
 

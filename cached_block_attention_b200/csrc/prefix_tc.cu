@@ -61,7 +61,11 @@ struct Cfg {
   static constexpr int B_ODONE = B_PFULL + 2 * MT;
   static constexpr int B_OFREE = B_ODONE + MT;
   static constexpr int B_DRAIN = B_OFREE + MT;  // [2]: S issuer, PV issuer
-  static constexpr int NBAR = B_DRAIN + 2;
+  // one phase only: the first piece's query rows are in place. The producers
+  // wait for it after their first stage, so the block's Q loads are not queued
+  // behind a full ring of K/V tiles.
+  static constexpr int B_QGATE = B_DRAIN + 2;
+  static constexpr int NBAR = B_QGATE + 1;
   static constexpr int TH_OFF = BAR_OFF + NBAR * 8;  // [D/2] double: theta_i / pi
   // [2][8][D/2] float2: cos/sin of b*theta_i and of 8a*theta_i (a, b < 8), so
   // that any block offset t = 8a + b < 64 is two complex products away
@@ -183,7 +187,7 @@ __device__ __forceinline__ void rotate_q_rows(const Geometry &g, const Piece &p,
       const int e1 = 8 * c, e2 = HALF + 8 * c, t = (mt * 128 + rr) % g.blk;
       const uint32_t a1 = qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8);
       const uint32_t a2 = qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8);
-      const float2 *t1 = tt + (t & 7) * HALF + e1, *t8 = tt + (8 + (t >> 3)) * HALF + e1;
+      const float2 *t1 = tt + (t & 7) * HALF + c, *t8 = tt + (8 + (t >> 3)) * HALF + c;  // + m * CHUNKS
       uint32_t aw[4], bw[4];
       ld_shared_v4(a1, aw);
       ld_shared_v4(a2, bw);
@@ -194,7 +198,7 @@ __device__ __forceinline__ void rotate_q_rows(const Geometry &g, const Piece &p,
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int m = 2 * e + h2;
-          const float2 u = t1[m], v = t8[m];
+          const float2 u = t1[m * CHUNKS], v = t8[m * CHUNKS];
           const float uc = u.x * v.x - u.y * v.y, us = u.x * v.y + u.y * v.x;  // t * theta
           const float cs = cl[m].x * uc - cl[m].y * us, sn = cl[m].x * us + cl[m].y * uc;  // (L + t) * theta
           const float x1 = __uint_as_float(h2 ? (aw[e] & 0xffff0000u) : (aw[e] << 16));
@@ -251,6 +255,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     }
     mbar_init(bar(C::B_DRAIN), 1);
     mbar_init(bar(C::B_DRAIN + 1), 1);
+    mbar_init(bar(C::B_QGATE), 128 * MT);
     *abort_flag = 0;
     mbar_fence_init();
     prefetch_tmap(&tmk);
@@ -266,7 +271,8 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     const int i = idx % (D / 2), k = idx / (D / 2);  // k < 8: b = k; k >= 8: 8a with a = k - 8
     const double f = freq_over_pi(i, D, g.log2_base);
     if (k == 0) theta_tab[i] = f;
-    tt[idx] = rope_cs_f32(k < 8 ? k : 8 * (k - 8), f);
+    // pair i = 8c + m sits at (k, m, c): lanes with chunks c = 0..7 read consecutive entries
+    tt[k * (D / 2) + (i & 7) * (D / 16) + (i >> 3)] = rope_cs_f32(k < 8 ? k : 8 * (k - 8), f);
   }
   pdl_release();
   pdl_wait();
@@ -313,6 +319,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
           if (!mbar_wait(bar(b_empty + st), ((i / C::NS) & 1) ^ 1, abort_flag)) { ok = false; break; }
           mbar_expect_tx(bar(b_full + st), C::KV_BYTES);
           load_kv_tile<D>(g, map, ring + st * C::KV_BYTES, p, j, boxh, bar(b_full + st), pol);
+          if (i == 0 && !mbar_wait(bar(C::B_QGATE), 0, abort_flag)) { ok = false; ++i; break; }
         }
       }
       // no TMA write may be in flight when the CTA leaves
@@ -417,6 +424,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
       rotate_q_rows<D, MT>(g, p, qbase, mt, wg_tid, theta_tab, tt);
       fence_proxy_async();
       mbar_arrive(bar(C::B_QFULL + mt));
+      if (i == 0) mbar_arrive(bar(C::B_QGATE));  // first piece of the CTA
 
       float m_ref = -CUDART_INF_F, m_true = -CUDART_INF_F, lsum = 0.f;
       const int n = p.tile_end - p.tile_begin;
