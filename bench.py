@@ -459,7 +459,7 @@ def run_ours(args, wl, rank, world, local):
                 "algorithmic_bytes_per_launch": dom_bytes, "launch_us": dom_launch_ms * 1e3}
     pfx_gbs = kv_bytes / (pfx_ms * 1e-3) / 1e9
     pfx_tfs = pfx_flops / (pfx_ms * 1e-3) / 1e12
-    n_per_block = 2 + S + 1
+    n_per_block = 2 + S + 2  # prefix (share kernel + reduce), S steps, commit (rows + lengths)
 
     value = world * args.steps * S / (total_ms * 1e-3)
     line = {

@@ -147,8 +147,8 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
     // chunks c = 0..7 of one row read 8 consecutive float4 (no bank conflict)
     cs[t * HALF + ((i >> 1) & 3) * (D / 8) + (i >> 3) * 2 + (i & 1)] = make_float2(c, sn);
   }
-  pdl_release();
   pdl_wait();
+  pdl_release();
 
   // ---- 1. every global read of the CTA, issued at once
   const long long kv_row0 = (long long)b * blk * g.hkv + kvh;  // token t: row kv_row0 + t*hkv
@@ -501,8 +501,8 @@ __global__ void __launch_bounds__(THREADS) block_merge_f32_kernel(
   const int r0 = blockIdx.x * RC;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const double rope_f = freq_over_pi(tid % HALF, D, g.log2_base);
-  pdl_release();
   pdl_wait();
+  pdl_release();
   int L = g.lens[b];
   if (L < 0) {
     raise_flag(g, FBK_DEVERR_PREFIX_LEN);

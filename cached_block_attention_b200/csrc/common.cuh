@@ -264,8 +264,10 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // (inputs, prefix lengths, states), and before its first global write. Only
 // work on kernel parameters and shared memory comes before it. pdl_release()
 // lets the next kernel in the stream start launching; each kernel calls it
-// once all of its CTAs are running, i.e. at its top. Both are no-ops for a
-// kernel launched without the attribute.
+// right after its wait, so that only the next kernel runs ahead (its CTAs do
+// their parameter-only set-up while this one works) instead of the whole
+// chain piling up on the SMs. Both are no-ops for a kernel launched without
+// the attribute.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_release() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

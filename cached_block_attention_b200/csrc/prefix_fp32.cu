@@ -43,8 +43,8 @@ __global__ void __launch_bounds__(THREADS) prefix_fp32_kernel(Geometry g,
 
   int *s_len = reinterpret_cast<int *>(sm + S::LEN_OFF);
   int *s_scan = reinterpret_cast<int *>(sm + S::SCAN_OFF);
-  pdl_release();
   pdl_wait();
+  pdl_release();
   const long long T = load_tile_scan(g, s_len, s_scan);
   if (T == 0) return;
   PieceWalker walk;

@@ -274,8 +274,8 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     // pair i = 8c + m sits at (k, m, c): lanes with chunks c = 0..7 read consecutive entries
     tt[k * (D / 2) + (i & 7) * (D / 16) + (i >> 3)] = rope_cs_f32(k < 8 ? k : 8 * (k - 8), f);
   }
-  pdl_release();
   pdl_wait();
+  pdl_release();
   fence_before_sync();
   const long long T = load_tile_scan(g, s_len, s_scan);  // reads prefix_lens; two CTA barriers
   fence_after_sync();

@@ -22,8 +22,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) split_reduce_kernel(Geometry g,
   const int u = blockIdx.x, b = u / g.hkv, kvh = u % g.hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.y * WARPS + warp;
-  pdl_release();
   pdl_wait();
+  pdl_release();
 
   // tiles before sequence b and in total: parallel loads, block reduction
   __shared__ long long red[2][WARPS];
