@@ -445,14 +445,19 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
             for (int c = 0; c < 64; ++c)
               if (c >= nval) sr[c] = __float_as_uint(-CUDART_INF_F);
           }
-          // tile max of the raw scores (tau > 0): 8 independent chains, then a tree
+          // tile max of the raw scores (tau > 0): 8 independent chains of
+          // three-input maxima, then a tree
+          auto sv = [&](int c) { return __uint_as_float(sr[c]); };
           float mx[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
+          for (int k = 0; k < 8; ++k) mx[k] = fmax3(sv(k), sv(k + 8), sv(k + 16));
 #pragma unroll
-          for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
-          const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+          for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv(k + 24), sv(k + 32));
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv(k + 40), sv(k + 48));
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], sv(k + 56));
+          const float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7])) * sl2;
           m_true = fmaxf(m_true, tmax);
           const bool need = jj > 0 && tmax > m_ref + 8.f;
           if (jj == 0) m_ref = tmax;
@@ -485,16 +490,17 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
             // packed to bf16 pairs in place (pair c overwrites sr[c] after sr[2c],
             // sr[2c+1] are read) and stored over the first 32 columns of this
             // S buffer, where the PV issuer reads it as the A operand
-            const float neg = -m_ref;
-            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            // (paired FP32 instructions for the scale-and-shift and the sums)
+            const float2 sc2 = make_float2(sl2, sl2), ng2 = make_float2(-m_ref, -m_ref);
+            float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, neg));
-              const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, neg));
-              sr[c] = pack_bf16(p0, p1);
-              ps[c & 3] += p0 + p1;
+              const float2 x = ffma2(make_float2(sv(2 * c), sv(2 * c + 1)), sc2, ng2);
+              const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+              sr[c] = pack_bf16(pp.x, pp.y);
+              acc[c & 1] = fadd2(acc[c & 1], pp);
             }
-            lsum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+            lsum += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
             tmem_st32(ts, *reinterpret_cast<uint32_t(*)[32]>(sr));
             tmem_wait_st();
           }
