@@ -153,7 +153,8 @@ fbk_status fbk_prefix_partial(const fbk_shape *shape, const void *q_blk, const f
   if (st != FBK_OK) return st;
   if ((st = check_cache(shape, cache)) != FBK_OK) return st;
   if (!q_blk || !out || !out->o_unnorm || !out->m || !out->l || num_splits < 0) return FBK_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(q_blk) & 15u) return FBK_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(q_blk) | reinterpret_cast<uintptr_t>(out->o_unnorm)) & 15u)
+    return FBK_ERR_UNSUPPORTED;
   const int shares = num_splits ? num_splits : default_shares();
   if (shares < 1) return FBK_ERR_CUDA;
   size_t ob, mlb;
@@ -234,7 +235,8 @@ fbk_status fbk_prefix_partial_static_scratch(const fbk_shape *shape, const void 
   if (st != FBK_OK) return st;
   if ((st = check_cache(shape, cache)) != FBK_OK) return st;
   if (!q_blk || !out || !out->o_unnorm || !out->m || !out->l || num_splits < 0) return FBK_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(q_blk) & 15u) return FBK_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(q_blk) | reinterpret_cast<uintptr_t>(out->o_unnorm)) & 15u)
+    return FBK_ERR_UNSUPPORTED;
   const int shares = num_splits ? num_splits : default_shares();
   if (shares < 1) return FBK_ERR_CUDA;
   size_t ob, mlb;

@@ -57,13 +57,24 @@ __device__ __forceinline__ int prefix_len(const Geometry &g, int b) {
 __device__ __forceinline__ int tiles_of(int L) { return (L + KV_TILE - 1) / KV_TILE; }
 
 // Share c of P covers list positions [c*T/P, (c+1)*T/P).
+// floor(n / d) for 0 <= n, 1 <= d < 2^31. Below 2^53 the quotient comes from
+// one fp64 division (correctly rounded, so within one of the true quotient)
+// and one integer correction, instead of a 64-bit integer division routine.
+__host__ __device__ __forceinline__ long long floordiv_nonneg(long long n, long long d) {
+  if (n >= (1ll << 53)) return n / d;
+  long long q = (long long)((double)n / (double)d);
+  if (q * d > n) --q;
+  else if ((q + 1) * d <= n) ++q;
+  return q;
+}
+
 __host__ __device__ __forceinline__ long long share_begin(long long c, long long T, long long P) {
-  return (c * T) / P;
+  return floordiv_nonneg(c * T, P);
 }
 
 // The share that holds list position x (largest c with share_begin(c) <= x).
 __device__ __forceinline__ long long share_of(long long x, long long T, long long P) {
-  return ((x + 1) * P - 1) / T;
+  return floordiv_nonneg((x + 1) * P - 1, T);
 }
 
 // Per-sequence tile counts, loaded once per CTA: s_len[b] = validated L_b,
@@ -136,9 +147,9 @@ struct PieceWalker {
     }
     const int L = len[b], tb = tiles_of(L);
     const long long acc = scan[b] - (long long)g.hkv * tb;  // list position where sequence b starts
-    const long long off = pos - acc;
-    const int kvh = (int)(off / tb);
-    const int j0 = (int)(off - (long long)kvh * tb);
+    const int off = (int)(pos - acc);  // < Hkv * tiles of one sequence < 2^31
+    const int kvh = off / tb;
+    const int j0 = off - kvh * tb;
     const long long unit_end = acc + (long long)(kvh + 1) * tb;
     const long long stop = unit_end < end ? unit_end : end;
     p.b = b;

@@ -85,15 +85,31 @@ __global__ void __launch_bounds__(WARPS * 32, 1) split_reduce_kernel(Geometry g,
         const float w = __shfl_sync(0xffffffffu, wc, j);
         const long long rj = __shfl_sync(0xffffffffu, row, j);
         const float *src = ws.o + rj * D + lane * CPL;  // empty shares read share c_lo's row, weight 0
+        if constexpr (CPL == 4) {
+          const float4 v = *reinterpret_cast<const float4 *>(src);  // 16-byte aligned: D*4 and the slot base are
+          acc[0] += w * v.x;
+          acc[1] += w * v.y;
+          acc[2] += w * v.z;
+          acc[3] += w * v.w;
+        } else {
 #pragma unroll
-        for (int cc = 0; cc < CPL; ++cc) acc[cc] += w * src[cc];
+          for (int cc = 0; cc < CPL; cc += 2) {
+            const float2 v = *reinterpret_cast<const float2 *>(src + cc);
+            acc[cc] += w * v.x;
+            acc[cc + 1] += w * v.y;
+          }
+        }
       }
       M = Mn;
     }
   }
   float *dst = out.o_unnorm + orow * D + lane * CPL;
+  if constexpr (CPL == 4) {
+    *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  } else {
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) dst[c] = acc[c];
+    for (int c = 0; c < CPL; c += 2) *reinterpret_cast<float2 *>(dst + c) = make_float2(acc[c], acc[c + 1]);
+  }
   if (lane == 0) {
     out.m[orow] = M;
     out.l[orow] = Lsum;

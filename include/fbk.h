@@ -127,7 +127,8 @@ int32_t fbk_default_num_splits(void);
  * cached block-external attention).
  *  q_blk: bf16 [b, B, Hq, d], PRE-RoPE; row t of sequence b is rotated at
  *         position prefix_lens[b] + t inside the kernel.
- *  out:   the state, written in full (every row of every head).
+ *  out:   the state, written in full (every row of every head); o_unnorm
+ *         16-byte aligned (FBK_ERR_UNSUPPORTED otherwise), like q_blk.
  *  ws:    device scratch of at least fbk_prefix_workspace_bytes(...) bytes,
  *         caller-owned, contents irrelevant on entry.
  *  num_splits: number of equal shares of the flattened (sequence, kv-head,
