@@ -509,7 +509,7 @@ def run_ours(args, wl, rank, world, local):
                      "hbm_frac": dom_bytes / (dom_launch_ms * 1e-3) / 1e9 / hbm_gbs})
     pfx_gbs = kv_bytes / (pfx_ms * 1e-3) / 1e9
     pfx_tfs = pfx_flops / (pfx_ms * 1e-3) / 1e12
-    n_per_block = 2 + S + 2  # prefix (share kernel + reduce), S steps, commit (rows + lengths)
+    n_per_block = 3 + S + 2  # prefix (query rotation, share kernel, reduce), S steps, commit (rows, lengths)
 
     value = aggregate_steps_per_s(world, args.steps, S, total_ms)
     line = {

@@ -92,12 +92,37 @@ int default_shares() {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Workspace: per-share states for P + b*Hkv - 1 slots (share + unit).
-void ws_sizes(const fbk_shape *s, int shares, size_t *o_bytes, size_t *ml_bytes, long long *slots) {
+// Workspace layout: per-share states for P + b*Hkv - 1 slots (share + unit),
+// O~ then m then l, followed by the rotated block queries of every unit in
+// the tensor-core kernel's M-tile order ([b*Hkv][MT*128][d] bf16). Every
+// region starts on a 256-byte boundary.
+struct WsLayout {
+  size_t o, m, l, qrot, total;
+  long long slots;
+};
+
+WsLayout ws_layout(const fbk_shape *s, int shares) {
   const long long rows = (long long)(s->n_q_heads / s->n_kv_heads) * s->block_len;
-  *slots = (long long)shares + (long long)s->batch * s->n_kv_heads;
-  *o_bytes = align256((size_t)(*slots * rows * s->head_dim) * sizeof(float));
-  *ml_bytes = align256((size_t)(*slots * rows) * sizeof(float));
+  const long long units = (long long)s->batch * s->n_kv_heads, mt = rows > 128 ? 2 : 1;
+  WsLayout w;
+  w.slots = (long long)shares + units;
+  w.o = 0;
+  w.m = w.o + align256((size_t)(w.slots * rows * s->head_dim) * sizeof(float));
+  w.l = w.m + align256((size_t)(w.slots * rows) * sizeof(float));
+  w.qrot = w.l + align256((size_t)(w.slots * rows) * sizeof(float));
+  w.total = w.qrot + align256((size_t)(units * mt * 128 * s->head_dim) * 2);
+  return w;
+}
+
+Workspace carve(const WsLayout &l, void *base) {
+  char *p = static_cast<char *>(base);
+  Workspace w;
+  w.o = reinterpret_cast<float *>(p + l.o);
+  w.m = reinterpret_cast<float *>(p + l.m);
+  w.l = reinterpret_cast<float *>(p + l.l);
+  w.qrot = reinterpret_cast<__nv_bfloat16 *>(p + l.qrot);
+  w.slots = l.slots;
+  return w;
 }
 
 fbk_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FBK_OK : FBK_ERR_CUDA; }
@@ -140,10 +165,7 @@ size_t fbk_prefix_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *ca
   if (check_shape(shape) != FBK_OK || num_splits < 0) return 0;
   const int shares = num_splits ? num_splits : default_shares();
   if (shares < 1) return 0;
-  size_t ob, mlb;
-  long long slots;
-  ws_sizes(shape, shares, &ob, &mlb, &slots);
-  return ob + 2 * mlb;
+  return ws_layout(shape, shares).total;
 }
 
 fbk_status fbk_prefix_partial(const fbk_shape *shape, const void *q_blk, const fbk_kv_cache *cache,
@@ -157,15 +179,10 @@ fbk_status fbk_prefix_partial(const fbk_shape *shape, const void *q_blk, const f
     return FBK_ERR_UNSUPPORTED;
   const int shares = num_splits ? num_splits : default_shares();
   if (shares < 1) return FBK_ERR_CUDA;
-  size_t ob, mlb;
-  long long slots;
-  ws_sizes(shape, shares, &ob, &mlb, &slots);
-  if (!ws || ws_bytes < ob + 2 * mlb) return FBK_ERR_WORKSPACE;
-  Workspace w;
-  w.o = static_cast<float *>(ws);
-  w.m = reinterpret_cast<float *>(static_cast<char *>(ws) + ob);
-  w.l = reinterpret_cast<float *>(static_cast<char *>(ws) + ob + mlb);
-  w.slots = slots;
+  const WsLayout lay = ws_layout(shape, shares);
+  if (!ws || ws_bytes < lay.total) return FBK_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return FBK_ERR_UNSUPPORTED;  // TMA reads the query rows
+  const Workspace w = carve(lay, ws);
   const Geometry g = make_geometry(shape, cache);
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_blk);
@@ -239,17 +256,11 @@ fbk_status fbk_prefix_partial_static_scratch(const fbk_shape *shape, const void 
     return FBK_ERR_UNSUPPORTED;
   const int shares = num_splits ? num_splits : default_shares();
   if (shares < 1) return FBK_ERR_CUDA;
-  size_t ob, mlb;
-  long long slots;
-  ws_sizes(shape, shares, &ob, &mlb, &slots);
-  if (ob + 2 * mlb > (size_t)FBK_STATIC_SCRATCH_BYTES) return FBK_ERR_SCRATCH_LIMIT;
+  const WsLayout lay = ws_layout(shape, shares);
+  if (lay.total > (size_t)FBK_STATIC_SCRATCH_BYTES) return FBK_ERR_SCRATCH_LIMIT;
   void *scratch = nullptr;
   if ((st = static_scratch_address(&scratch)) != FBK_OK) return st;
-  Workspace w;
-  w.o = static_cast<float *>(scratch);
-  w.m = reinterpret_cast<float *>(static_cast<char *>(scratch) + ob);
-  w.l = reinterpret_cast<float *>(static_cast<char *>(scratch) + ob + mlb);
-  w.slots = slots;
+  const Workspace w = carve(lay, scratch);
   const Geometry g = make_geometry(shape, cache);
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_blk);

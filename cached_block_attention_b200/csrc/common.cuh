@@ -290,6 +290,7 @@ struct Workspace {
   float *m;  // [slots, rows]
   float *l;  // [slots, rows]
   long long slots;
+  __nv_bfloat16 *qrot;  // [units, MT * 128, d]: rotated block queries (bf16 mode)
 };
 
 }  // namespace fbk

@@ -33,6 +33,8 @@
 // FBK_DEVERR_TIMEOUT and all roles drain and return.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "launch.h"
 #include "tc.cuh"
 
@@ -52,8 +54,8 @@ struct Cfg {
   static constexpr int BAR_OFF = V_OFF + NS * KV_BYTES;
   // barrier indices
   static constexpr int B_KFULL = 0, B_KEMPTY = NS, B_VFULL = 2 * NS, B_VEMPTY = 3 * NS;
-  static constexpr int B_QFULL = 4 * NS;
-  static constexpr int B_SFULL = B_QFULL + MT;        // [MT][2]
+  static constexpr int B_QLOAD = 4 * NS;              // a piece's rotated query rows landed (TMA)
+  static constexpr int B_SFULL = B_QLOAD + 1;         // [MT][2]
   static constexpr int B_SEMPTY = B_SFULL + 2 * MT;   // [MT][2]: S buffer (and the P~ in it) free
   // [MT][2]: P~ of the tile in S buffer `buf` is written. One barrier per S
   // buffer, so an arrival for tile i+1 can never count toward tile i.
@@ -61,16 +63,8 @@ struct Cfg {
   static constexpr int B_ODONE = B_PFULL + 2 * MT;
   static constexpr int B_OFREE = B_ODONE + MT;
   static constexpr int B_DRAIN = B_OFREE + MT;  // [2]: S issuer, PV issuer
-  // one phase only: the first piece's query rows are in place. The producers
-  // wait for it after their first stage, so the block's Q loads are not queued
-  // behind a full ring of K/V tiles.
-  static constexpr int B_QGATE = B_DRAIN + 2;
-  static constexpr int NBAR = B_QGATE + 1;
-  static constexpr int TH_OFF = BAR_OFF + NBAR * 8;  // [D/2] double: theta_i / pi
-  // [2][8][D/2] float2: cos/sin of b*theta_i and of 8a*theta_i (a, b < 8), so
-  // that any block offset t = 8a + b < 64 is two complex products away
-  static constexpr int TT_OFF = TH_OFF + (D / 2) * 8;
-  static constexpr int LEN_OFF = TT_OFF + 2 * 8 * (D / 2) * 8;  // [MAX_BATCH] int: validated L_b
+  static constexpr int NBAR = B_DRAIN + 2;
+  static constexpr int LEN_OFF = BAR_OFF + NBAR * 8;  // [MAX_BATCH] int: validated L_b
   static constexpr int SCAN_OFF = LEN_OFF + MAX_BATCH * 4;  // [MAX_BATCH] int: tile scan
   static constexpr int MISC_OFF = SCAN_OFF + MAX_BATCH * 4;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;   // + slack to align the base to 1024
@@ -90,32 +84,9 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr)
-               : "memory");
-}
-
-__device__ __forceinline__ void cp_async16_s(uint32_t smem_addr, const void *gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr), "l"(gsrc) : "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&v);
-}
-
-// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128-byte
-// swizzled K-major tile (8-row atoms of 1024 bytes).
-__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
-  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
 template <int D>
@@ -135,91 +106,12 @@ __device__ __forceinline__ void load_kv_tile(const Geometry &g, const CUtensorMa
   }
 }
 
-// Query rows of one unit for M-tile mt, in two halves so the copies can be
-// requested early. An item is 8 rotation pairs of one row (chunk c of each
-// half of the row); thread wg_tid of the warpgroup owns items wg_tid + 128k.
-// issue_q_rows copies the raw bf16 chunks straight into their 128B-swizzled
-// slots of the Q tile (padding rows get zeros); rotate_q_rows waits for this
-// thread's own copies and rotates them in place (RoPE at L + t), so no other
-// thread ever touches those bytes.
-template <int D, int MT>
-__device__ __forceinline__ void issue_q_rows(const Geometry &g, const __nv_bfloat16 *__restrict__ q,
-                                             const Piece &p, uint32_t qbase, int mt, int wg_tid) {
-  constexpr int CHUNKS = D / 16;
-  const int real_rows = min(128, g.rows - mt * 128);
-#pragma unroll
-  for (int k = 0; k < CHUNKS; ++k) {
-    const int item = wg_tid + 128 * k, rr = item / CHUNKS, c = item % CHUNKS;
-    const int e1 = 8 * c, e2 = D / 2 + 8 * c;
-    const uint32_t a1 = qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8);
-    const uint32_t a2 = qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8);
-    if (rr < real_rows) {
-      const int r2 = mt * 128 + rr, t = r2 % g.blk, hl = r2 / g.blk;
-      const __nv_bfloat16 *src = q + (((long long)p.b * g.blk + t) * g.hq + p.kvh * g.group + hl) * D;
-      cp_async16_s(a1, src + e1);
-      cp_async16_s(a2, src + e2);
-    } else {
-      st_shared_v4(a1, 0, 0, 0, 0);
-      st_shared_v4(a2, 0, 0, 0, 0);
-    }
-  }
-}
-
-// Rotates this thread's own copies in place (RoPE at L + t). Every item of a
-// thread has the same chunk c (8 pairs i = 8c + m), so the thread forms
-// cos/sin(L theta_i) for its 8 pairs once per piece, fp64-reduced, while its
-// copies are in flight; the block offset t = 8a + b then enters through two
-// complex products with the tables of b*theta_i and 8a*theta_i.
-template <int D, int MT>
-__device__ __forceinline__ void rotate_q_rows(const Geometry &g, const Piece &p, uint32_t qbase, int mt,
-                                              int wg_tid, const double *theta_tab, const float2 *tt) {
-  constexpr int CHUNKS = D / 16, HALF = D / 2;
-  const int real_rows = min(128, g.rows - mt * 128);
-  const int c = wg_tid % CHUNKS;
-  float2 cl[8];
-#pragma unroll
-  for (int m = 0; m < 8; ++m) cl[m] = rope_cs_fast(p.L, theta_tab[8 * c + m]);
-  cp_async_wait_all();
-#pragma unroll
-  for (int k = 0; k < CHUNKS; ++k) {
-    const int item = wg_tid + 128 * k, rr = item / CHUNKS;
-    if (rr < real_rows) {
-      const int e1 = 8 * c, e2 = HALF + 8 * c, t = (mt * 128 + rr) % g.blk;
-      const uint32_t a1 = qbase + (e1 / 64) * 16384 + sw128(rr, (e1 % 64) / 8);
-      const uint32_t a2 = qbase + (e2 / 64) * 16384 + sw128(rr, (e2 % 64) / 8);
-      const float2 *t1 = tt + (t & 7) * HALF + c, *t8 = tt + (8 + (t >> 3)) * HALF + c;  // + m * CHUNKS
-      uint32_t aw[4], bw[4];
-      ld_shared_v4(a1, aw);
-      ld_shared_v4(a2, bw);
-      uint32_t y1w[4], y2w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float y1[2], y2[2];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int m = 2 * e + h2;
-          const float2 u = t1[m * CHUNKS], v = t8[m * CHUNKS];
-          const float uc = u.x * v.x - u.y * v.y, us = u.x * v.y + u.y * v.x;  // t * theta
-          const float cs = cl[m].x * uc - cl[m].y * us, sn = cl[m].x * us + cl[m].y * uc;  // (L + t) * theta
-          const float x1 = __uint_as_float(h2 ? (aw[e] & 0xffff0000u) : (aw[e] << 16));
-          const float x2 = __uint_as_float(h2 ? (bw[e] & 0xffff0000u) : (bw[e] << 16));
-          y1[h2] = x1 * cs - x2 * sn;
-          y2[h2] = x2 * cs + x1 * sn;
-        }
-        y1w[e] = pack_bf16(y1[0], y1[1]);
-        y2w[e] = pack_bf16(y2[0], y2[1]);
-      }
-      st_shared_v4(a1, y1w[0], y1w[1], y1w[2], y1w[3]);
-      st_shared_v4(a2, y2w[0], y2w[1], y2w[2], y2w[3]);
-    }
-  }
-}
-
 template <int D, int MT>
 __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     prefix_tc_kernel(const __grid_constant__ Geometry g, const __nv_bfloat16 *__restrict__ q,
                      const Workspace ws, const int shares, const __grid_constant__ CUtensorMap tmk,
-                     const __grid_constant__ CUtensorMap tmv, const int boxh) {
+                     const __grid_constant__ CUtensorMap tmv, const int boxh,
+                     const __grid_constant__ CUtensorMap tmq) {
   using C = Cfg<D, MT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -242,8 +134,8 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
       mbar_init(bar(C::B_VFULL + s), 1);
       mbar_init(bar(C::B_VEMPTY + s), 1);
     }
+    mbar_init(bar(C::B_QLOAD), 1);
     for (int mt = 0; mt < MT; ++mt) {
-      mbar_init(bar(C::B_QFULL + mt), 128);
       mbar_init(bar(C::B_SFULL + 2 * mt), 1);
       mbar_init(bar(C::B_SFULL + 2 * mt + 1), 1);
       mbar_init(bar(C::B_SEMPTY + 2 * mt), 1);
@@ -255,24 +147,15 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     }
     mbar_init(bar(C::B_DRAIN), 1);
     mbar_init(bar(C::B_DRAIN + 1), 1);
-    mbar_init(bar(C::B_QGATE), 128 * MT);
     *abort_flag = 0;
     mbar_fence_init();
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
+    prefetch_tmap(&tmq);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
-  }
-  double *theta_tab = reinterpret_cast<double *>(smem + C::TH_OFF);
-  float2 *tt = reinterpret_cast<float2 *>(smem + C::TT_OFF);
-  for (int idx = threadIdx.x; idx < 2 * 8 * (D / 2); idx += C::THREADS) {
-    const int i = idx % (D / 2), k = idx / (D / 2);  // k < 8: b = k; k >= 8: 8a with a = k - 8
-    const double f = freq_over_pi(i, D, g.log2_base);
-    if (k == 0) theta_tab[i] = f;
-    // pair i = 8c + m sits at (k, m, c): lanes with chunks c = 0..7 read consecutive entries
-    tt[k * (D / 2) + (i & 7) * (D / 16) + (i >> 3)] = rope_cs_f32(k < 8 ? k : 8 * (k - 8), f);
   }
   pdl_wait();
   pdl_release();
@@ -285,16 +168,12 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     return;
   }
 
-  // The softmax warpgroups request their first unit's query rows right away;
-  // the producers start the K/V stream at the same time.
   PieceWalker sm_walk;
   Piece sm_piece;
   bool sm_more = false;
   if (warp >= 4) {
     sm_walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
     sm_more = sm_walk.next(g, sm_piece);
-    if (sm_more) issue_q_rows<D, MT>(g, q, sm_piece, sb + C::Q_OFF + ((warp - 4) >> 2) * C::Q_BYTES,
-                                     (warp - 4) >> 2, threadIdx.x & 127);
   }
 
   if (warp == 0 || warp == 3) {
@@ -319,7 +198,6 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
           if (!mbar_wait(bar(b_empty + st), ((i / C::NS) & 1) ^ 1, abort_flag)) { ok = false; break; }
           mbar_expect_tx(bar(b_full + st), C::KV_BYTES);
           load_kv_tile<D>(g, map, ring + st * C::KV_BYTES, p, j, boxh, bar(b_full + st), pol);
-          if (i == 0 && !mbar_wait(bar(C::B_QGATE), 0, abort_flag)) { ok = false; ++i; break; }
         }
       }
       // no TMA write may be in flight when the CTA leaves
@@ -330,14 +208,31 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     // ---------------------------------------------------------------- S = Q K^T issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, KV_TILE, false);
+      const uint64_t qpol = policy_evict_last();
       PieceWalker walk;
       walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
       Piece p;
       int i = 0, pi = 0;
       bool ok = true;
       while (ok && walk.next(g, p)) {
-        for (int mt = 0; mt < MT && ok; ++mt) ok = mbar_wait(bar(C::B_QFULL + mt), pi & 1, abort_flag);
+        // the piece's rotated query rows, M-tile order, by TMA into the Q tiles;
+        // from the second piece on, once the previous piece's last S products
+        // (the only readers of the Q tiles) have completed
+        if (pi > 0)
+          for (int mt = 0; mt < MT && ok; ++mt)
+            ok = mbar_wait(bar(C::B_SFULL + 2 * mt + ((i - 1) & 1)), ((i - 1) >> 1) & 1, abort_flag);
         if (!ok) break;
+        mbar_expect_tx(bar(C::B_QLOAD), MT * C::Q_BYTES);
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int cb = 0; cb < D / 64; ++cb)
+            tma_load_2d(sb + C::Q_OFF + mt * C::Q_BYTES + cb * 16384, &tmq, cb * 64, (p.u * MT + mt) * 128,
+                        bar(C::B_QLOAD), qpol);
+        if (!mbar_wait(bar(C::B_QLOAD), pi & 1, abort_flag)) {
+          mbar_wait_drain(bar(C::B_QLOAD), pi & 1);  // no TMA write may be in flight when the CTA leaves
+          ok = false;
+          break;
+        }
         fence_after_sync();
         for (int j = p.tile_begin; j < p.tile_end && ok; ++j, ++i) {
           const int st = i % C::NS, buf = i & 1;
@@ -409,22 +304,14 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     const bool wact = mt * 128 + wq * 32 < g.rows;  // warp holds at least one real row
     const uint32_t tl = (uint32_t)(wq * 32) << 16;
     const float sl2 = g.tau * 1.4426950408889634f;  // scores in log2 units
-    const int wg_tid = threadIdx.x & 127;           // 0..127 inside the warpgroup
-    const uint32_t qbase = sb + C::Q_OFF + mt * C::Q_BYTES;
     // waits are made warp-uniform so that warp-collective TMEM accesses never diverge
     auto wwait = [&](uint32_t b, uint32_t ph) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(b, ph, abort_flag));
     };
     Piece& p = sm_piece;
     int i = 0;
-    bool ok = true, first_piece = true;
+    bool ok = true;
     while (ok && sm_more) {
-      if (!first_piece) issue_q_rows<D, MT>(g, q, p, qbase, mt, wg_tid);
-      first_piece = false;
-      rotate_q_rows<D, MT>(g, p, qbase, mt, wg_tid, theta_tab, tt);
-      fence_proxy_async();
-      mbar_arrive(bar(C::B_QFULL + mt));
-      if (i == 0) mbar_arrive(bar(C::B_QGATE));  // first piece of the CTA
 
       float m_ref = -CUDART_INF_F, m_true = -CUDART_INF_F, lsum = 0.f;
       const int n = p.tile_end - p.tile_begin;
@@ -556,6 +443,53 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
   if (threadIdx.x == 0 && *abort_flag) raise_flag(g, FBK_DEVERR_TIMEOUT);
 }
 
+// Rotated block queries for the prefix kernel, in its M-tile order: row
+// (u * MT * 128 + r) of qrot holds query row r = hl * B + t of unit u =
+// (b, kvh), i.e. head kvh * G + hl at position L_b + t, RoPE-rotated (rotate
+// half, fp64-reduced angle, fast sine/cosine) and rounded to bf16; rows r >=
+// G*B are zero. One thread per 8 rotation pairs (chunk c of each half of a row).
+template <int D, int MT>
+__global__ void __launch_bounds__(256) rope_q_kernel(Geometry g, const __nv_bfloat16 *__restrict__ q,
+                                                    __nv_bfloat16 *__restrict__ qrot) {
+  constexpr int HALF = D / 2, KI = D / 16, ROWS = MT * 128;
+  __shared__ double theta[HALF];
+  for (int i = threadIdx.x; i < HALF; i += blockDim.x) theta[i] = freq_over_pi(i, D, g.log2_base);
+  __syncthreads();
+  pdl_wait();
+  pdl_release();
+  const long long n_items = (long long)g.batch * g.hkv * ROWS * KI;
+  for (long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x; item < n_items;
+       item += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(item % KI);
+    const long long rowi = item / KI;
+    const int r = (int)(rowi % ROWS);
+    const int u = (int)(rowi / ROWS), b = u / g.hkv, kvh = u % g.hkv;
+    uint4 y1 = make_uint4(0, 0, 0, 0), y2 = make_uint4(0, 0, 0, 0);
+    if (r < g.rows) {
+      const int t = r % g.blk, h = kvh * g.group + r / g.blk;
+      const int L = prefix_len(g, b);
+      const uint4 *src = reinterpret_cast<const uint4 *>(q + (((long long)b * g.blk + t) * g.hq + h) * D);
+      const uint4 a = src[c], bq = src[c + KI];
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {bq.x, bq.y, bq.z, bq.w};
+      uint32_t o1[4], o2[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 c0 = rope_cs_fast(L + t, theta[8 * c + 2 * e]);
+        const float2 c1 = rope_cs_fast(L + t, theta[8 * c + 2 * e + 1]);
+        const float x1l = __uint_as_float(aw[e] << 16), x1h = __uint_as_float(aw[e] & 0xffff0000u);
+        const float x2l = __uint_as_float(bw[e] << 16), x2h = __uint_as_float(bw[e] & 0xffff0000u);
+        o1[e] = pack_bf16(x1l * c0.x - x2l * c0.y, x1h * c1.x - x2h * c1.y);
+        o2[e] = pack_bf16(x2l * c0.x + x1l * c0.y, x2h * c1.x + x1h * c1.y);
+      }
+      y1 = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+      y2 = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(qrot + rowi * D);
+    dst[c] = y1;
+    dst[c + KI] = y2;
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;  // driver entry point, looked up once
   if (!fn) {
@@ -590,10 +524,20 @@ cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const Workspac
   CUtensorMap mk, mv;
   if (!make_map(&mk, g.kc, rows, D, boxh) || !make_map(&mv, g.vc, rows, D, boxh))
     return cudaErrorInvalidValue;
-  auto kern = prefix_tc_kernel<D, MT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  // the rotated query rows: [units * MT * 128, D], boxes of 64 columns x 128 rows
+  CUtensorMap mq;
+  const long long qrows = (long long)g.batch * g.hkv * MT * 128;
+  if (qrows > 0x7fffffffll || !make_map(&mq, ws.qrot, qrows, D, 128)) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long items = qrows * (D / 16);
+  const int rq_ctas = (int)std::min<long long>((items + 255) / 256, 8ll * sms);
+  cudaError_t e = launch_pdl(rope_q_kernel<D, MT>, dim3(rq_ctas), dim3(256), 0, st, g, q, ws.qrot);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(shares), dim3(C::THREADS), C::SMEM, st, g, q, ws, shares, mk, mv, boxh);
+  auto kern = prefix_tc_kernel<D, MT>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(shares), dim3(C::THREADS), C::SMEM, st, g, q, ws, shares, mk, mv, boxh, mq);
 }
 
 }  // namespace

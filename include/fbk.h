@@ -113,9 +113,11 @@ typedef struct fbk_partial {
 } fbk_partial;
 
 /* Bytes of scratch fbk_prefix_partial needs for `num_splits` work shares
- * (0 = one share per SM of the current device). Depends only on b, Hkv, G*B,
- * d and the share count, not on the prefix lengths. Returns 0 for an invalid
- * shape. */
+ * (0 = one share per SM of the current device): (shares + b*Hkv) * G*B * (d+2)
+ * fp32 for the per-share states plus b*Hkv * 128*ceil(G*B/128) * d bf16 for the
+ * rotated query rows, each region rounded up to 256 bytes. Depends only on b,
+ * Hkv, G*B, d and the share count, not on the prefix lengths. Returns 0 for an
+ * invalid shape. */
 size_t fbk_prefix_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache,
                                   int32_t num_splits);
 
@@ -130,11 +132,15 @@ int32_t fbk_default_num_splits(void);
  *  out:   the state, written in full (every row of every head); o_unnorm
  *         16-byte aligned (FBK_ERR_UNSUPPORTED otherwise), like q_blk.
  *  ws:    device scratch of at least fbk_prefix_workspace_bytes(...) bytes,
- *         caller-owned, contents irrelevant on entry.
+ *         256-byte aligned (FBK_ERR_UNSUPPORTED otherwise), caller-owned,
+ *         contents irrelevant on entry. It holds the per-share states and the
+ *         RoPE-rotated block queries that the tensor-core kernel reads by TMA.
  *  num_splits: number of equal shares of the flattened (sequence, kv-head,
  *         64-key tile) work list, one CTA each (0 = one per SM).
- * Two launches: the share kernel, then a fixed-order LSE reduction of the
- * per-share states (deterministic run to run). */
+ * Launches (FBK_BF16): the query rotation into ws, the tensor-core share
+ * kernel, then a fixed-order LSE reduction of the per-share states
+ * (deterministic run to run). FBK_FP32_CHECK: the fp32 share kernel (which
+ * rotates the queries itself) and the same reduction. */
 fbk_status fbk_prefix_partial(const fbk_shape *shape, const void *q_blk, const fbk_kv_cache *cache,
                               const fbk_partial *out, void *ws, size_t ws_bytes,
                               int32_t num_splits, void *cuda_stream);

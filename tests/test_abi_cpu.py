@@ -116,8 +116,10 @@ def test_workspace_size_and_check(fbk):
     c = _cache(fbk)
     n = fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), ctypes.byref(c), 10)
     slots = 10 + 2
-    assert n >= slots * 64 * 130 * 4
-    assert n < slots * 64 * 130 * 4 + 3 * 256
+    states = slots * 64 * 130 * 4            # O~, m, l per slot and row (fp32)
+    qrot = 2 * 128 * 128 * 2                 # rotated queries: units x one 128-row M-tile x d (bf16)
+    assert n >= states + qrot
+    assert n < states + qrot + 4 * 256
     p = fbk.CPartial(0x40000, 0x50000, 0x60000)
     st = fbk.lib.fbk_prefix_partial(ctypes.byref(s), ctypes.c_void_p(0x70000), ctypes.byref(c),
                                     ctypes.byref(p), ctypes.c_void_p(0x80000), n - 1, 10, None)
