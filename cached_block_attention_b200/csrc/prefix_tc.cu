@@ -45,17 +45,20 @@ using namespace tc;
 
 template <int D, int MT>
 struct Cfg {
-  static constexpr int NS = (D == 128) ? (MT == 2 ? 4 : 5) : 8;  // K and V ring depth
+  static constexpr int NS = (D == 128) ? 4 : 8;        // K and V ring depth
+  // Q buffers: two where shared memory allows (all but d = 128 with two
+  // M-tiles), so the next piece's query rows load while this piece streams
+  static constexpr int QB = (D == 128 && MT == 2) ? 1 : 2;
   static constexpr int Q_BYTES = 128 * D * 2;          // one M-tile of Q
   static constexpr int KV_BYTES = KV_TILE * D * 2;     // one K (or V) stage
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + MT * Q_BYTES;
+  static constexpr int K_OFF = Q_OFF + QB * MT * Q_BYTES;
   static constexpr int V_OFF = K_OFF + NS * KV_BYTES;
   static constexpr int BAR_OFF = V_OFF + NS * KV_BYTES;
   // barrier indices
   static constexpr int B_KFULL = 0, B_KEMPTY = NS, B_VFULL = 2 * NS, B_VEMPTY = 3 * NS;
-  static constexpr int B_QLOAD = 4 * NS;              // a piece's rotated query rows landed (TMA)
-  static constexpr int B_SFULL = B_QLOAD + 1;         // [MT][2]
+  static constexpr int B_QLOAD = 4 * NS;              // [QB]: a piece's rotated query rows landed (TMA)
+  static constexpr int B_SFULL = B_QLOAD + QB;        // [MT][2]
   static constexpr int B_SEMPTY = B_SFULL + 2 * MT;   // [MT][2]: S buffer (and the P~ in it) free
   // [MT][2]: P~ of the tile in S buffer `buf` is written. One barrier per S
   // buffer, so an arrival for tile i+1 can never count toward tile i.
@@ -134,7 +137,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
       mbar_init(bar(C::B_VFULL + s), 1);
       mbar_init(bar(C::B_VEMPTY + s), 1);
     }
-    mbar_init(bar(C::B_QLOAD), 1);
+    for (int qb = 0; qb < C::QB; ++qb) mbar_init(bar(C::B_QLOAD + qb), 1);
     for (int mt = 0; mt < MT; ++mt) {
       mbar_init(bar(C::B_SFULL + 2 * mt), 1);
       mbar_init(bar(C::B_SFULL + 2 * mt + 1), 1);
@@ -211,29 +214,42 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
       const uint64_t qpol = policy_evict_last();
       PieceWalker walk;
       walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
-      Piece p;
+      Piece p, pn;
+      bool have = walk.next(g, p);
+      bool have_next = have && walk.next(g, pn);
       int i = 0, pi = 0;
       bool ok = true;
-      while (ok && walk.next(g, p)) {
-        // the piece's rotated query rows, M-tile order, by TMA into the Q tiles;
-        // from the second piece on, once the previous piece's last S products
-        // (the only readers of the Q tiles) have completed
-        if (pi > 0)
-          for (int mt = 0; mt < MT && ok; ++mt)
-            ok = mbar_wait(bar(C::B_SFULL + 2 * mt + ((i - 1) & 1)), ((i - 1) >> 1) & 1, abort_flag);
-        if (!ok) break;
-        mbar_expect_tx(bar(C::B_QLOAD), MT * C::Q_BYTES);
+      // rotated query rows of piece `pc` (M-tile order) by TMA into Q buffer qb
+      auto load_q = [&](const Piece &pc, int qb) {
+        mbar_expect_tx(bar(C::B_QLOAD + qb), MT * C::Q_BYTES);
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
           for (int cb = 0; cb < D / 64; ++cb)
-            tma_load_2d(sb + C::Q_OFF + mt * C::Q_BYTES + cb * 16384, &tmq, cb * 64, (p.u * MT + mt) * 128,
-                        bar(C::B_QLOAD), qpol);
-        if (!mbar_wait(bar(C::B_QLOAD), pi & 1, abort_flag)) {
-          mbar_wait_drain(bar(C::B_QLOAD), pi & 1);  // no TMA write may be in flight when the CTA leaves
+            tma_load_2d(sb + C::Q_OFF + (qb * MT + mt) * C::Q_BYTES + cb * 16384, &tmq, cb * 64,
+                        (pc.u * MT + mt) * 128, bar(C::B_QLOAD + qb), qpol);
+      };
+      // the previous piece's last S products (the last readers of its Q buffer) have completed
+      auto prev_s_done = [&]() {
+        bool good = true;
+        for (int mt = 0; mt < MT && good; ++mt)
+          good = mbar_wait(bar(C::B_SFULL + 2 * mt + ((i - 1) & 1)), ((i - 1) >> 1) & 1, abort_flag);
+        return good;
+      };
+      if (have) load_q(p, 0);
+      while (ok && have) {
+        const int qb = C::QB == 2 ? (pi & 1) : 0;
+        const uint32_t qpar = C::QB == 2 ? ((pi >> 1) & 1) : (pi & 1);
+        if (!mbar_wait(bar(C::B_QLOAD + qb), qpar, abort_flag)) {
+          mbar_wait_drain(bar(C::B_QLOAD + qb), qpar);  // no TMA write may be in flight when the CTA leaves
           ok = false;
           break;
         }
         fence_after_sync();
+        if (C::QB == 2 && have_next) {  // prefetch the next piece's rows into the other buffer
+          if (pi > 0 && !prev_s_done()) { ok = false; break; }
+          load_q(pn, qb ^ 1);
+        }
+        const uint32_t q_base = sb + C::Q_OFF + qb * MT * C::Q_BYTES;
         for (int j = p.tile_begin; j < p.tile_end && ok; ++j, ++i) {
           const int st = i % C::NS, buf = i & 1;
           if (!mbar_wait(bar(C::B_KFULL + st), (i / C::NS) & 1, abort_flag)) { ok = false; break; }
@@ -245,7 +261,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const int cb = kk >> 2, ko = (kk & 3) * 32;
-              const uint64_t a = sdesc_sw128(sb + C::Q_OFF + mt * C::Q_BYTES + cb * 128 * 128 + ko, 16, 1024);
+              const uint64_t a = sdesc_sw128(q_base + mt * C::Q_BYTES + cb * 128 * 128 + ko, 16, 1024);
               const uint64_t b = sdesc_sw128(sb + C::K_OFF + st * C::KV_BYTES + cb * KV_TILE * 128 + ko, 16, 1024);
               mma_bf16(d_tmem, a, b, IDESC_S, kk > 0 ? 1u : 0u);
             }
@@ -253,8 +269,18 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
           }
           if (ok) mma_commit(bar(C::B_KEMPTY + st));
         }
+        if (ok && C::QB == 1 && have_next) {  // one Q buffer: reload once this piece's S products are done
+          if (!prev_s_done()) { ok = false; break; }
+          load_q(pn, 0);
+        }
         ++pi;
+        p = pn;
+        have = have_next;
+        have_next = have && walk.next(g, pn);
       }
+      // a prefetched load may still be in flight after an early exit
+      if (!ok && C::QB == 2 && have)
+        mbar_wait_drain(bar(C::B_QLOAD + (pi & 1)), (pi >> 1) & 1);
       mma_commit(bar(C::B_DRAIN));
       mbar_wait_drain(bar(C::B_DRAIN), 0);
     }
