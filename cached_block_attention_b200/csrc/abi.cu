@@ -45,9 +45,9 @@ fbk_status check_cache(const fbk_shape *s, const fbk_kv_cache *c) {
     rows = (long long)s->batch * s->n_kv_heads * c->capacity_tokens;
   }
   if (rows > 0x7fffffffll) return FBK_ERR_CAPACITY;  // TMA row coordinates are int32
-  // the prefix kernels' tile list must stay below 2^31 entries
+  // the prefix kernels' work list (tiles plus UNIT_LEAD per unit) must stay below 2^31 entries
   const long long per_seq = c->paged ? (long long)c->max_pages_per_seq * c->page_size : c->capacity_tokens;
-  if ((long long)s->batch * s->n_kv_heads * ((per_seq + KV_TILE - 1) / KV_TILE) > 0x7fffffffll)
+  if ((long long)s->batch * s->n_kv_heads * ((per_seq + KV_TILE - 1) / KV_TILE + UNIT_LEAD) > 0x7fffffffll)
     return FBK_ERR_CAPACITY;
   return FBK_OK;
 }

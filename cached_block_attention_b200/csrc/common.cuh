@@ -54,7 +54,18 @@ __device__ __forceinline__ int prefix_len(const Geometry &g, int b) {
   return L;
 }
 
-__device__ __forceinline__ int tiles_of(int L) { return (L + KV_TILE - 1) / KV_TILE; }
+__host__ __device__ __forceinline__ int tiles_of(int L) { return (L + KV_TILE - 1) / KV_TILE; }
+
+// In the work list every non-empty unit occupies UNIT_LEAD positions before
+// its tiles. They carry no work: a share whose range starts a new unit pays
+// for the switch (a piece epilogue and the next piece's start, a few tiles'
+// time) in list positions, so the shares that hold several pieces get fewer
+// tiles and finish with the others.
+constexpr int UNIT_LEAD = 4;
+__host__ __device__ __forceinline__ int span_of(int L) {
+  const int tb = tiles_of(L);
+  return tb > 0 ? tb + UNIT_LEAD : 0;
+}
 
 // Share c of P covers list positions [c*T/P, (c+1)*T/P).
 // floor(n / d) for 0 <= n, 1 <= d < 2^31. Below 2^53 the quotient comes from
@@ -77,10 +88,10 @@ __device__ __forceinline__ long long share_of(long long x, long long T, long lon
   return floordiv_nonneg((x + 1) * P - 1, T);
 }
 
-// Per-sequence tile counts, loaded once per CTA: s_len[b] = validated L_b,
-// s_scan[b] = Hkv * sum_{b' <= b} ceil(L_b' / KV_TILE) (inclusive scan; the
-// host keeps the total below 2^31). All threads call it; the loads are issued
-// in parallel, one per thread. Returns T, the total tile count.
+// Per-sequence list lengths, loaded once per CTA: s_len[b] = validated L_b,
+// s_scan[b] = Hkv * sum_{b' <= b} span_of(L_b') (inclusive scan; the host
+// keeps the total below 2^31). All threads call it; the loads are issued in
+// parallel, one per thread. Returns T, the total list length.
 constexpr int MAX_BATCH = 1024;  // sequences per call (shared-memory scan)
 
 __device__ __forceinline__ int load_tile_scan(const Geometry &g, int *s_len, int *s_scan) {
@@ -90,7 +101,7 @@ __device__ __forceinline__ int load_tile_scan(const Geometry &g, int *s_len, int
     int carry = 0;
     for (int b0 = 0; b0 < g.batch; b0 += 32) {
       const int b = b0 + (int)threadIdx.x;
-      int v = b < g.batch ? g.hkv * tiles_of(s_len[b]) : 0;
+      int v = b < g.batch ? g.hkv * span_of(s_len[b]) : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int n = __shfl_up_sync(0xffffffffu, v, o);
@@ -138,28 +149,30 @@ struct PieceWalker {
   }
 
   __device__ __forceinline__ bool next(const Geometry &g, Piece &p) {
-    if (pos >= end) return false;
-    while (pos >= scan[b]) {
-      if (++b >= g.batch) {  // unreachable while the scan is consistent
-        pos = end;
-        return false;
+    while (pos < end) {
+      while (pos >= scan[b]) {
+        if (++b >= g.batch) {  // unreachable while the scan is consistent
+          pos = end;
+          return false;
+        }
       }
+      const int L = len[b], tb = tiles_of(L), span = tb + UNIT_LEAD;  // tb > 0: the scan grew at b
+      const long long acc = scan[b] - (long long)g.hkv * span;       // list position where sequence b starts
+      const int kvh = (int)(pos - acc) / span;                       // < Hkv * span < 2^31
+      const long long ustart = acc + (long long)kvh * span, first = ustart + UNIT_LEAD;
+      const long long stop = ustart + span < end ? ustart + span : end;
+      const long long lo = pos > first ? pos : first;
+      pos = stop;
+      if (lo >= stop) continue;  // only lead positions of this unit in the share
+      p.b = b;
+      p.kvh = kvh;
+      p.u = b * g.hkv + kvh;
+      p.L = L;
+      p.tile_begin = (int)(lo - first);
+      p.tile_end = (int)(stop - first);
+      return true;
     }
-    const int L = len[b], tb = tiles_of(L);
-    const long long acc = scan[b] - (long long)g.hkv * tb;  // list position where sequence b starts
-    const int off = (int)(pos - acc);  // < Hkv * tiles of one sequence < 2^31
-    const int kvh = off / tb;
-    const int j0 = off - kvh * tb;
-    const long long unit_end = acc + (long long)(kvh + 1) * tb;
-    const long long stop = unit_end < end ? unit_end : end;
-    p.b = b;
-    p.kvh = kvh;
-    p.u = b * g.hkv + kvh;
-    p.L = L;
-    p.tile_begin = j0;
-    p.tile_end = j0 + (int)(stop - pos);
-    pos = stop;
-    return true;
+    return false;
   }
 };
 

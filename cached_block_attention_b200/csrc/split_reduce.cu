@@ -31,10 +31,10 @@ __global__ void __launch_bounds__(WARPS * 32) split_reduce_kernel(Geometry g, Wo
   pdl_wait();
   pdl_release();
 
-  // tiles before sequence b and in total: parallel loads, block reduction
+  // list positions before sequence b and in total: parallel loads, block reduction
   long long before = 0, T = 0;
   for (int bb = threadIdx.x; bb < g.batch; bb += WARPS * 32) {
-    const long long n = (long long)g.hkv * tiles_of(prefix_len(g, bb));
+    const long long n = (long long)g.hkv * span_of(prefix_len(g, bb));
     if (bb < b) before += n;
     T += n;
   }
@@ -54,8 +54,9 @@ __global__ void __launch_bounds__(WARPS * 32) split_reduce_kernel(Geometry g, Wo
     before += red[0][w];
     T += red[1][w];
   }
+  // the unit's tiles in the work list: after its UNIT_LEAD lead positions
   const int tb = tiles_of(prefix_len(g, b));
-  const long long A = before + (long long)kvh * tb, E = A + tb;
+  const long long A = before + (long long)kvh * span_of(prefix_len(g, b)) + UNIT_LEAD, E = A + tb;
 
   // the unit's pieces: shares c_lo .. c_hi, each non-empty one holding the
   // piece's state in slot c + u (computed once per CTA, in increasing share order)
