@@ -254,6 +254,28 @@ def test_all_prefixes_empty(mode, mname):
     assert int(case.dev["cache"].error_flags.item()) == 0
 
 
+@pytest.mark.parametrize("page_size", [0, 16])
+def test_maximum_batch(page_size):
+    """b = 1024, the largest batch the shared-memory tile scan takes, with
+    ragged short prefixes (a fifth of them empty): every sequence's prefix
+    state, one step against uncached attention, and the commit's lengths."""
+    from cached_block_attention_b200 import fbk
+    rng = np.random.Generator(np.random.PCG64(1024))
+    lens = rng.integers(0, 140, size=1024)
+    lens[rng.random(1024) < 0.2] = 0
+    case = H.make_case(1024, 2, 1, 64, 8, tuple(lens), page_size, 1.0, seed=1024).upload()
+    pfx = H.run_prefix(case, case.dev["steps"][0][0])
+    ref = orc.prefix_partial(case.step_f64(0)[0], case.k_pfx(), case.v_pfx(), case.lens, 1, 1.0, case.base)
+    H.check_partial(H.partial_to_host(pfx), ref, "bf16", "b=1024")
+    out, _ = H.run_step(case, pfx, 0)
+    H.assert_close(H.host_f64(out), oracle_full(case, 0)[0], "bf16", "b=1024 step")
+    q, k, v = case.dev["steps"][0]
+    fbk.commit_block_rope_append(case.shape, k, v, case.dev["cache"])
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(case.dev["cache"].prefix_lens.cpu().numpy(), case.lens + 8)
+    assert int(case.dev["cache"].error_flags.item()) == 0
+
+
 def test_bad_prefix_len_and_page_are_flagged_not_read():
     from cached_block_attention_b200 import fbk
     case = H.make_case(2, 4, 2, 128, 16, (100, 100), 64, 1.0, seed=81).upload()
