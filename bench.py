@@ -57,11 +57,17 @@ API_KERNEL = {"fbk_block_attn_merge": "block_merge_mma_kernel", "fbk_prefix_part
 
 
 def sources_hash(kernel):
+    """Hash of the kernel's source files with comments and blank space removed,
+    so that a comment edit does not orphan a capture of unchanged code."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, "cached_block_attention_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "cached_block_attention_b200", "csrc", f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(re.sub(r"\s+", " ", text).strip().encode())
     return h.hexdigest()[:16]
 
 

@@ -14,15 +14,17 @@
 // The step moves a few MB and is latency-bound, so both variants are built
 // around one DRAM round trip: every input of the CTA is requested up front
 // (cp.async for block K/V and query rows, register loads for the prefix
-// state), the RoPE cos/sin table is computed while those requests fly, and
-// the rest runs from shared memory and registers.
-//  * FBK_BF16: a CTA holds 16 query rows of one (sequence, kv-head) unit and
-//    that unit's block K/V; its 4 warps split the keys of S = Q^ K^T and the
-//    columns of O = P~ V, which are warp-level bf16 tensor-core MMAs
-//    (mma.sync m16n8k16, fp32 accumulation; at 16 x B x d these products are
-//    far too small for the TMEM/tcgen05 machinery to pay off). Many small
-//    CTAs keep the per-warp chain of dependent steps short, which is what a
-//    step's latency is made of.
+// state), and the rest runs from shared memory and registers.
+//  * FBK_BF16: a CTA holds RT tiles of 16 query rows of one (sequence,
+//    kv-head) unit and that unit's block K/V. S = Q^ K^T and O = P~ V are
+//    warp-level bf16 tensor-core MMAs (mma.sync m16n8k16, fp32 accumulation;
+//    at 16 x B x d these products are far too small for the TMEM/tcgen05
+//    machinery to pay off). With few row tiles, 4 warps per tile split the
+//    keys of S and the columns of O, keeping each warp's chain of dependent
+//    steps short (what a step's latency is made of); with many, one warp per
+//    tile does the fewest instructions. The RoPE table depends on kernel
+//    parameters only (rotation at block offsets, see the kernel) and is built
+//    before the kernel waits for its predecessor.
 //  * FBK_FP32_CHECK: the same steps on CUDA cores in fp32 (no bf16 rounding of
 //    Q^, K^ or P~): lane j scores keys j and j + 32, warp-shuffle row max/sum.
 #include "launch.h"

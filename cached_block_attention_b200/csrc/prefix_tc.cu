@@ -6,24 +6,29 @@
 // (Eq. 2-6) whose result FACache keeps in HBM, here for the block's own query
 // rows (FlashBlock, Abstract: cached block-external attention).
 //
-// How (one CTA per SM-sized share of the flattened (unit, 64-key tile) list),
-// warp-specialised, each role one elected lane or one warpgroup:
+// How (one CTA per SM-sized share of the flattened (unit, 64-key tile) list,
+// each unit preceded by a few lead positions that stand for the cost of
+// switching units), warp-specialised, each role one elected lane or one
+// warpgroup. The block queries were rotated beforehand by rope_q_kernel into
+// the workspace, in this kernel's M-tile order:
 //  * warps 0 and 3: TMA producers of 64-key K and V tiles of the bf16 cache
 //    (contiguous rows or pages) into NS-stage rings, 128-byte swizzled, L2
 //    evict-first (each KV byte is read once). K and V have separate rings and
 //    producers: a K stage frees as soon as S = Q K^T is done, a V stage only
 //    after O += P~ V, so K runs ahead of V.
-//  * warp 1: issues S = Q K^T (M = 128 query rows, N = 64 keys, K = d) into
-//    a double-buffered TMEM S; warp 2: issues O += P~ V (M = 128, N = d,
+//  * warp 1: loads each piece's rotated query rows by TMA (into one of two Q
+//    buffers where shared memory allows, so the next piece's rows arrive
+//    while this one streams) and issues S = Q K^T (M = 128 query rows, N = 64
+//    keys, K = d) into a double-buffered TMEM S; warp 2: issues O += P~ V (M = 128, N = d,
 //    K = 64 keys) into a TMEM accumulator. Both are tcgen05.mma kind::f16 with
 //    fp32 accumulation; two issuers keep a late K tile from holding back a
 //    ready PV product.
 //  * warps 4..4+4*MT-1: one warpgroup per 128-row M-tile (MT = ceil(G*B/128)).
 //    GQA packing: all G query heads of a kv-head share each staged K/V tile,
-//    so every KV byte is read from HBM once per unit. The warpgroup rotates
-//    and writes Q (bf16, swizzled) at the start of a piece; then each thread
-//    owns one query row = one TMEM lane: it reads its S row from TMEM, applies
-//    the recurrence in the log2 domain and writes P~ (bf16) for the PV MMA.
+//    so every KV byte is read from HBM once per unit. Each thread owns one
+//    query row = one TMEM lane: it reads its S row from TMEM, applies the
+//    recurrence in the log2 domain (paired fp32 instructions where they
+//    apply: the loop is issue-bound) and writes P~ (bf16) for the PV MMA.
 //    The O accumulator stays in TMEM; it is rescaled only when the running
 //    max grows by more than 2^8 over the reference max, which leaves the
 //    state exact (O~ and l share one reference max) and bounds P~ by 256.
