@@ -128,3 +128,19 @@ def test_workspace_size_and_check(fbk):
                                     ctypes.byref(p), None, n, 10, None)
     assert st == -4
     assert fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), ctypes.byref(c), -1) == 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "llada8b", "dream7b_gqa", "long131k", "ragged_paged"])
+def test_static_scratch_covers_every_workload(fbk, name):
+    """The built-in 32 MiB scratch of fbk_prefix_partial_static_scratch holds the
+    workspace of every workload shape at one share per SM of a B200 (148)."""
+    from cached_block_attention_b200 import synth
+    wl = synth.WORKLOADS[name]
+    s = fbk.CShape(batch=wl.batch, n_q_heads=wl.n_q_heads, n_kv_heads=wl.n_kv_heads,
+                   head_dim=wl.head_dim, block_len=wl.block_len, softmax_scale=1.0,
+                   rope_base=wl.rope_base, mode=0)
+    n = fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), None, 148)
+    rows = wl.n_q_heads // wl.n_kv_heads * wl.block_len
+    units = wl.batch * wl.n_kv_heads
+    assert n >= (148 + units) * rows * (wl.head_dim + 2) * 4 + units * 128 * ((rows + 127) // 128) * wl.head_dim * 2
+    assert n <= fbk.STATIC_SCRATCH_BYTES
