@@ -44,7 +44,7 @@ import numpy as np
 __all__ = [
     "kv_head_of", "rope_freqs", "rope", "softmax_partial", "online_partial",
     "merge", "finalize", "prefix_partial", "block_partial", "full_attention",
-    "step_output", "block_schedule", "bf16_rne_bits", "bits_to_f64",
+    "step_output", "block_schedule", "refresh_schedule", "bf16_rne_bits", "bits_to_f64",
     "commit_contiguous", "commit_paged", "gather_paged",
 ]
 
@@ -283,6 +283,27 @@ def block_schedule(steps, k_pfx, v_pfx, lens, n_kv_heads, tau, base, heads=None,
     pfx = prefix_partial(q0, k_pfx, v_pfx, lens, n_kv_heads, tau, base, heads, batches)
     return [step_output(pfx, q, k, v, lens, n_kv_heads, tau, base, heads, batches)
             for (q, k, v) in steps]
+
+
+def refresh_schedule(steps, k_pfx, v_pfx, lens, n_kv_heads, tau, base, interval,
+                     heads=None, batches=None):
+    """The block schedule with a cache update interval r (LaCache App. C: the
+    interval trades speed for accuracy when the cached state is reused across
+    steps). Steps are numbered from 0 inside the block; at steps 0, r, 2r, ...
+    the prefix state is computed afresh from that step's block queries, and the
+    steps in between reuse the latest one.
+
+    r = 1 recomputes at every step, so every step is exact full attention;
+    r >= len(steps) is block_schedule. Returns a list of (O, lse), one per step.
+    """
+    if interval < 1:
+        raise ValueError("refresh interval must be >= 1")
+    outs, pfx = [], None
+    for s, (q, k, v) in enumerate(steps):
+        if s % interval == 0:
+            pfx = prefix_partial(q, k_pfx, v_pfx, lens, n_kv_heads, tau, base, heads, batches)
+        outs.append(step_output(pfx, q, k, v, lens, n_kv_heads, tau, base, heads, batches))
+    return outs
 
 
 # ------------------------------------------------------------------ commit

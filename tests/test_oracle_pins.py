@@ -378,6 +378,57 @@ def test_block_schedule_first_step_is_exact():
     np.testing.assert_allclose(outs[1][0], want[0], rtol=1e-14)
 
 
+# ------------------------------------------------------------------ refresh interval (LaCache App. C)
+
+def _steps(seed0, n, q_from=None):
+    """n steps of fresh (q, k_blk, v_blk); q_from[s] = s' makes step s reuse step s' queries."""
+    out = []
+    for s in range(n):
+        q, kb, vb, _, _, _ = make_case(seed0 + 10 * s, lens=(6, 3))
+        out.append([q, kb, vb])
+    for s, src in enumerate(q_from or []):
+        out[s][0] = out[src][0]
+    return [tuple(t) for t in out]
+
+
+def check_refresh_schedule(refresh_schedule):
+    _, _, _, kp, vp, L = make_case(160, lens=(6, 3))
+    full = lambda st: orc.full_attention(st[0], st[1], st[2], kp, vp, L, 2, 1.0, 1e4)
+    # r = 1: every step recomputes, so every step is exact full attention
+    steps = _steps(170, 4)
+    for st, (o, lse) in zip(steps, refresh_schedule(steps, kp, vp, L, 2, 1.0, 1e4, 1)):
+        np.testing.assert_allclose(o, full(st)[0], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(lse, full(st)[1], rtol=1e-12, atol=1e-13)
+    # r >= S: the reuse schedule
+    for r in (4, 7):
+        for a, b in zip(refresh_schedule(steps, kp, vp, L, 2, 1.0, 1e4, r),
+                        orc.block_schedule(steps, kp, vp, L, 2, 1.0, 1e4)):
+            np.testing.assert_allclose(a[0], b[0], rtol=1e-14, atol=0)
+    # r = 3 over 7 steps whose queries change only at steps 0, 3 and 6: every
+    # step's prefix state was refreshed with its own queries, so all are exact
+    steps = _steps(200, 7, q_from=[0, 0, 0, 3, 3, 3, 6])
+    for st, (o, _) in zip(steps, refresh_schedule(steps, kp, vp, L, 2, 1.0, 1e4, 3)):
+        np.testing.assert_allclose(o, full(st)[0], rtol=1e-12, atol=1e-13)
+    # queries that change between refreshes (steps 1, 2, 4, 5) are not exact:
+    # there the state of the latest refresh step is reused
+    steps = _steps(300, 6)
+    outs = refresh_schedule(steps, kp, vp, L, 2, 1.0, 1e4, 3)
+    for s in (1, 2, 4, 5):
+        assert np.abs(outs[s][0] - full(steps[s])[0]).max() > 1e-3
+        pfx = orc.prefix_partial(steps[3 * (s // 3)][0], kp, vp, L, 2, 1.0, 1e4)
+        want = orc.step_output(pfx, *steps[s], L, 2, 1.0, 1e4)
+        np.testing.assert_allclose(outs[s][0], want[0], rtol=1e-14, atol=0)
+
+
+def test_refresh_interval_schedule():
+    check_refresh_schedule(orc.refresh_schedule)
+
+
+def test_refresh_interval_rejects_zero():
+    with pytest.raises(ValueError):
+        orc.refresh_schedule(_steps(400, 2), [], [], np.array([0, 0]), 2, 1.0, 1e4, 0)
+
+
 # ------------------------------------------------------------------ negative controls
 
 def _fails(fn, *args, **kw):
@@ -446,3 +497,25 @@ def test_negative_control_online_without_alpha():
             o = o + p @ v[j0:j0 + tile]
         return o, m, l
     _fails(check_online_matches_two_pass, bad_online)
+
+
+def test_negative_control_refresh_off_by_one():
+    def late_refresh(steps, kp, vp, lens, Hkv, tau, base, r, heads=None, batches=None):
+        outs, pfx = [], None
+        for s, (q, k, v) in enumerate(steps):
+            if s % r == min(1, r - 1):
+                pfx = orc.prefix_partial(q, kp, vp, lens, Hkv, tau, base)
+            if pfx is None:
+                pfx = orc.prefix_partial(q, kp, vp, lens, Hkv, tau, base)
+            outs.append(orc.step_output(pfx, q, k, v, lens, Hkv, tau, base))
+        return outs
+
+    def previous_queries(steps, kp, vp, lens, Hkv, tau, base, r, heads=None, batches=None):
+        outs, pfx = [], None
+        for s, (q, k, v) in enumerate(steps):
+            if s % r == 0:
+                pfx = orc.prefix_partial(steps[max(s - 1, 0)][0], kp, vp, lens, Hkv, tau, base)
+            outs.append(orc.step_output(pfx, q, k, v, lens, Hkv, tau, base))
+        return outs
+    _fails(check_refresh_schedule, late_refresh)
+    _fails(check_refresh_schedule, previous_queries)
