@@ -42,6 +42,12 @@ def parse():
     ap.add_argument("--workload", default="llada8b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=1,
+                    help="attention layers per block; > 1 runs the whole block through fbk_decode_block")
+    ap.add_argument("--refresh-interval", default="",
+                    help="cache update interval(s) for --layers, comma-separated; the first is the "
+                         "reported value, every one is timed and its error against interval 1 reported "
+                         "(default: the workload's step count, i.e. the reuse schedule)")
     return ap.parse_args()
 
 
@@ -92,6 +98,57 @@ def load_peaks():
                 float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured")
     except Exception:
         return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ roofline
+
+def algorithmic_units(wl):
+    """Algorithmic bytes / flops of one launch of each kernel on the workload:
+    the prefix kernel reads K and V of every committed token once (and does
+    4 * Hq * B * d flops per token: QK^T and PV); the step kernel reads the
+    block Q/K/V and the prefix state and writes O."""
+    L_sum = int(wl.prefix_lens().sum())
+    rows = wl.batch * wl.n_q_heads * wl.block_len
+    return {
+        "kv_bytes": 4 * wl.n_kv_heads * wl.head_dim * L_sum,
+        "pfx_flops": 4 * wl.n_q_heads * wl.block_len * wl.head_dim * L_sum,
+        "step_bytes": (rows * wl.head_dim * 2                                      # Q
+                       + 2 * wl.batch * wl.block_len * wl.n_kv_heads * wl.head_dim * 2  # K, V
+                       + rows * (wl.head_dim + 2) * 4                              # prefix state read
+                       + rows * wl.head_dim * 2),                                  # O write
+    }
+
+
+def dominant_roofline(wl, pfx_total_ms, pfx_launch_ms, steps_total_ms, step_launch_ms):
+    """Roofline of the kernel with the larger share of the timed region: HBM
+    bytes, or (prefix only) tensor flops when their time at the sustained
+    bf16 peak exceeds the bytes' time at the HBM peak."""
+    hbm_gbs, tflops, tflops_sus, peak_kind = load_peaks()
+    u = algorithmic_units(wl)
+    units = {
+        "fbk_block_attn_merge": (steps_total_ms, u["step_bytes"], step_launch_ms),
+        "fbk_prefix_partial": (pfx_total_ms, u["kv_bytes"], pfx_launch_ms),
+    }
+    dom = max(units, key=lambda k: units[k][0])
+    _, dom_bytes, dom_launch_ms = units[dom]
+    tr = measured_traffic(API_KERNEL[dom], wl.name)
+    t_hbm = dom_bytes / (hbm_gbs * 1e9)
+    t_tensor = u["pfx_flops"] / (tflops_sus * 1e12) if dom == "fbk_prefix_partial" else 0.0
+    if t_tensor > t_hbm:
+        achieved = u["pfx_flops"] / (dom_launch_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": tflops_sus, "unit": "TFLOP/s",
+                    "frac": achieved / tflops_sus, "peak_kind": f"{peak_kind} bf16_tflops_sustained",
+                    "algorithmic_flops_per_launch": u["pfx_flops"]}
+    else:
+        achieved = dom_bytes / (dom_launch_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                    "frac": achieved / hbm_gbs, "peak_kind": f"{peak_kind} hbm_gbs"}
+    roofline.update({"traffic": tr["dram_bytes_per_launch"] if tr else None,
+                     "traffic_source": tr["profile"] if tr else "no ncu capture of the current kernel source",
+                     "kernel": dom, "algorithmic_bytes_per_launch": dom_bytes,
+                     "launch_us": dom_launch_ms * 1e3,
+                     "hbm_frac": dom_bytes / (dom_launch_ms * 1e-3) / 1e9 / hbm_gbs})
+    return roofline, u
 
 
 # ------------------------------------------------------------------ clocks
@@ -475,44 +532,12 @@ def run_ours(args, wl, rank, world, local):
     h2d = (h_q.numel() + h_k.numel() + h_v.numel()) * 2
     d2h = h_out.numel() * 2
 
-    # roofline of the dominant kernel (by time share inside the timed region)
-    hbm_gbs, tflops, tflops_sus, peak_kind = load_peaks()
-    L_sum = int(lens_np.sum())
-    kv_bytes = 4 * wl.n_kv_heads * wl.head_dim * L_sum
-    pfx_flops = 4 * wl.n_q_heads * wl.block_len * wl.head_dim * L_sum
-    rows = wl.batch * wl.n_q_heads * wl.block_len
-    step_bytes = (rows * wl.head_dim * 2                       # Q
-                  + 2 * wl.batch * wl.block_len * wl.n_kv_heads * wl.head_dim * 2  # K, V
-                  + rows * (wl.head_dim + 2) * 4               # prefix state read
-                  + rows * wl.head_dim * 2)                    # O write
+    hbm_gbs, tflops, tflops_sus, _ = load_peaks()
     mean = lambda x: sum(x) / len(x)
     pfx_ms, steps_ms, commit_ms = mean(t_pfx), mean(t_steps), mean(t_commit)
     step_launch_ms = steps_ms / S
-    units = {
-        "fbk_block_attn_merge": (steps_ms, step_bytes, step_launch_ms, S),
-        "fbk_prefix_partial": (pfx_ms, kv_bytes, pfx_ms, 1),
-    }
-    dom = max(units, key=lambda k: units[k][0])
-    _, dom_bytes, dom_launch_ms, _ = units[dom]
-    tr = measured_traffic(API_KERNEL[dom], wl.name)
-    # the binding roofline of the dominant kernel: HBM bytes, or (prefix only)
-    # tensor flops when their time at the sustained bf16 peak is the larger one
-    t_hbm = dom_bytes / (hbm_gbs * 1e9)
-    t_tensor = pfx_flops / (tflops_sus * 1e12) if dom == "fbk_prefix_partial" else 0.0
-    if t_tensor > t_hbm:
-        achieved = pfx_flops / (dom_launch_ms * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": tflops_sus, "unit": "TFLOP/s",
-                    "frac": achieved / tflops_sus, "peak_kind": f"{peak_kind} bf16_tflops_sustained",
-                    "algorithmic_flops_per_launch": pfx_flops}
-    else:
-        achieved = dom_bytes / (dom_launch_ms * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
-                    "frac": achieved / hbm_gbs, "peak_kind": f"{peak_kind} hbm_gbs"}
-    roofline.update({"traffic": tr["dram_bytes_per_launch"] if tr else None,
-                     "traffic_source": tr["profile"] if tr else "no ncu capture of the current kernel source",
-                     "kernel": dom, "algorithmic_bytes_per_launch": dom_bytes,
-                     "launch_us": dom_launch_ms * 1e3,
-                     "hbm_frac": dom_bytes / (dom_launch_ms * 1e-3) / 1e9 / hbm_gbs})
+    roofline, u = dominant_roofline(wl, pfx_ms, pfx_ms, steps_ms, step_launch_ms)
+    kv_bytes, pfx_flops = u["kv_bytes"], u["pfx_flops"]
     pfx_gbs = kv_bytes / (pfx_ms * 1e-3) / 1e9
     pfx_tfs = pfx_flops / (pfx_ms * 1e-3) / 1e12
     n_per_block = 3 + S + 2  # prefix (query rotation, share kernel, reduce), S steps, commit (rows, lengths)
@@ -554,17 +579,293 @@ def run_ours(args, wl, rank, world, local):
     del graphs, g_block, g_pfx, g_steps, g_commit, g_recomp
 
 
+# ------------------------------------------------------------------ many layers per block
+
+def oracle_layer_block(case, steps, interval):
+    """One layer's block under the refresh schedule, fp64 numpy (the oracle)."""
+    from oracle import fbk_oracle as orc
+    st = [case["steps"][s % len(case["steps"])] for s in range(steps)]
+    orc.refresh_schedule(st, case["kp"], case["vp"], case["lens"], case["hkv"], 1.0, case["base"], interval)
+    q, k, v = st[-1]
+    orc.commit_contiguous(case["kc"], case["vc"], k, case["vbits"], case["lens"], case["base"])
+
+
+def run_reference_layers(args, wl, rank):
+    """The oracle on a bounded sample of the many-layer block: one layer's
+    block (at most 8 steps) per bench step; a denoising step of the whole
+    model counts args.layers layer-steps."""
+    if rank != 0:
+        return
+    r = intervals_of(args, wl)[0]
+    case = oracle_case(wl)
+    s = min(wl.steps, 8)
+    for _ in range(args.warmup):
+        oracle_layer_block(case, s, r)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_layer_block(case, s, r)
+    dt = time.perf_counter() - t0
+    v = args.steps * s / dt / args.layers
+    sample = f"one layer's block with {s} of {wl.steps} steps (interval {r}) per bench step; value / {args.layers} layers"
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "denoising steps/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "layers": args.layers, "refresh_interval": r,
+                       "description": wl.description},
+            "cpu_baseline": {"value": v, "unit": "denoising steps/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "denoising steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_layers(args, wl, rank, world, local):
+    """N attention layers x S denoising steps per block through one
+    fbk_decode_block call, replayed as one CUDA graph per block, with a cache
+    update interval r (LaCache App. C): each layer recomputes its prefix state
+    at steps 0, r, 2r, ... Every layer has its own cache, block inputs and
+    outputs (same synthetic content, separate buffers)."""
+    import torch
+    from cached_block_attention_b200 import fbk, synth
+
+    dev = torch.device("cuda", local)
+    S, N = wl.steps, args.layers
+    intervals = intervals_of(args, wl)
+    lens_np = wl.prefix_lens()
+    ks, vs = synth.gen_prefix(wl, lens_np)
+    extra = wl.block_len
+    if wl.page_size:
+        kp, vp, table = synth.paged_cache(ks, vs, wl.n_kv_heads, wl.head_dim, wl.page_size, extra, wl.page_seed)
+        kh, vh, page_table = kp, vp, torch.from_numpy(table).to(dev)
+    else:
+        kh, vh = synth.contiguous_cache(ks, vs, wl.n_kv_heads, wl.head_dim, int(lens_np.max()) + extra)
+        page_table = None
+    del ks, vs
+    k_src = torch.from_numpy(kh.view(np.int16)).view(torch.bfloat16).to(dev)
+    v_src = torch.from_numpy(vh.view(np.int16)).view(torch.bfloat16).to(dev)
+    del kh, vh
+    lens0 = torch.from_numpy(np.tile(lens_np.astype(np.int32), (N, 1))).to(dev)  # [N, b]
+    lens = lens0.clone()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    shape = fbk.Shape(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.block_len, 1.0, wl.rope_base,
+                      fbk.BF16)
+    host_steps = [synth.gen_step(wl, s) for s in range(S)]
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    h_q = torch.stack([pin(q) for q, _, _ in host_steps]).pin_memory()
+    h_k = torch.stack([pin(k) for _, k, _ in host_steps]).pin_memory()
+    h_v = torch.stack([pin(v) for _, _, v in host_steps]).pin_memory()
+    caches, ins, pfxs, outs = [], [], [], []
+    for l in range(N):
+        caches.append(fbk.KVCache(k_src.clone(), v_src.clone(), lens[l], page_table, err))
+        ins.append((h_q.to(dev), h_k.to(dev), h_v.to(dev)))
+        pfxs.append(fbk.Partial.empty(shape, dev))
+        outs.append(torch.empty(S, wl.batch, wl.block_len, wl.n_q_heads, wl.head_dim, dtype=torch.bfloat16,
+                                device=dev))
+    del k_src, v_src
+    ws = torch.empty(fbk.prefix_workspace_bytes(shape, caches[0], 0), dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    def blocks_for(r):
+        return [fbk.LayerBlock(ins[l][0], ins[l][1], ins[l][2], caches[l], pfxs[l], outs[l], r) for l in range(N)]
+
+    def run_block(r):
+        lens.copy_(lens0)  # every bench step decodes the same block position
+        fbk.decode_block(shape, blocks_for(r), ws, commit=True)
+
+    def seg_prefix():  # one refresh of every layer
+        for l in range(N):
+            fbk.prefix_partial(shape, ins[l][0][0], caches[l], pfxs[l], ws)
+
+    def seg_step():  # one denoising step of every layer
+        for l in range(N):
+            fbk.block_attn_merge(shape, ins[l][0][0], ins[l][1][0], ins[l][2][0], lens[l], pfxs[l], outs[l][0])
+
+    for r in intervals:
+        for _ in range(2):
+            run_block(r)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+
+    # accuracy of each interval against interval 1 (every step exact up to kernel rounding)
+    run_block(1)
+    torch.cuda.synchronize()
+    exact = torch.stack(outs).float()
+    acc = {}
+    for r in intervals:
+        run_block(r)
+        torch.cuda.synchronize()
+        d = (torch.stack(outs).float() - exact)
+        acc[r] = {"max_abs_vs_interval_1": float(d.abs().max()),
+                  "rel_l2_vs_interval_1": float(d.norm() / exact.norm())}
+    del exact
+
+    st = torch.cuda.Stream(dev)
+    st.wait_stream(torch.cuda.current_stream(dev))
+    graphs = {}
+    with torch.cuda.stream(st):
+        for key, fn in [(("block", r), (lambda r=r: run_block(r))) for r in intervals] + \
+                       [(("prefix", 0), seg_prefix), (("step", 0), seg_step)]:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st, capture_error_mode="thread_local"):
+                fn()
+            graphs[key] = g
+    torch.cuda.synchronize()
+
+    def timed(g, n):
+        evs = []
+        with torch.cuda.stream(st):
+            for _ in range(n):
+                flush.zero_()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e[0].record(st)
+                g.replay()
+                e[1].record(st)
+                evs.append(e)
+        return evs
+
+    main_r = intervals[0]
+    timed(graphs[("block", main_r)], args.warmup)
+    barrier(world)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    evs = timed(graphs[("block", main_r)], args.steps)
+    barrier(world)
+    clock_info = clocks.stop()
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), world)
+    assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+
+    sweep = []
+    for r in intervals:
+        ev = timed(graphs[("block", r)], max(3, args.steps // 2))
+        torch.cuda.synchronize()
+        ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+        sweep.append({"refresh_interval": r, "value": S / (ms * 1e-3), "unit": "denoising steps/s",
+                      "ms_per_block": ms, "refreshes_per_layer": -(-S // r), **acc[r]})
+    ev_p = timed(graphs[("prefix", 0)], max(3, args.steps // 2))
+    ev_s = timed(graphs[("step", 0)], max(3, args.steps // 2))
+    torch.cuda.synchronize()
+    pfx_launch_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev_p) / N
+    step_launch_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev_s) / N
+    n_ref = -(-S // main_r)
+    roofline, u = dominant_roofline(wl, n_ref * N * pfx_launch_ms, pfx_launch_ms, S * N * step_launch_ms,
+                                    step_launch_ms)
+
+    # end to end through the public API: each block's inputs for every layer
+    # go host -> device from pinned memory and every layer's outputs come back
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    h_out = [torch.empty(outs[0].shape, dtype=torch.bfloat16).pin_memory() for _ in range(N)]
+    ev_in, ev_done, ev_back = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
+
+    def e2e_blocks(n):
+        for k in range(n):
+            with torch.cuda.stream(s_in):
+                if k:
+                    s_in.wait_event(ev_done)  # the previous block no longer reads the inputs
+                for l in range(N):
+                    for dst, src in zip(ins[l], (h_q, h_k, h_v)):
+                        dst.copy_(src, non_blocking=True)
+                ev_in.record(s_in)
+            with torch.cuda.stream(st):
+                st.wait_event(ev_in)
+                if k:
+                    st.wait_event(ev_back)  # the previous outputs have left the device buffers
+                flush.zero_()
+                lens.copy_(lens0)
+                fbk.decode_block(shape, blocks_for(main_r), ws, commit=True, stream=st)
+                ev_done.record(st)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done)
+                for l in range(N):
+                    h_out[l].copy_(outs[l], non_blocking=True)
+                ev_back.record(s_out)
+
+    e2e_blocks(1)
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, args.steps // 4)
+    a.record(s_in)
+    st.wait_event(a)
+    s_out.wait_event(a)
+    e2e_blocks(n_e2e)
+    st.wait_event(ev_back)
+    b.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world)
+    h2d = N * (h_q.numel() + h_k.numel() + h_v.numel()) * 2
+    d2h = N * outs[0].numel() * 2
+
+    n_launch = N * (3 * n_ref + S + 2)
+    value = aggregate_steps_per_s(world, args.steps, S, total_ms)
+    line = {
+        "metric": METRIC, "value": value, "unit": "denoising steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "layers": N, "refresh_interval": main_r,
+                   "description": wl.description,
+                   "bench_step": f"one block of {N} layers x {S} denoising steps through one fbk_decode_block "
+                                 f"call (prefix state refreshed every {main_r} steps, then the commit), "
+                                 "one CUDA graph per block; a denoising step counts all layers",
+                   "l2": "flushed (2x L2 memset) before every timed block, outside the events",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": roofline,
+        "prefix_us": pfx_launch_ms * 1e3, "step_us": step_launch_ms * 1e3,
+        "interval_sweep": sweep,
+        "e2e": {"value": aggregate_steps_per_s(world, 1, S, e2e_ms), "unit": "denoising steps/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "one fbk_decode_block call per block; every layer's inputs H2D from pinned host and "
+                        "outputs D2H inside the timed region (copy-out of a block overlaps copy-in of the next)"},
+        "gpu_launches": n_launch * args.steps,
+        "clocks": clock_info,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        case = oracle_case(wl)
+        s = min(wl.steps, 8)
+        t0 = time.perf_counter()
+        oracle_layer_block(case, s, main_r)
+        one = time.perf_counter() - t0
+        n = max(1, min(20, int(12.0 / max(one, 1e-3))))
+        t0 = time.perf_counter()
+        for _ in range(n):
+            oracle_layer_block(case, s, main_r)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n * s / dt / N, "unit": "denoising steps/s", "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n} blocks of one layer ({s} steps, interval {main_r}, commit), "
+                                          f"fp64 numpy; value / {N} layers"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    graphs.clear()
+
+
+def layer_mode(args):
+    return args.layers > 1 or bool(args.refresh_interval)
+
+
+def intervals_of(args, wl):
+    return [int(x) for x in args.refresh_interval.split(",")] if args.refresh_interval else [wl.steps]
+
+
 def main():
     args = parse()
     from cached_block_attention_b200 import synth
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
-        run_reference(args, wl, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        if layer_mode(args):
+            run_reference_layers(args, wl, rank)
+        else:
+            run_reference(args, wl, rank, int(os.environ.get("WORLD_SIZE", "1")))
         return
     rank, world, local = dist_setup(args.gpus)
     try:
-        run_ours(args, wl, rank, world, local)
+        if layer_mode(args):
+            run_layers(args, wl, rank, world, local)
+        else:
+            run_ours(args, wl, rank, world, local)
     finally:
         if world > 1:
             import torch.distributed as dist

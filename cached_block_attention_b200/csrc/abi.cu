@@ -4,7 +4,9 @@
 #include <math.h>
 #include <string.h>
 
+#include <initializer_list>
 #include <mutex>
+#include <vector>
 
 #include "launch.h"
 
@@ -127,6 +129,79 @@ Workspace carve(const WsLayout &l, void *base) {
 
 fbk_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FBK_OK : FBK_ERR_CUDA; }
 
+bool misaligned16(std::initializer_list<const void *> ptrs) {
+  uintptr_t bits = 0;
+  for (const void *p : ptrs) bits |= reinterpret_cast<uintptr_t>(p);
+  return (bits & 15u) != 0;
+}
+
+// Host checks of fbk_prefix_partial's pointers (after check_shape and check_cache).
+fbk_status check_prefix_ptrs(const void *q_blk, const fbk_partial *out) {
+  if (!q_blk || !out || !out->o_unnorm || !out->m || !out->l) return FBK_ERR_INVALID_ARG;
+  if (misaligned16({q_blk, out->o_unnorm})) return FBK_ERR_UNSUPPORTED;
+  return FBK_OK;
+}
+
+// Host checks of fbk_block_attn_merge's pointers (after check_shape).
+fbk_status check_merge_ptrs(const void *q_blk, const void *k_blk, const void *v_blk,
+                            const int32_t *prefix_lens, const fbk_partial *prefix, const void *out) {
+  if (!q_blk || !k_blk || !v_blk || !prefix_lens || !prefix || !prefix->o_unnorm || !prefix->m ||
+      !prefix->l || !out)
+    return FBK_ERR_INVALID_ARG;
+  if (misaligned16({q_blk, k_blk, v_blk, out, prefix->o_unnorm})) return FBK_ERR_UNSUPPORTED;
+  return FBK_OK;
+}
+
+// Host checks of the commit's block pointers (after check_shape and check_cache).
+fbk_status check_commit_ptrs(const void *k_blk, const void *v_blk) {
+  if (!k_blk || !v_blk) return FBK_ERR_INVALID_ARG;
+  if (misaligned16({k_blk, v_blk})) return FBK_ERR_UNSUPPORTED;
+  return FBK_OK;
+}
+
+// Share count and workspace checks of a prefix computation.
+fbk_status check_workspace(const fbk_shape *shape, int32_t num_splits, const void *ws, size_t ws_bytes,
+                           int *shares, WsLayout *lay) {
+  *shares = num_splits ? num_splits : default_shares();
+  if (*shares < 1) return FBK_ERR_CUDA;
+  *lay = ws_layout(shape, *shares);
+  if (!ws || ws_bytes < lay->total) return FBK_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return FBK_ERR_UNSUPPORTED;  // TMA reads the query rows
+  return FBK_OK;
+}
+
+// The launches of one prefix computation: query rotation and share kernel (or
+// the fp32 share kernel), then the fixed-order split reduction.
+cudaError_t enqueue_prefix(const fbk_shape *shape, const Geometry &g, const void *q_blk, const Workspace &w,
+                           int shares, const fbk_partial &out, cudaStream_t s) {
+  const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_blk);
+  cudaError_t e = shape->mode == FBK_BF16 ? launch_prefix_tc(g, q, w, shares, s)
+                                          : launch_prefix_fp32(g, q, w, shares, s);
+  if (e != cudaSuccess) return e;
+  return launch_split_reduce(g, w, shares, out, s);
+}
+
+// Geometry of the step kernel: no cache, only the prefix lengths.
+Geometry merge_geometry(const fbk_shape *shape, const int32_t *prefix_lens) {
+  Geometry g = make_geometry(shape, nullptr);
+  g.lens = prefix_lens;
+  return g;
+}
+
+cudaError_t enqueue_merge(const fbk_shape *shape, const Geometry &g, const void *q_blk, const void *k_blk,
+                          const void *v_blk, const fbk_partial &prefix, void *out, float *lse, cudaStream_t s) {
+  return launch_block_merge(g, static_cast<const __nv_bfloat16 *>(q_blk), static_cast<const __nv_bfloat16 *>(k_blk),
+                            static_cast<const __nv_bfloat16 *>(v_blk), prefix, out, lse,
+                            shape->mode == FBK_FP32_CHECK, s);
+}
+
+cudaError_t enqueue_commit(const Geometry &g, const void *k_blk, const void *v_blk, const fbk_kv_cache *cache,
+                           cudaStream_t s) {
+  return launch_commit(g, static_cast<const __nv_bfloat16 *>(k_blk), static_cast<const __nv_bfloat16 *>(v_blk),
+                       static_cast<__nv_bfloat16 *>(cache->k), static_cast<__nv_bfloat16 *>(cache->v),
+                       cache->prefix_lens, s);
+}
+
 // Built-in scratch of fbk_prefix_partial_static_scratch: one array per device,
 // part of this file's device image, so using it allocates nothing.
 static __device__ __align__(256) unsigned char g_static_scratch[FBK_STATIC_SCRATCH_BYTES];
@@ -174,22 +249,13 @@ fbk_status fbk_prefix_partial(const fbk_shape *shape, const void *q_blk, const f
   fbk_status st = check_shape(shape);
   if (st != FBK_OK) return st;
   if ((st = check_cache(shape, cache)) != FBK_OK) return st;
-  if (!q_blk || !out || !out->o_unnorm || !out->m || !out->l || num_splits < 0) return FBK_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(q_blk) | reinterpret_cast<uintptr_t>(out->o_unnorm)) & 15u)
-    return FBK_ERR_UNSUPPORTED;
-  const int shares = num_splits ? num_splits : default_shares();
-  if (shares < 1) return FBK_ERR_CUDA;
-  const WsLayout lay = ws_layout(shape, shares);
-  if (!ws || ws_bytes < lay.total) return FBK_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(ws) & 255u) return FBK_ERR_UNSUPPORTED;  // TMA reads the query rows
-  const Workspace w = carve(lay, ws);
-  const Geometry g = make_geometry(shape, cache);
-  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_blk);
-  cudaError_t e = shape->mode == FBK_BF16 ? launch_prefix_tc(g, q, w, shares, s)
-                                          : launch_prefix_fp32(g, q, w, shares, s);
-  if (e != cudaSuccess) return FBK_ERR_CUDA;
-  return from_cuda(launch_split_reduce(g, w, shares, *out, s));
+  if (num_splits < 0) return FBK_ERR_INVALID_ARG;
+  if ((st = check_prefix_ptrs(q_blk, out)) != FBK_OK) return st;
+  int shares;
+  WsLayout lay;
+  if ((st = check_workspace(shape, num_splits, ws, ws_bytes, &shares, &lay)) != FBK_OK) return st;
+  return from_cuda(enqueue_prefix(shape, make_geometry(shape, cache), q_blk, carve(lay, ws), shares, *out,
+                                  static_cast<cudaStream_t>(cuda_stream)));
 }
 
 fbk_status fbk_block_attn_merge(const fbk_shape *shape, const void *q_blk, const void *k_blk,
@@ -197,20 +263,9 @@ fbk_status fbk_block_attn_merge(const fbk_shape *shape, const void *q_blk, const
                                 const fbk_partial *prefix, void *out, float *lse, void *cuda_stream) {
   fbk_status st = check_shape(shape);
   if (st != FBK_OK) return st;
-  if (!q_blk || !k_blk || !v_blk || !prefix_lens || !prefix || !prefix->o_unnorm || !prefix->m ||
-      !prefix->l || !out)
-    return FBK_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(q_blk) | reinterpret_cast<uintptr_t>(k_blk) |
-       reinterpret_cast<uintptr_t>(v_blk) | reinterpret_cast<uintptr_t>(out) |
-       reinterpret_cast<uintptr_t>(prefix->o_unnorm)) & 15u)
-    return FBK_ERR_UNSUPPORTED;
-  Geometry g = make_geometry(shape, nullptr);
-  g.lens = prefix_lens;
-  return from_cuda(launch_block_merge(g, static_cast<const __nv_bfloat16 *>(q_blk),
-                                      static_cast<const __nv_bfloat16 *>(k_blk),
-                                      static_cast<const __nv_bfloat16 *>(v_blk), *prefix, out, lse,
-                                      shape->mode == FBK_FP32_CHECK,
-                                      static_cast<cudaStream_t>(cuda_stream)));
+  if ((st = check_merge_ptrs(q_blk, k_blk, v_blk, prefix_lens, prefix, out)) != FBK_OK) return st;
+  return from_cuda(enqueue_merge(shape, merge_geometry(shape, prefix_lens), q_blk, k_blk, v_blk, *prefix, out,
+                                 lse, static_cast<cudaStream_t>(cuda_stream)));
 }
 
 fbk_status fbk_commit_block_rope_append(const fbk_shape *shape, const void *k_blk, const void *v_blk,
@@ -218,14 +273,9 @@ fbk_status fbk_commit_block_rope_append(const fbk_shape *shape, const void *k_bl
   fbk_status st = check_shape(shape);
   if (st != FBK_OK) return st;
   if ((st = check_cache(shape, cache)) != FBK_OK) return st;
-  if (!k_blk || !v_blk) return FBK_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(k_blk) | reinterpret_cast<uintptr_t>(v_blk)) & 15u)
-    return FBK_ERR_UNSUPPORTED;
-  const Geometry g = make_geometry(shape, cache);
-  return from_cuda(launch_commit(g, static_cast<const __nv_bfloat16 *>(k_blk),
-                                 static_cast<const __nv_bfloat16 *>(v_blk),
-                                 static_cast<__nv_bfloat16 *>(cache->k), static_cast<__nv_bfloat16 *>(cache->v),
-                                 cache->prefix_lens, static_cast<cudaStream_t>(cuda_stream)));
+  if ((st = check_commit_ptrs(k_blk, v_blk)) != FBK_OK) return st;
+  return from_cuda(enqueue_commit(make_geometry(shape, cache), k_blk, v_blk, cache,
+                                  static_cast<cudaStream_t>(cuda_stream)));
 }
 
 fbk_status fbk_full_ref_attn(const fbk_shape *shape, const void *q_blk, const void *k_blk,
@@ -251,23 +301,76 @@ fbk_status fbk_prefix_partial_static_scratch(const fbk_shape *shape, const void 
   fbk_status st = check_shape(shape);
   if (st != FBK_OK) return st;
   if ((st = check_cache(shape, cache)) != FBK_OK) return st;
-  if (!q_blk || !out || !out->o_unnorm || !out->m || !out->l || num_splits < 0) return FBK_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(q_blk) | reinterpret_cast<uintptr_t>(out->o_unnorm)) & 15u)
-    return FBK_ERR_UNSUPPORTED;
+  if (num_splits < 0) return FBK_ERR_INVALID_ARG;
+  if ((st = check_prefix_ptrs(q_blk, out)) != FBK_OK) return st;
   const int shares = num_splits ? num_splits : default_shares();
   if (shares < 1) return FBK_ERR_CUDA;
   const WsLayout lay = ws_layout(shape, shares);
   if (lay.total > (size_t)FBK_STATIC_SCRATCH_BYTES) return FBK_ERR_SCRATCH_LIMIT;
   void *scratch = nullptr;
   if ((st = static_scratch_address(&scratch)) != FBK_OK) return st;
-  const Workspace w = carve(lay, scratch);
-  const Geometry g = make_geometry(shape, cache);
+  return from_cuda(enqueue_prefix(shape, make_geometry(shape, cache), q_blk, carve(lay, scratch), shares, *out,
+                                  static_cast<cudaStream_t>(cuda_stream)));
+}
+
+fbk_status fbk_decode_block(const fbk_shape *shape, const fbk_layer_block *layers, int32_t n_layers,
+                            int32_t steps, int32_t commit, void *ws, size_t ws_bytes, int32_t num_splits,
+                            void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if (!layers || n_layers < 1 || steps < 1 || num_splits < 0) return FBK_ERR_INVALID_ARG;
+  // every layer is checked before the first launch
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const fbk_layer_block &L = layers[l];
+    if ((st = check_cache(shape, &L.cache)) != FBK_OK) return st;
+    if (L.refresh_interval < 1) return FBK_ERR_INVALID_ARG;
+    if ((st = check_prefix_ptrs(L.q, &L.prefix)) != FBK_OK) return st;
+    if ((st = check_merge_ptrs(L.q, L.k, L.v, L.cache.prefix_lens, &L.prefix, L.out)) != FBK_OK) return st;
+    if (commit) {
+      for (int32_t j = 0; j < l; ++j)  // a shared length array would be advanced once per layer
+        if (layers[j].cache.prefix_lens == L.cache.prefix_lens) return FBK_ERR_INVALID_ARG;
+    }
+  }
+  // element strides of one step inside each layer's step-major arrays
+  const size_t b = shape->batch, B = shape->block_len, d = shape->head_dim;
+  const size_t q_step = b * B * shape->n_q_heads * d, kv_step = b * B * shape->n_kv_heads * d;
+  const size_t out_step_bytes = q_step * (shape->mode == FBK_FP32_CHECK ? 4 : 2);
+  const size_t lse_step = b * shape->n_q_heads * B;
+  if ((size_t)steps > ((size_t)1 << 62) / (out_step_bytes * 2)) return FBK_ERR_CAPACITY;
+  int shares;
+  WsLayout lay;
+  if ((st = check_workspace(shape, num_splits, ws, ws_bytes, &shares, &lay)) != FBK_OK) return st;
+  const Workspace w = carve(lay, ws);
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_blk);
-  cudaError_t e = shape->mode == FBK_BF16 ? launch_prefix_tc(g, q, w, shares, s)
-                                          : launch_prefix_fp32(g, q, w, shares, s);
-  if (e != cudaSuccess) return FBK_ERR_CUDA;
-  return from_cuda(launch_split_reduce(g, w, shares, *out, s));
+
+  std::vector<Geometry> geo(n_layers);  // prefix and commit geometry of each layer
+  for (int32_t l = 0; l < n_layers; ++l) geo[l] = make_geometry(shape, &layers[l].cache);
+  Geometry gm = make_geometry(shape, nullptr);
+  auto at = [](const void *p, size_t bytes) { return static_cast<const char *>(p) + bytes; };
+
+  for (int32_t step = 0; step < steps; ++step) {
+    for (int32_t l = 0; l < n_layers; ++l) {
+      const fbk_layer_block &L = layers[l];
+      const void *q = at(L.q, step * q_step * 2);
+      if (step % L.refresh_interval == 0) {
+        if (enqueue_prefix(shape, geo[l], q, w, shares, L.prefix, s) != cudaSuccess) return FBK_ERR_CUDA;
+      }
+      gm.lens = L.cache.prefix_lens;
+      void *out = static_cast<char *>(L.out) + step * out_step_bytes;
+      float *lse = L.lse ? L.lse + step * lse_step : nullptr;
+      if (enqueue_merge(shape, gm, q, at(L.k, step * kv_step * 2), at(L.v, step * kv_step * 2), L.prefix, out, lse,
+                        s) != cudaSuccess)
+        return FBK_ERR_CUDA;
+    }
+  }
+  if (commit) {
+    for (int32_t l = 0; l < n_layers; ++l) {
+      const fbk_layer_block &L = layers[l];
+      const size_t last = (size_t)(steps - 1) * kv_step * 2;
+      if (enqueue_commit(geo[l], at(L.k, last), at(L.v, last), &L.cache, s) != cudaSuccess) return FBK_ERR_CUDA;
+    }
+  }
+  return FBK_OK;
 }
 
 const char *fbk_status_string(fbk_status status) {

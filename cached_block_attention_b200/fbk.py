@@ -33,7 +33,7 @@ DEVERR_TIMEOUT = 8
 
 EXPORTS = ("fbk_prefix_workspace_bytes", "fbk_default_num_splits", "fbk_prefix_partial",
            "fbk_block_attn_merge", "fbk_commit_block_rope_append", "fbk_full_ref_attn",
-           "fbk_status_string", "fbk_prefix_partial_static_scratch")
+           "fbk_status_string", "fbk_prefix_partial_static_scratch", "fbk_decode_block")
 
 STATIC_SCRATCH_BYTES = 32 << 20  # FBK_STATIC_SCRATCH_BYTES
 
@@ -57,6 +57,12 @@ class _Partial(ctypes.Structure):
     _fields_ = [("o_unnorm", ctypes.c_void_p), ("m", ctypes.c_void_p), ("l", ctypes.c_void_p)]
 
 
+class _LayerBlock(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("cache", _Cache), ("prefix", _Partial), ("out", ctypes.c_void_p),
+                ("lse", ctypes.c_void_p), ("refresh_interval", ctypes.c_int32)]
+
+
 _P = ctypes.POINTER
 _vp = ctypes.c_void_p
 _lib.fbk_prefix_workspace_bytes.argtypes = [_P(_Shape), _P(_Cache), ctypes.c_int32]
@@ -75,6 +81,9 @@ _lib.fbk_full_ref_attn.restype = ctypes.c_int
 _lib.fbk_prefix_partial_static_scratch.argtypes = [_P(_Shape), _vp, _P(_Cache), _P(_Partial),
                                                    ctypes.c_int32, _vp]
 _lib.fbk_prefix_partial_static_scratch.restype = ctypes.c_int
+_lib.fbk_decode_block.argtypes = [_P(_Shape), _P(_LayerBlock), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                  _vp, ctypes.c_size_t, ctypes.c_int32, _vp]
+_lib.fbk_decode_block.restype = ctypes.c_int
 _lib.fbk_status_string.argtypes = [ctypes.c_int]
 _lib.fbk_status_string.restype = ctypes.c_char_p
 
@@ -216,6 +225,41 @@ def full_ref_attn(shape: Shape, q_blk, k_blk, v_blk, cache: KVCache, out, lse=No
            "fbk_full_ref_attn")
 
 
+@dataclass
+class LayerBlock:
+    """One layer's buffers for decode_block: q [S, b, B, Hq, d], k / v [S, b, B, Hkv, d]
+    (bf16, pre-RoPE), out [S, b, B, Hq, d], lse [S, b, Hq, B] or None, and the
+    layer's cache, prefix state and cache update interval."""
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    cache: KVCache
+    prefix: Partial
+    out: torch.Tensor
+    refresh_interval: int
+    lse: torch.Tensor | None = None
+
+    def c(self) -> _LayerBlock:
+        return _LayerBlock(self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(), self.cache.c(),
+                           self.prefix.c(), self.out.data_ptr(),
+                           self.lse.data_ptr() if self.lse is not None else None, self.refresh_interval)
+
+
+def decode_block(shape: Shape, layers, ws: torch.Tensor, commit: bool = True, num_splits: int = 0,
+                 stream=None) -> None:
+    """All denoising steps of one block for every layer in `layers` (one C call):
+    prefix refresh every refresh_interval steps, a step output per step, then
+    (commit=True) the commit of each layer's last-step K/V."""
+    steps = {int(L.q.shape[0]) for L in layers}
+    if len(steps) != 1:
+        raise ValueError(f"layers disagree on the number of steps: {sorted(steps)}")
+    arr = (_LayerBlock * len(layers))(*[L.c() for L in layers])
+    cs = shape.c()
+    _check(_lib.fbk_decode_block(ctypes.byref(cs), arr, len(layers), steps.pop(), 1 if commit else 0,
+                                 _ptr(ws), ws.numel() * ws.element_size(), num_splits, _stream(stream)),
+           "fbk_decode_block")
+
+
 # raw handles for tests of the C ABI itself
 lib = _lib
-CShape, CCache, CPartial = _Shape, _Cache, _Partial
+CShape, CCache, CPartial, CLayerBlock = _Shape, _Cache, _Partial, _LayerBlock

@@ -17,8 +17,8 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Memory. Every pointer argument is DEVICE memory owned by the caller,
- *    except the structs themselves (fbk_shape, fbk_kv_cache, fbk_partial),
- *    which are host structs read during the call only. The library allocates
+ *    except the structs themselves (fbk_shape, fbk_kv_cache, fbk_partial,
+ *    fbk_layer_block), which are host structs read during the call only. The library allocates
  *    nothing and never synchronises. Apart from fbk_prefix_partial_static_scratch
  *    (last below), it keeps no state between calls.
  *  - Streams. `cuda_stream` is a cudaStream_t (NULL = legacy default stream).
@@ -167,7 +167,9 @@ fbk_status fbk_block_attn_merge(const fbk_shape *shape, const void *q_blk, const
  * rounded once to bf16 (nearest even), V copied bit for bit, both written to
  * cache slots L_b .. L_b+B-1; then prefix_lens[b] += B (RoPECache,
  * LaCache §3.3.2, Eq. 1). A sequence whose block does not fit is left
- * unchanged and FBK_DEVERR_COMMIT is flagged. One CTA per sequence. */
+ * unchanged and FBK_DEVERR_COMMIT is flagged. Two launches: the rows (one
+ * CTA per sequence, block token and group of up to 16 kv-heads), then the
+ * length update. */
 fbk_status fbk_commit_block_rope_append(const fbk_shape *shape, const void *k_blk,
                                         const void *v_blk, fbk_kv_cache *cache,
                                         void *cuda_stream);
@@ -222,6 +224,54 @@ fbk_status fbk_full_ref_attn(const fbk_shape *shape, const void *q_blk, const vo
 fbk_status fbk_prefix_partial_static_scratch(const fbk_shape *shape, const void *q_blk,
                                              const fbk_kv_cache *cache, const fbk_partial *out,
                                              int32_t num_splits, void *cuda_stream);
+
+/* One layer's buffers for fbk_decode_block. The inputs of every denoising
+ * step of the block are stored step-major: step s of q starts s*b*B*Hq*d
+ * elements after q, step s of k and v s*b*B*Hkv*d elements after k and v. */
+typedef struct fbk_layer_block {
+  const void *q;            /* bf16 [steps, b, B, Hq, d], pre-RoPE block queries, 16-byte aligned */
+  const void *k;            /* bf16 [steps, b, B, Hkv, d], pre-RoPE block keys, 16-byte aligned */
+  const void *v;            /* bf16 [steps, b, B, Hkv, d], block values, 16-byte aligned */
+  fbk_kv_cache cache;       /* this layer's cache and prefix lengths */
+  fbk_partial prefix;       /* this layer's prefix state (rewritten at every refresh) */
+  void *out;                /* [steps, b, B, Hq, d]: bf16 (FBK_BF16) or fp32 (FBK_FP32_CHECK) */
+  float *lse;               /* fp32 [steps, b, Hq, B], or NULL */
+  int32_t refresh_interval; /* r >= 1, see fbk_decode_block */
+} fbk_layer_block;
+
+/* Every denoising step of one block for n_layers attention layers, in one
+ * call, with a cache update interval per layer (LaCache App. C: the longer
+ * the interval, the faster the decoding and the larger the error).
+ *
+ * For step s = 0 .. steps-1, and within a step for layer l = 0 .. n_layers-1:
+ *   if s % r_l == 0, the layer's prefix state is recomputed from step s's block
+ *   queries (the launches of fbk_prefix_partial, same workspace rules);
+ *   then the step output of layer l (fbk_block_attn_merge), into out[s] and lse[s].
+ * Then, if commit != 0, each layer commits the K and V of the last step
+ * (fbk_commit_block_rope_append), which advances its prefix_lens by B.
+ *
+ * r_l = 1 is the recompute-every-step schedule: every step is exact full
+ * attention over prefix and block. r_l >= steps computes the state once per
+ * block from step 0's queries (FlashBlock's reuse of the block-external
+ * attention). Intervals may differ between layers, for instance to refresh
+ * deeper layers more often.
+ *
+ *  layers: host array of n_layers structs, read during the call only.
+ *  ws, ws_bytes, num_splits: as for fbk_prefix_partial; one workspace serves
+ *         every layer, since all launches are ordered on the one stream.
+ *  commit: with commit != 0 no two layers may share a prefix_lens array
+ *         (FBK_ERR_INVALID_ARG), since each layer's commit advances its own.
+ *
+ * Every argument of every layer is checked before the first launch, with
+ * the codes of the single calls. If a launch fails, FBK_ERR_CUDA is returned
+ * and the launches before it stay enqueued. Like every call here, this one
+ * only enqueues work, so a whole block can be captured as one CUDA graph. The
+ * pages have no counterpart to the call itself: it is the loop over steps and
+ * layers that a decoder runs, moved into the library so that the launches are
+ * issued from native code. */
+fbk_status fbk_decode_block(const fbk_shape *shape, const fbk_layer_block *layers, int32_t n_layers,
+                            int32_t steps, int32_t commit, void *ws, size_t ws_bytes,
+                            int32_t num_splits, void *cuda_stream);
 
 /* Static text for a status code. */
 const char *fbk_status_string(fbk_status status);

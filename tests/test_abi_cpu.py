@@ -144,3 +144,40 @@ def test_static_scratch_covers_every_workload(fbk, name):
     units = wl.batch * wl.n_kv_heads
     assert n >= (148 + units) * rows * (wl.head_dim + 2) * 4 + units * 128 * ((rows + 127) // 128) * wl.head_dim * 2
     assert n <= fbk.STATIC_SCRATCH_BYTES
+
+
+def _layer(fbk, lens=0x30000, interval=2, q=0x70000, cache_kw=None):
+    c = _cache(fbk, prefix_lens=lens, **(cache_kw or {}))
+    return fbk.CLayerBlock(q, 0x71000, 0x72000, c, fbk.CPartial(0x40000, 0x50000, 0x60000), 0x90000, None,
+                           interval)
+
+
+def _decode(fbk, layers, steps=4, commit=1, ws=None, ws_bytes=0, splits=4, shape=None):
+    s = shape or _shape(fbk)
+    arr = (fbk.CLayerBlock * max(1, len(layers)))(*layers)
+    return fbk.lib.fbk_decode_block(ctypes.byref(s), arr if layers else None, len(layers), steps, commit,
+                                    ctypes.c_void_p(ws) if ws else None, ws_bytes, splits, None)
+
+
+def test_decode_block_argument_checks(fbk):
+    """fbk_decode_block checks every layer before any launch; a workspace that
+    is missing (-4) is the last check, so reaching it means the rest passed."""
+    ok = [_layer(fbk, lens=0x30000), _layer(fbk, lens=0x31000, interval=1)]
+    assert _decode(fbk, ok) == -4
+    assert _decode(fbk, []) == -1                                     # no layers
+    assert _decode(fbk, ok, steps=0) == -1
+    assert _decode(fbk, ok, splits=-1) == -1
+    assert _decode(fbk, ok, shape=_shape(fbk, head_dim=96)) == -2
+    assert _decode(fbk, [ok[0], _layer(fbk, lens=0x31000, interval=0)]) == -1
+    assert _decode(fbk, [ok[0], _layer(fbk, lens=0x31000, cache_kw=dict(k=None))]) == -1
+    assert _decode(fbk, [ok[0], _layer(fbk, lens=0x31000, q=0x70008)]) == -2
+    bad_prefix = _layer(fbk, lens=0x31000)
+    bad_prefix.prefix = fbk.CPartial(0x40000, None, 0x60000)
+    assert _decode(fbk, [ok[0], bad_prefix]) == -1
+    # a shared length array is refused only when the layers commit
+    shared = [_layer(fbk, lens=0x30000), _layer(fbk, lens=0x30000)]
+    assert _decode(fbk, shared, commit=1) == -1
+    assert _decode(fbk, shared, commit=0) == -4
+    n = fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(_shape(fbk)), None, 4)
+    assert _decode(fbk, ok, ws=0x100000, ws_bytes=n - 1) == -4
+    assert _decode(fbk, ok, ws=0x100010, ws_bytes=n) == -2          # workspace not 256-byte aligned
