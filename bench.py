@@ -42,6 +42,9 @@ def parse():
     ap.add_argument("--workload", default="llada8b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="attention", choices=["attention", "fp8_group_quant"],
+                    help="attention: the cached block attention block (default); fp8_group_quant: the "
+                         "per-group FP8 activation quantisation on the FP8_WORKLOADS shapes")
     ap.add_argument("--layers", type=int, default=1,
                     help="attention layers per block; > 1 runs the whole block through fbk_decode_block")
     ap.add_argument("--refresh-interval", default="",
@@ -58,6 +61,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "cached_block_attention_b200", "ncu_traffic.js
 KERNEL_SOURCES = {
     "block_merge_mma_kernel": ["block_merge.cu", "common.cuh", "tc.cuh", "launch.h"],
     "prefix_tc_kernel": ["prefix_tc.cu", "common.cuh", "tc.cuh", "launch.h"],
+    "fp8_group_quant_kernel": ["fp8_quant.cu", "common.cuh", "launch.h"],
 }
 API_KERNEL = {"fbk_block_attn_merge": "block_merge_mma_kernel", "fbk_prefix_partial": "prefix_tc_kernel"}
 
@@ -841,6 +845,159 @@ def run_layers(args, wl, rank, world, local):
     graphs.clear()
 
 
+# ------------------------------------------------------------------ per-group FP8 quantisation
+
+# FFN activations of the LLaDA-8B-shaped sequence (prefix 4096 + block 32 tokens):
+# the gate-up input (hidden width 4096) and the ffout input (FFN width 12288).
+FP8_WORKLOADS = {
+    "ffn_out_llada8b": (4128, 12288, 12288),   # rows, cols, seed
+    "ffn_in_llada8b": (4128, 4096, 4096),
+}
+FP8_METRIC = "per-group FP8 (E4M3, 1x128) activation quantisation, algorithmic GB/s (1×B200)"
+
+
+def fp8_bytes(rows, cols):
+    """Algorithmic bytes of one quantisation: bf16 in, E4M3 codes and fp32 scales out."""
+    return rows * cols * 2 + rows * cols + rows * (cols // 128) * 4
+
+
+def oracle_fp8_sample(x_bits, budget_s=10.0):
+    """The oracle on repeated 256-row samples for about budget_s seconds: GB/s."""
+    from oracle import fp8_quant as fq
+    sample = x_bits[:256]
+    t0 = time.perf_counter()
+    fq.fp8_group_quant(sample)
+    one = time.perf_counter() - t0
+    n = max(1, min(50, int(budget_s / max(one, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(n):
+        fq.fp8_group_quant(sample)
+    dt = time.perf_counter() - t0
+    return n * fp8_bytes(*sample.shape) / dt / 1e9, n
+
+
+def run_fp8_reference(args, name, rank):
+    if rank != 0:
+        return
+    from cached_block_attention_b200 import synth
+    rows, cols, seed = FP8_WORKLOADS[name]
+    x = synth.gen_activations(rows, cols, seed)
+    from oracle import fp8_quant as fq
+    sample = x[:256]
+    for _ in range(args.warmup):
+        fq.fp8_group_quant(sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fq.fp8_group_quant(sample)
+    dt = time.perf_counter() - t0
+    v = args.steps * fp8_bytes(*sample.shape) / dt / 1e9
+    line = {"impl": "reference", "metric": FP8_METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": name, "rows": rows, "cols": cols},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"256 of the {rows} rows per bench step, numpy"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_fp8(args, name, rank, world, local):
+    """One bench step = one fbk_fp8_group_quant launch over the whole activation
+    matrix, resident in HBM, after an L2 flush (the input alone fits in L2)."""
+    import torch
+    from cached_block_attention_b200 import fbk, synth
+    dev = torch.device("cuda", local)
+    rows, cols, seed = FP8_WORKLOADS[name]
+    x_bits = synth.gen_activations(rows, cols, seed)
+    h_x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    x = h_x.to(dev)
+    codes = torch.empty(rows, cols, dtype=torch.uint8, device=dev)
+    scales = torch.empty(rows, cols // 128, dtype=torch.float32, device=dev)
+    h_codes = torch.empty(rows, cols, dtype=torch.uint8).pin_memory()
+    h_scales = torch.empty(rows, cols // 128, dtype=torch.float32).pin_memory()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    st = torch.cuda.Stream(dev)
+    nbytes = fp8_bytes(rows, cols)
+
+    def timed(n):
+        evs = []
+        with torch.cuda.stream(st):
+            for _ in range(n):
+                flush.zero_()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e[0].record(st)
+                fbk.fp8_group_quant(x, codes, scales, stream=st)
+                e[1].record(st)
+                evs.append(e)
+        return evs
+
+    timed(max(3, args.warmup))
+    barrier(world)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    evs = timed(args.steps)
+    barrier(world)
+    clock_info = clocks.stop()
+    t = [e[0].elapsed_time(e[1]) for e in evs]
+    total_ms = max_over_ranks(sum(t), world)
+    launch_ms = sum(t) / len(t)
+
+    # end to end: the activations H2D from pinned memory, the launch, codes and scales D2H
+    def e2e(n):
+        with torch.cuda.stream(st):
+            for _ in range(n):
+                x.copy_(h_x, non_blocking=True)
+                fbk.fp8_group_quant(x, codes, scales, stream=st)
+                h_codes.copy_(codes, non_blocking=True)
+                h_scales.copy_(scales, non_blocking=True)
+    e2e(1)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, args.steps // 2)
+    a.record(st)
+    e2e(n_e2e)
+    b.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world)
+
+    hbm_gbs, _, _, peak_kind = load_peaks()
+    achieved = nbytes / (launch_ms * 1e-3) / 1e9
+    tr = measured_traffic("fp8_group_quant_kernel", name)
+    line = {
+        "metric": FP8_METRIC, "value": world * args.steps * nbytes / (total_ms * 1e-3) / 1e9, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": name, "rows": rows, "cols": cols, "group": 128,
+                   "description": "bf16 activations N(0,1) with 1% outlier columns x20 -> E4M3 codes + fp32 "
+                                  "scales per 1x128 group (LaCache §3.4 Eq. 7-8)",
+                   "bench_step": "one fbk_fp8_group_quant launch over the whole matrix",
+                   "l2": "flushed (2x L2 memset) before every timed launch, outside the events",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                     "frac": achieved / hbm_gbs, "peak_kind": f"{peak_kind} hbm_gbs",
+                     "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                     "traffic_source": tr["profile"] if tr else "no ncu capture of the current kernel source",
+                     "kernel": "fbk_fp8_group_quant", "algorithmic_bytes_per_launch": nbytes,
+                     "launch_us": launch_ms * 1e3},
+        "elements_per_s": rows * cols / (launch_ms * 1e-3),
+        "e2e": {"value": world * nbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": rows * cols * 2, "d2h_bytes_per_step": rows * cols + rows * (cols // 128) * 4,
+                "note": "activations H2D from pinned host, the launch, codes and scales D2H, one stream"},
+        "gpu_launches": args.steps,
+        "clocks": clock_info,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n = oracle_fp8_sample(x_bits)
+        line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{n} x 256 of the {rows} rows, numpy"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def layer_mode(args):
     return args.layers > 1 or bool(args.refresh_interval)
 
@@ -852,6 +1009,19 @@ def intervals_of(args, wl):
 def main():
     args = parse()
     from cached_block_attention_b200 import synth
+    if args.op == "fp8_group_quant":
+        name = args.workload if args.workload in FP8_WORKLOADS else "ffn_out_llada8b"
+        if args.impl == "reference":
+            run_fp8_reference(args, name, int(os.environ.get("RANK", "0")))
+            return
+        rank, world, local = dist_setup(args.gpus)
+        try:
+            run_fp8(args, name, rank, world, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))

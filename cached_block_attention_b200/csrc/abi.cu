@@ -11,6 +11,11 @@
 #include "launch.h"
 
 namespace fbk {
+
+// Per-group FP8 quantisation (fp8_quant.cu).
+cudaError_t launch_fp8_group_quant(const __nv_bfloat16 *x, long long groups, uint8_t *codes, float *scales,
+                                   int sms, cudaStream_t st);
+
 namespace {
 
 bool is_pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -371,6 +376,22 @@ fbk_status fbk_decode_block(const fbk_shape *shape, const fbk_layer_block *layer
     }
   }
   return FBK_OK;
+}
+
+fbk_status fbk_fp8_group_quant(const void *x, int64_t rows, int64_t cols, void *codes, float *scales,
+                               void *cuda_stream) {
+  if (rows < 0 || cols < 0 || cols % FBK_FP8_GROUP != 0) return FBK_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return FBK_OK;  // nothing to quantise, nothing enqueued
+  if (rows > ((int64_t)1 << 40) / cols) return FBK_ERR_CAPACITY;
+  if (!x || !codes || !scales) return FBK_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(codes) & 7u) ||
+      (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return FBK_ERR_UNSUPPORTED;
+  const int sms = default_shares();
+  if (sms < 1) return FBK_ERR_CUDA;
+  return from_cuda(launch_fp8_group_quant(static_cast<const __nv_bfloat16 *>(x), rows * cols / FBK_FP8_GROUP,
+                                          static_cast<uint8_t *>(codes), scales, sms,
+                                          static_cast<cudaStream_t>(cuda_stream)));
 }
 
 const char *fbk_status_string(fbk_status status) {

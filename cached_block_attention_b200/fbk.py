@@ -33,7 +33,8 @@ DEVERR_TIMEOUT = 8
 
 EXPORTS = ("fbk_prefix_workspace_bytes", "fbk_default_num_splits", "fbk_prefix_partial",
            "fbk_block_attn_merge", "fbk_commit_block_rope_append", "fbk_full_ref_attn",
-           "fbk_status_string", "fbk_prefix_partial_static_scratch", "fbk_decode_block")
+           "fbk_status_string", "fbk_prefix_partial_static_scratch", "fbk_decode_block",
+           "fbk_fp8_group_quant")
 
 STATIC_SCRATCH_BYTES = 32 << 20  # FBK_STATIC_SCRATCH_BYTES
 
@@ -84,6 +85,8 @@ _lib.fbk_prefix_partial_static_scratch.restype = ctypes.c_int
 _lib.fbk_decode_block.argtypes = [_P(_Shape), _P(_LayerBlock), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                   _vp, ctypes.c_size_t, ctypes.c_int32, _vp]
 _lib.fbk_decode_block.restype = ctypes.c_int
+_lib.fbk_fp8_group_quant.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
+_lib.fbk_fp8_group_quant.restype = ctypes.c_int
 _lib.fbk_status_string.argtypes = [ctypes.c_int]
 _lib.fbk_status_string.restype = ctypes.c_char_p
 
@@ -258,6 +261,19 @@ def decode_block(shape: Shape, layers, ws: torch.Tensor, commit: bool = True, nu
     _check(_lib.fbk_decode_block(ctypes.byref(cs), arr, len(layers), steps.pop(), 1 if commit else 0,
                                  _ptr(ws), ws.numel() * ws.element_size(), num_splits, _stream(stream)),
            "fbk_decode_block")
+
+
+FP8_GROUP = 128  # FBK_FP8_GROUP
+
+
+def fp8_group_quant(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, stream=None) -> None:
+    """Per-group FP8 (E4M3) quantisation: x bf16 [rows, cols] -> codes uint8
+    [rows, cols] and scales fp32 [rows, cols // 128]."""
+    if x.dim() != 2:
+        raise ValueError("x must be a 2-D [rows, cols] tensor")
+    rows, cols = x.shape
+    _check(_lib.fbk_fp8_group_quant(_ptr(x), rows, cols, _ptr(codes), _ptr(scales), _stream(stream)),
+           "fbk_fp8_group_quant")
 
 
 # raw handles for tests of the C ABI itself

@@ -24,6 +24,10 @@ Recipe (per workload):
   * paged layout: pages of ``page_size`` tokens, room for one more block per
     sequence; physical page ids are ``Generator(PCG64(page_seed)).permutation``
     of the logical pages.
+  * FFN activations for the per-group FP8 quantisation (LaCache §3.4, whose
+    Fig. 4 shows activation peaks): ``Generator(PCG64(seed))`` draws x
+    [rows, cols] from N(0, 1), then picks ``round(0.01 * cols)`` distinct
+    outlier columns and multiplies them by 20; rounded to bf16.
 """
 from __future__ import annotations
 
@@ -168,6 +172,17 @@ def gen_random(shape, seed, scale=1.0):
 
 
 # ---------------------------------------------------------------- layouts
+
+def gen_activations(rows: int, cols: int, seed: int, outlier_frac: float = 0.01,
+                    outlier_gain: float = 20.0) -> np.ndarray:
+    """FFN input activations [rows, cols] (bf16 bits) with outlier channels."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = rng.standard_normal((rows, cols), dtype=np.float32)
+    n_out = int(round(outlier_frac * cols))
+    if n_out:
+        x[:, rng.choice(cols, size=n_out, replace=False)] *= np.float32(outlier_gain)
+    return bf16_bits(x)
+
 
 def contiguous_cache(ks, vs, n_kv_heads, head_dim, capacity):
     """Pack per-sequence prefixes into [b, Hkv, capacity, d] (zeros past L_b)."""

@@ -273,6 +273,30 @@ fbk_status fbk_decode_block(const fbk_shape *shape, const fbk_layer_block *layer
                             int32_t steps, int32_t commit, void *ws, size_t ws_bytes,
                             int32_t num_splits, void *cuda_stream);
 
+/* Elements per quantisation group of fbk_fp8_group_quant (1 x 128). */
+#define FBK_FP8_GROUP 128
+
+/* Per-group FP8 quantisation of activations (LaCache §3.4, Mixed precision
+ * strategy, Eq. 7-8): the FFN input is cut into groups of 1 x FBK_FP8_GROUP
+ * consecutive elements of a row, and for each group g
+ *   scale_g = max_{i in g} |x_i| / 448                          (Eq. 8)
+ *   x'_i    = E4M3(clip(x_i / scale_g, -448, 448)),  i in g     (Eq. 7)
+ * so that x_i ~ x'_i * scale_g. E4M3 is the OCP FP8 format with 4 exponent
+ * bits (bias 7) and 3 mantissa bits, largest finite value 448. Both divisions
+ * are IEEE fp32 divisions; the quotient is rounded to E4M3 to nearest, ties
+ * to even. A group whose elements are all zero gets scale 0 and keeps its
+ * zeros (with their signs) as codes. Inputs must be finite.
+ *  x:      bf16 [rows, cols], row-major, 16-byte aligned.
+ *  rows, cols: rows >= 0, cols >= 0 and a multiple of FBK_FP8_GROUP
+ *          (FBK_ERR_INVALID_ARG otherwise); rows * cols <= 2^40
+ *          (FBK_ERR_CAPACITY). rows == 0 or cols == 0 enqueues nothing.
+ *  codes:  uint8 [rows, cols] E4M3 codes, 8-byte aligned.
+ *  scales: fp32 [rows, cols / FBK_FP8_GROUP], 4-byte aligned; group j of row r
+ *          at r * cols / FBK_FP8_GROUP + j.
+ * One launch. Misaligned pointers return FBK_ERR_UNSUPPORTED. */
+fbk_status fbk_fp8_group_quant(const void *x, int64_t rows, int64_t cols, void *codes, float *scales,
+                               void *cuda_stream);
+
 /* Static text for a status code. */
 const char *fbk_status_string(fbk_status status);
 

@@ -181,3 +181,21 @@ def test_decode_block_argument_checks(fbk):
     n = fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(_shape(fbk)), None, 4)
     assert _decode(fbk, ok, ws=0x100000, ws_bytes=n - 1) == -4
     assert _decode(fbk, ok, ws=0x100010, ws_bytes=n) == -2          # workspace not 256-byte aligned
+
+
+def test_fp8_group_quant_argument_checks(fbk):
+    """Host checks of fbk_fp8_group_quant; none of these reach a CUDA call."""
+    q = fbk.lib.fbk_fp8_group_quant
+    x, c, s = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000)
+    assert q(x, 4, 100, c, s, None) == -1                   # cols not a multiple of 128
+    assert q(x, -1, 128, c, s, None) == -1
+    assert q(x, 4, -128, c, s, None) == -1
+    assert q(None, 0, 128, None, None, None) == 0           # empty: nothing enqueued
+    assert q(None, 4, 0, None, None, None) == 0
+    assert q(None, 4, 128, c, s, None) == -1
+    assert q(x, 4, 128, None, s, None) == -1
+    assert q(x, 4, 128, c, None, None) == -1
+    assert q(ctypes.c_void_p(0x10008), 4, 128, c, s, None) == -2   # x not 16-byte aligned
+    assert q(x, 4, 128, ctypes.c_void_p(0x20004), s, None) == -2   # codes not 8-byte aligned
+    assert q(x, 4, 128, c, ctypes.c_void_p(0x30002), None) == -2   # scales not 4-byte aligned
+    assert q(x, 1 << 33, 1 << 8, c, s, None) == -3          # more than 2^40 elements

@@ -40,7 +40,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_rank_max_and_aggregate():
     os.environ["PYTHONPATH"] = ROOT + os.pathsep + os.environ.get("PYTHONPATH", "")
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a multi-threaded process
     out = mgr.dict()
     mp.spawn(_rank_main, args=(2, _free_port(), out), nprocs=2, join=True)
     for rank in (0, 1):
