@@ -91,6 +91,24 @@ def test_special_values():
     check(bits, "special values")
 
 
+def test_every_scale():
+    """Every positive finite bf16 max|x| A (so every scale the kernel can
+    meet), twice: a group of A and its 127 bf16 predecessors (quotients in the
+    densest code range below 448) and a group of A and 127 random bf16 values
+    below it; signs alternate. Exercises the shared-reciprocal division of
+    every scale, its IEEE fallback for tiny groups and elements, and the
+    subnormal codes."""
+    r = np.random.Generator(np.random.PCG64(17))
+    A = np.arange(1, 0x7F80, dtype=np.int64)                       # bf16 bit patterns of A > 0
+    pred = np.maximum(A[:, None] - np.arange(1, 128)[None, :], 0)  # 127 predecessors (0 below the bottom)
+    rand = (r.random((len(A), 127)) * A[:, None]).astype(np.int64)  # random patterns below A
+    sign = np.where(np.arange(127) % 2, 0x8000, 0)[None, :]
+    g1 = np.concatenate([A[:, None], pred | sign], axis=1)
+    g2 = np.concatenate([A[:, None] | 0x8000, rand | sign], axis=1)
+    bits = np.concatenate([g1, g2], axis=0).astype(np.uint16)      # [2 * 32639, 128]
+    check(bits, "every scale", chunk=8192)
+
+
 def test_hand_computed_fixture():
     """The hand-computed fixture through the kernel: codes and scales equal the
     values worked out from Eq. 7-8 and the E4M3 format by hand."""
