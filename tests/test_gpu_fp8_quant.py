@@ -95,9 +95,9 @@ def test_every_scale():
     """Every positive finite bf16 max|x| A (so every scale the kernel can
     meet), twice: a group of A and its 127 bf16 predecessors (quotients in the
     densest code range below 448) and a group of A and 127 random bf16 values
-    below it; signs alternate. Exercises the shared-reciprocal division of
-    every scale, its IEEE fallback for tiny groups and elements, and the
-    subnormal codes."""
+    below it; signs alternate. Exercises the shared-reciprocal division at
+    every scale, the IEEE division of tiny groups, tiny elements of normal
+    groups, and the subnormal codes."""
     r = np.random.Generator(np.random.PCG64(17))
     A = np.arange(1, 0x7F80, dtype=np.int64)                       # bf16 bit patterns of A > 0
     pred = np.maximum(A[:, None] - np.arange(1, 128)[None, :], 0)  # 127 predecessors (0 below the bottom)
