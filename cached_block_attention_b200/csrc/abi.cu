@@ -8,6 +8,7 @@
 #include <mutex>
 #include <vector>
 
+#include "facache_rows.h"
 #include "launch.h"
 
 namespace fbk {
@@ -16,11 +17,14 @@ namespace fbk {
 cudaError_t launch_fp8_group_quant(const __nv_bfloat16 *x, long long groups, uint8_t *codes, float *scales,
                                    int sms, cudaStream_t st);
 
+
 namespace {
 
 bool is_pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
 
-fbk_status check_shape(const fbk_shape *s) {
+// rows_limit: the block path keeps a kv-head's G*B query rows in at most two
+// 128-row tiles; entry points whose rows are not the block's skip that limit.
+fbk_status check_shape(const fbk_shape *s, bool rows_limit = true) {
   if (!s) return FBK_ERR_INVALID_ARG;
   if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_heads < 1 || s->block_len < 1 || s->head_dim < 1)
     return FBK_ERR_INVALID_ARG;
@@ -31,7 +35,7 @@ fbk_status check_shape(const fbk_shape *s) {
   if (s->head_dim != 64 && s->head_dim != 128) return FBK_ERR_UNSUPPORTED;
   if (s->n_q_heads % s->n_kv_heads != 0) return FBK_ERR_UNSUPPORTED;
   if (s->block_len > 64) return FBK_ERR_UNSUPPORTED;
-  if ((long long)(s->n_q_heads / s->n_kv_heads) * s->block_len > 256) return FBK_ERR_UNSUPPORTED;
+  if (rows_limit && (long long)(s->n_q_heads / s->n_kv_heads) * s->block_len > 256) return FBK_ERR_UNSUPPORTED;
   if (s->batch > MAX_BATCH) return FBK_ERR_UNSUPPORTED;
   return FBK_OK;
 }
@@ -392,6 +396,31 @@ fbk_status fbk_fp8_group_quant(const void *x, int64_t rows, int64_t cols, void *
   return from_cuda(launch_fp8_group_quant(static_cast<const __nv_bfloat16 *>(x), rows * cols / FBK_FP8_GROUP,
                                           static_cast<uint8_t *>(codes), scales, sms,
                                           static_cast<cudaStream_t>(cuda_stream)));
+}
+
+fbk_status fbk_facache_unchanged_rows(const fbk_shape *shape, int32_t n_rows, const void *q_u,
+                                      const fbk_partial *state, const void *k_blk, const void *v_blk,
+                                      const int32_t *block_pos, void *out, float *lse, void *cuda_stream) {
+  fbk_status st = check_shape(shape, false);
+  if (st != FBK_OK) return st;
+  if (shape->mode != FBK_BF16) return FBK_ERR_UNSUPPORTED;
+  if (n_rows < 0) return FBK_ERR_INVALID_ARG;
+  if (n_rows == 0) return FBK_OK;  // no unchanged rows, nothing enqueued
+  if ((long long)shape->batch * n_rows * shape->n_q_heads > 0x7fffffffll) return FBK_ERR_CAPACITY;
+  if ((st = check_merge_ptrs(q_u, k_blk, v_blk, block_pos, state, out)) != FBK_OK) return st;
+  const int sms = default_shares();
+  if (sms < 1) return FBK_ERR_CUDA;
+  FacRowsArgs a;
+  a.q = static_cast<const __nv_bfloat16 *>(q_u);
+  a.state = *state;
+  a.kb = static_cast<const __nv_bfloat16 *>(k_blk);
+  a.vb = static_cast<const __nv_bfloat16 *>(v_blk);
+  a.block_pos = block_pos;
+  a.out = static_cast<__nv_bfloat16 *>(out);
+  a.lse = lse;
+  a.n_rows = n_rows;
+  a.ctas_per_unit = 1;
+  return from_cuda(launch_facache_rows(make_geometry(shape, nullptr), a, sms, static_cast<cudaStream_t>(cuda_stream)));
 }
 
 const char *fbk_status_string(fbk_status status) {

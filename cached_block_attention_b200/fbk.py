@@ -34,7 +34,7 @@ DEVERR_TIMEOUT = 8
 EXPORTS = ("fbk_prefix_workspace_bytes", "fbk_default_num_splits", "fbk_prefix_partial",
            "fbk_block_attn_merge", "fbk_commit_block_rope_append", "fbk_full_ref_attn",
            "fbk_status_string", "fbk_prefix_partial_static_scratch", "fbk_decode_block",
-           "fbk_fp8_group_quant")
+           "fbk_fp8_group_quant", "fbk_facache_unchanged_rows")
 
 STATIC_SCRATCH_BYTES = 32 << 20  # FBK_STATIC_SCRATCH_BYTES
 
@@ -87,6 +87,9 @@ _lib.fbk_decode_block.argtypes = [_P(_Shape), _P(_LayerBlock), ctypes.c_int32, c
 _lib.fbk_decode_block.restype = ctypes.c_int
 _lib.fbk_fp8_group_quant.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
 _lib.fbk_fp8_group_quant.restype = ctypes.c_int
+_lib.fbk_facache_unchanged_rows.argtypes = [_P(_Shape), ctypes.c_int32, _vp, _P(_Partial), _vp, _vp, _vp, _vp,
+                                            _vp, _vp]
+_lib.fbk_facache_unchanged_rows.restype = ctypes.c_int
 _lib.fbk_status_string.argtypes = [ctypes.c_int]
 _lib.fbk_status_string.restype = ctypes.c_char_p
 
@@ -274,6 +277,17 @@ def fp8_group_quant(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, 
     rows, cols = x.shape
     _check(_lib.fbk_fp8_group_quant(_ptr(x), rows, cols, _ptr(codes), _ptr(scales), _stream(stream)),
            "fbk_fp8_group_quant")
+
+
+def facache_unchanged_rows(shape: Shape, q_u: torch.Tensor, state: Partial, k_blk, v_blk, block_pos, out,
+                           lse=None, stream=None) -> None:
+    """FACache step of a sequence's unchanged rows: q_u [b, U, Hq, d] after RoPE,
+    state [b, Hq, U, d] / [b, Hq, U], block K/V [b, B, Hkv, d] (K before RoPE),
+    block_pos int32 [b] -> out [b, U, Hq, d], lse [b, Hq, U]."""
+    cs, ps = shape.c(), state.c()
+    _check(_lib.fbk_facache_unchanged_rows(ctypes.byref(cs), q_u.shape[1], _ptr(q_u), ctypes.byref(ps),
+                                           _ptr(k_blk), _ptr(v_blk), _ptr(block_pos), _ptr(out), _ptr(lse),
+                                           _stream(stream)), "fbk_facache_unchanged_rows")
 
 
 # raw handles for tests of the C ABI itself

@@ -297,6 +297,34 @@ fbk_status fbk_decode_block(const fbk_shape *shape, const fbk_layer_block *layer
 fbk_status fbk_fp8_group_quant(const void *x, int64_t rows, int64_t cols, void *codes, float *scales,
                                void *cuda_stream);
 
+/* FACache step for the unchanged rows of a whole sequence (LaCache §3.3.3
+ * FACache, Eq. 2-6, and App. J). The sequence's rows outside the current
+ * block (the set U: prompt, earlier blocks and the masked suffix, n_rows per
+ * sequence, in sequence order with the block removed) keep their
+ * online-softmax state over U's keys for the whole block. This call streams
+ * only the block's B keys for every row of U and every query head, merges
+ * with that state and normalises:
+ *   O = (e^(m1-m) O~1 + e^(m2-m) O~2) / (e^(m1-m) l1 + e^(m2-m) l2),
+ * (O~1, m1, l1) the cached state and (O~2, m2, l2) the row's state over the
+ * block's keys. The block's own rows are the other half of a step: they attend
+ * to U's keys and the block's.
+ *  q_u:   bf16 [b, n_rows, Hq, d], AFTER RoPE at the rows' own positions
+ *         (RoPECache); 16-byte aligned.
+ *  state: the cached state of U's rows over U's keys: o_unnorm fp32
+ *         [b, Hq, n_rows, d] (16-byte aligned), m and l fp32 [b, Hq, n_rows].
+ *  k_blk, v_blk: bf16 [b, B, Hkv, d], K before RoPE; 16-byte aligned.
+ *  block_pos: int32 [b] on the device: c0, the block's first position. The
+ *         block's keys are rotated at c0 + t. Any value is safe: it only
+ *         selects rotation angles.
+ *  out:   bf16 [b, n_rows, Hq, d]; lse: fp32 [b, Hq, n_rows] or NULL.
+ * FBK_BF16 mode only (FBK_ERR_UNSUPPORTED otherwise). The shape rules are
+ * those of fbk_shape except G*B <= 256, which does not apply here (B <= 64
+ * still does). n_rows = 0 enqueues nothing; b * n_rows * Hq must stay below
+ * 2^31 (FBK_ERR_CAPACITY). One launch. */
+fbk_status fbk_facache_unchanged_rows(const fbk_shape *shape, int32_t n_rows, const void *q_u,
+                                      const fbk_partial *state, const void *k_blk, const void *v_blk,
+                                      const int32_t *block_pos, void *out, float *lse, void *cuda_stream);
+
 /* Static text for a status code. */
 const char *fbk_status_string(fbk_status status);
 

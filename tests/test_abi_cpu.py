@@ -199,3 +199,31 @@ def test_fp8_group_quant_argument_checks(fbk):
     assert q(x, 4, 128, ctypes.c_void_p(0x20004), s, None) == -2   # codes not 8-byte aligned
     assert q(x, 4, 128, c, ctypes.c_void_p(0x30002), None) == -2   # scales not 4-byte aligned
     assert q(x, 1 << 33, 1 << 8, c, s, None) == -3          # more than 2^40 elements
+
+
+def test_facache_unchanged_rows_argument_checks(fbk):
+    """Host checks of fbk_facache_unchanged_rows; none of these reach a CUDA call."""
+    f = fbk.lib.fbk_facache_unchanged_rows
+    p = fbk.CPartial(0x40000, 0x50000, 0x60000)
+    ptr = ctypes.c_void_p
+    args = lambda **kw: dict(dict(q=ptr(0x70000), k=ptr(0x71000), v=ptr(0x72000), pos=ptr(0x30000),
+                                  out=ptr(0x90000)), **kw)
+
+    def call(shape=None, n=100, part=p, **kw):
+        a = args(**kw)
+        s = shape or _shape(fbk)
+        return f(ctypes.byref(s), n, a["q"], ctypes.byref(part) if part is not None else None, a["k"], a["v"],
+                 a["pos"], a["out"], None, None)
+    assert call(shape=_shape(fbk, mode=1)) == -2           # bf16 mode only
+    assert call(shape=_shape(fbk, head_dim=96)) == -2
+    assert call(n=-1) == -1
+    assert call(n=0, q=None, part=None) == 0               # no rows: nothing enqueued
+    assert call(q=None) == -1
+    assert call(pos=None) == -1
+    assert call(part=fbk.CPartial(0x40000, None, 0x60000)) == -1
+    assert call(q=ptr(0x70008)) == -2
+    assert call(part=fbk.CPartial(0x40008, 0x50000, 0x60000)) == -2
+    assert call(n=1 << 30, shape=_shape(fbk, batch=4)) == -3
+    # the block path's G*B <= 256 limit does not apply (its rows are U's), B <= 64 does
+    assert call(n=1 << 30, shape=_shape(fbk, n_q_heads=16, n_kv_heads=1, block_len=64)) == -3
+    assert call(shape=_shape(fbk, block_len=65)) == -2
