@@ -42,9 +42,10 @@ def parse():
     ap.add_argument("--workload", default="llada8b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="attention", choices=["attention", "fp8_group_quant"],
+    ap.add_argument("--op", default="attention", choices=["attention", "fp8_group_quant", "facache_rows"],
                     help="attention: the cached block attention block (default); fp8_group_quant: the "
-                         "per-group FP8 activation quantisation on the FP8_WORKLOADS shapes")
+                         "per-group FP8 activation quantisation on the FP8_WORKLOADS shapes; facache_rows: "
+                         "the FACache step of a whole sequence's unchanged rows (FACACHE_WORKLOADS)")
     ap.add_argument("--layers", type=int, default=1,
                     help="attention layers per block; > 1 runs the whole block through fbk_decode_block")
     ap.add_argument("--refresh-interval", default="",
@@ -998,6 +999,172 @@ def run_fp8(args, name, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ FACache over a whole sequence
+
+# (b, Hq, Hkv, d, B, unchanged rows, c0, seed): a LLaDA-8B-shaped layer over a
+# 4096-token prompt, the 32-token block and a 1024-token masked suffix
+FACACHE_WORKLOADS = {
+    "llada8b_seq": (1, 32, 32, 128, 32, 4096 + 1024, 4096, 31),
+}
+FACACHE_METRIC = "FACache step of a sequence's unchanged rows, algorithmic GB/s (1×B200)"
+
+
+def facache_bytes(b, hq, hkv, d, blk, rows):
+    """Algorithmic bytes of one step of the unchanged rows: each row and head
+    reads q (bf16) and its state (fp32 O~, m, l) and writes O (bf16); the
+    block's K and V are read once per kv-head."""
+    return b * rows * hq * (2 * d + 4 * (d + 2) + 2 * d) + 2 * b * blk * hkv * d * 2
+
+
+def facache_inputs(name):
+    """Seeded inputs (host): q_u bf16 bits, a synthetic state (fp32; m, l > 0),
+    block K/V bf16 bits."""
+    from cached_block_attention_b200 import synth
+    b, hq, hkv, d, blk, rows, c0, seed = FACACHE_WORKLOADS[name]
+    r = np.random.Generator(np.random.PCG64(seed))
+    sc = 1.0 / np.sqrt(d)
+    q = synth.bf16_bits(r.standard_normal((b, rows, hq, d), dtype=np.float32) * np.float32(sc))
+    m = r.uniform(-0.5, 0.5, (b, hq, rows)).astype(np.float32)
+    l = r.uniform(1.0, 6000.0, (b, hq, rows)).astype(np.float32)
+    o = (r.standard_normal((b, hq, rows, d), dtype=np.float32) * np.float32(0.05)) * l[..., None]
+    kb = synth.bf16_bits(r.standard_normal((b, blk, hkv, d), dtype=np.float32) * np.float32(sc))
+    vb = synth.bf16_bits(r.standard_normal((b, blk, hkv, d), dtype=np.float32) * np.float32(sc))
+    return q, (o, m, l), kb, vb
+
+
+def oracle_facache_sample(name, n_rows=256, budget_s=10.0):
+    """The oracle's step for the first n_rows unchanged rows, repeated for
+    about budget_s seconds: GB/s in the same algorithmic units."""
+    from oracle import facache as fc
+    from oracle import fbk_oracle as orc
+    b, hq, hkv, d, blk, rows, c0, seed = FACACHE_WORKLOADS[name]
+    q, (o, m, l), kb, vb = facache_inputs(name)
+    qs, st = orc.bits_to_f64(q[:, :n_rows]), (o[:, :, :n_rows], m[:, :, :n_rows], l[:, :, :n_rows])
+    kf, vf = orc.bits_to_f64(kb), orc.bits_to_f64(vb)
+
+    def one():
+        pos = c0 + np.arange(blk)
+        kr = orc.rope(kf, pos[None, :, None], 1e4)
+        return orc.finalize(orc.merge(st, fc._state(qs, kr, vf, hkv, 1.0)))
+    t0 = time.perf_counter()
+    one()
+    n = max(1, min(50, int(budget_s / max(time.perf_counter() - t0, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(n):
+        one()
+    dt = time.perf_counter() - t0
+    return n * facache_bytes(b, hq, hkv, d, blk, n_rows) / dt / 1e9, n, dt / n
+
+
+def run_facache_reference(args, name, rank):
+    if rank != 0:
+        return
+    v, n, per = oracle_facache_sample(name, budget_s=max(1.0, 0.5 * args.steps))
+    line = {"impl": "reference", "metric": FACACHE_METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": n, "warmup": args.warmup, "ms_per_step": 1e3 * per, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{n} runs of the step for 256 of the unchanged rows, numpy"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_facache(args, name, rank, world, local):
+    """One bench step = one fbk_facache_unchanged_rows launch over every
+    unchanged row, inputs resident in HBM, after an L2 flush."""
+    import torch
+    from cached_block_attention_b200 import fbk
+    dev = torch.device("cuda", local)
+    b, hq, hkv, d, blk, rows, c0, seed = FACACHE_WORKLOADS[name]
+    q, (o, m, l), kb, vb = facache_inputs(name)
+    to_bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    h_q = to_bf16(q).pin_memory()
+    d_q, d_k, d_v = h_q.to(dev), to_bf16(kb).to(dev), to_bf16(vb).to(dev)
+    state = fbk.Partial(torch.from_numpy(o).to(dev), torch.from_numpy(m).to(dev), torch.from_numpy(l).to(dev))
+    pos = torch.full((b,), c0, dtype=torch.int32, device=dev)
+    out = torch.empty(b, rows, hq, d, dtype=torch.bfloat16, device=dev)
+    h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    shape = fbk.Shape(b, hq, hkv, d, blk, 1.0, 1e4)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    st = torch.cuda.Stream(dev)
+    nbytes = facache_bytes(b, hq, hkv, d, blk, rows)
+
+    def timed(n):
+        evs = []
+        with torch.cuda.stream(st):
+            for _ in range(n):
+                flush.zero_()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e[0].record(st)
+                fbk.facache_unchanged_rows(shape, d_q, state, d_k, d_v, pos, out, stream=st)
+                e[1].record(st)
+                evs.append(e)
+        return evs
+
+    timed(max(3, args.warmup))
+    barrier(world)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    evs = timed(args.steps)
+    barrier(world)
+    clock_info = clocks.stop()
+    t = [e[0].elapsed_time(e[1]) for e in evs]
+    total_ms = max_over_ranks(sum(t), world)
+    launch_ms = sum(t) / len(t)
+
+    # end to end: the rows' queries H2D (the state stays resident across the
+    # block's steps), the launch, the outputs D2H
+    def e2e(n):
+        with torch.cuda.stream(st):
+            for _ in range(n):
+                d_q.copy_(h_q, non_blocking=True)
+                fbk.facache_unchanged_rows(shape, d_q, state, d_k, d_v, pos, out, stream=st)
+                h_out.copy_(out, non_blocking=True)
+    e2e(1)
+    torch.cuda.synchronize()
+    a, bev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, args.steps // 2)
+    a.record(st)
+    e2e(n_e2e)
+    bev.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(bev) / n_e2e, world)
+
+    hbm_gbs, _, _, peak_kind = load_peaks()
+    achieved = nbytes / (launch_ms * 1e-3) / 1e9
+    line = {
+        "metric": FACACHE_METRIC, "value": world * args.steps * nbytes / (total_ms * 1e-3) / 1e9, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": name, "batch": b, "q_heads": hq, "kv_heads": hkv, "head_dim": d, "block": blk,
+                   "unchanged_rows": rows, "block_pos": c0,
+                   "description": "LLaDA-8B-shaped layer, 4096-token prompt + 32-token block + 1024-token "
+                                  "masked suffix; synthetic cached state",
+                   "bench_step": "one fbk_facache_unchanged_rows launch",
+                   "l2": "flushed (2x L2 memset) before every timed launch, outside the events",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                     "frac": achieved / hbm_gbs, "peak_kind": f"{peak_kind} hbm_gbs", "traffic": None,
+                     "traffic_source": "no ncu capture of this kernel yet",
+                     "kernel": "fbk_facache_unchanged_rows", "algorithmic_bytes_per_launch": nbytes,
+                     "launch_us": launch_ms * 1e3},
+        "e2e": {"value": world * nbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h_q.numel() * 2, "d2h_bytes_per_step": h_out.numel() * 2,
+                "note": "the rows' queries H2D, the launch, the outputs D2H, one stream"},
+        "gpu_launches": args.steps,
+        "clocks": clock_info,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n, _ = oracle_facache_sample(name)
+        line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{n} runs of the step for 256 of the {rows} unchanged rows, numpy"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def layer_mode(args):
     return args.layers > 1 or bool(args.refresh_interval)
 
@@ -1009,6 +1176,19 @@ def intervals_of(args, wl):
 def main():
     args = parse()
     from cached_block_attention_b200 import synth
+    if args.op == "facache_rows":
+        name = args.workload if args.workload in FACACHE_WORKLOADS else "llada8b_seq"
+        if args.impl == "reference":
+            run_facache_reference(args, name, int(os.environ.get("RANK", "0")))
+            return
+        rank, world, local = dist_setup(args.gpus)
+        try:
+            run_facache(args, name, rank, world, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
     if args.op == "fp8_group_quant":
         name = args.workload if args.workload in FP8_WORKLOADS else "ffn_out_llada8b"
         if args.impl == "reference":
