@@ -278,7 +278,7 @@ def oracle_case(wl, n_step_inputs=2):
     kc, vc = synth.contiguous_cache(ks, vs, wl.n_kv_heads, wl.head_dim, int(lens.max()) + wl.block_len)
     steps = []
     vbits = None
-    for s in range(n_step_inputs):
+    for s in range(min(n_step_inputs, wl.steps)):
         q, k, v = synth.gen_step(wl, s)
         steps.append((orc.bits_to_f64(q), orc.bits_to_f64(k), orc.bits_to_f64(v)))
         vbits = v

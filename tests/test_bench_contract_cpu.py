@@ -1,0 +1,34 @@
+"""bench.py's JSON line on the host: every mode's reference arm (the oracle,
+timed on the host cores) runs and prints one line with the contract's keys.
+The GPU arms need a device and are exercised on a B200."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+KEYS = {"impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+        "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
+
+
+@pytest.mark.parametrize("extra", [
+    [],
+    ["--workload", "tiny"],
+    ["--layers", "4", "--refresh-interval", "2"],
+    ["--op", "fp8_group_quant", "--workload", "ffn_in_llada8b"],
+    ["--op", "facache_rows"],
+])
+def test_reference_arm_prints_one_contract_line(extra):
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"] + extra, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert KEYS <= set(d), KEYS - set(d)
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["unit"] == d["unit"]
+    assert "workload" in d["config"]
