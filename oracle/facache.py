@@ -23,7 +23,7 @@ Diffusion Large Language Models"):
   keys, and a row in C streams all keys. Every output equals full attention
   over the whole sequence (the method is exact).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * scores are ``tau * <q, k>`` (the pages write S = Q K^T, i.e. tau = 1);
   * RoPE is the rotate-half form with positions 0-based, as in
     ``fbk_oracle.rope``; the GQA head map is kv_head = floor(h * Hkv / Hq);

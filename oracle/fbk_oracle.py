@@ -23,7 +23,7 @@ decoding):
 * RoPE is applied to block Q and K at their absolute positions, while prefix K
   in the cache is stored already rotated (LaCache §3.3.2 RoPECache, Eq. 1).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * scores are ``tau * <RoPE(q), k>`` with tau an explicit argument (the pages
     write S = Q K^T, i.e. tau = 1);
   * RoPE is the rotate-half form: pairs (i, i + d/2), theta_i = base^(-2i/d),

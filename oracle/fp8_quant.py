@@ -18,7 +18,7 @@ and each element the code
 
 stored in the FP8 E4M3 format, so that x_i ~ x'_i * scale_g.
 
-Readings where the passage is silent (each also listed in the design doc):
+Readings taken where the passage is silent:
   * the low-precision format is E4M3 with Q_max = 448 = -Q_min (the FP8 format
     whose tensor-core GEMMs the passage uses for activations);
   * x is bf16 and the arithmetic is fp32: scale_g = fp32(amax / 448) and
