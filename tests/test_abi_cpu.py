@@ -227,3 +227,42 @@ def test_facache_unchanged_rows_argument_checks(fbk):
     # the block path's G*B <= 256 limit does not apply (its rows are U's), B <= 64 does
     assert call(n=1 << 30, shape=_shape(fbk, n_q_heads=16, n_kv_heads=1, block_len=64)) == -3
     assert call(shape=_shape(fbk, block_len=65)) == -2
+
+
+def test_plain_c_host_builds_and_calls_the_library(fbk, tmp_path):
+    """A C99 program includes include/fbk.h, links libfbk.so and calls entry
+    points that answer on the host (status strings, workspace sizes, argument
+    errors): the boundary needs no C++, Python or torch."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "host.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "fbk.h"
+int main(void) {
+  fbk_shape s = {1, 4, 2, 128, 32, 1.0f, 10000.0, FBK_BF16};
+  fbk_kv_cache c;
+  memset(&c, 0, sizeof c);
+  if (strcmp(fbk_status_string(FBK_ERR_WORKSPACE), "workspace missing or too small") != 0) return 1;
+  if (fbk_prefix_workspace_bytes(&s, &c, 10) == 0) return 2;
+  s.head_dim = 96;
+  if (fbk_prefix_workspace_bytes(&s, &c, 10) != 0) return 3;
+  if (fbk_prefix_partial(&s, NULL, &c, NULL, NULL, 0, 4, NULL) != FBK_ERR_UNSUPPORTED) return 4;
+  s.head_dim = 128;
+  if (fbk_prefix_partial(&s, NULL, &c, NULL, NULL, 0, 4, NULL) != FBK_ERR_INVALID_ARG) return 5;
+  if (fbk_fp8_group_quant(NULL, 4, 100, NULL, NULL, NULL) != FBK_ERR_INVALID_ARG) return 6;
+  puts("ok");
+  return 0;
+}
+''')
+    lib_dir = os.path.dirname(fbk.LIB_PATH)
+    exe = tmp_path / "host"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", f"-I{ROOT}/include",
+                        str(src), f"-L{lib_dir}", "-lfbk", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
