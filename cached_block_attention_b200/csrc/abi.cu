@@ -10,6 +10,7 @@
 
 #include "facache_rows.h"
 #include "launch.h"
+#include "prefix_at.h"
 
 namespace fbk {
 
@@ -24,7 +25,7 @@ bool is_pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
 
 // rows_limit: the block path keeps a kv-head's G*B query rows in at most two
 // 128-row tiles; entry points whose rows are not the block's skip that limit.
-fbk_status check_shape(const fbk_shape *s, bool rows_limit = true) {
+fbk_status check_shape(const fbk_shape *s, bool rows_limit = true, int max_block = 64) {
   if (!s) return FBK_ERR_INVALID_ARG;
   if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_heads < 1 || s->block_len < 1 || s->head_dim < 1)
     return FBK_ERR_INVALID_ARG;
@@ -34,7 +35,7 @@ fbk_status check_shape(const fbk_shape *s, bool rows_limit = true) {
     return FBK_ERR_INVALID_ARG;
   if (s->head_dim != 64 && s->head_dim != 128) return FBK_ERR_UNSUPPORTED;
   if (s->n_q_heads % s->n_kv_heads != 0) return FBK_ERR_UNSUPPORTED;
-  if (s->block_len > 64) return FBK_ERR_UNSUPPORTED;
+  if (s->block_len > max_block) return FBK_ERR_UNSUPPORTED;
   if (rows_limit && (long long)(s->n_q_heads / s->n_kv_heads) * s->block_len > 256) return FBK_ERR_UNSUPPORTED;
   if (s->batch > MAX_BATCH) return FBK_ERR_UNSUPPORTED;
   return FBK_OK;
@@ -180,12 +181,13 @@ fbk_status check_workspace(const fbk_shape *shape, int32_t num_splits, const voi
 }
 
 // The launches of one prefix computation: query rotation and share kernel (or
-// the fp32 share kernel), then the fixed-order split reduction.
+// the fp32 share kernel), then the fixed-order split reduction. qpos: NULL, or
+// the rotation base of the block's rows per sequence.
 cudaError_t enqueue_prefix(const fbk_shape *shape, const Geometry &g, const void *q_blk, const Workspace &w,
-                           int shares, const fbk_partial &out, cudaStream_t s) {
+                           int shares, const fbk_partial &out, cudaStream_t s, const int *qpos = nullptr) {
   const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_blk);
-  cudaError_t e = shape->mode == FBK_BF16 ? launch_prefix_tc(g, q, w, shares, s)
-                                          : launch_prefix_fp32(g, q, w, shares, s);
+  cudaError_t e = shape->mode == FBK_BF16 ? launch_prefix_tc_at(g, q, qpos, w, shares, s)
+                                          : launch_prefix_fp32_at(g, q, qpos, w, shares, s);
   if (e != cudaSuccess) return e;
   return launch_split_reduce(g, w, shares, out, s);
 }
@@ -246,7 +248,8 @@ int32_t fbk_default_num_splits(void) { return default_shares(); }
 
 size_t fbk_prefix_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache, int32_t num_splits) {
   (void)cache;
-  if (check_shape(shape) != FBK_OK || num_splits < 0) return 0;
+  // any shape a prefix computation accepts (fbk_prefix_partial_at allows B > 64)
+  if (check_shape(shape, true, 256) != FBK_OK || num_splits < 0) return 0;
   const int shares = num_splits ? num_splits : default_shares();
   if (shares < 1) return 0;
   return ws_layout(shape, shares).total;
@@ -302,6 +305,21 @@ fbk_status fbk_full_ref_attn(const fbk_shape *shape, const void *q_blk, const vo
                                    static_cast<const __nv_bfloat16 *>(k_blk),
                                    static_cast<const __nv_bfloat16 *>(v_blk), out, lse,
                                    shape->mode == FBK_FP32_CHECK, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+fbk_status fbk_prefix_partial_at(const fbk_shape *shape, const void *q_blk, const int32_t *q_pos,
+                                 const fbk_kv_cache *cache, const fbk_partial *out, void *ws, size_t ws_bytes,
+                                 int32_t num_splits, void *cuda_stream) {
+  fbk_status st = check_shape(shape, true, 256);  // G*B <= 256 rows per kv-head, B up to 256
+  if (st != FBK_OK) return st;
+  if ((st = check_cache(shape, cache)) != FBK_OK) return st;
+  if (num_splits < 0 || !q_pos) return FBK_ERR_INVALID_ARG;
+  if ((st = check_prefix_ptrs(q_blk, out)) != FBK_OK) return st;
+  int shares;
+  WsLayout lay;
+  if ((st = check_workspace(shape, num_splits, ws, ws_bytes, &shares, &lay)) != FBK_OK) return st;
+  return from_cuda(enqueue_prefix(shape, make_geometry(shape, cache), q_blk, carve(lay, ws), shares, *out,
+                                  static_cast<cudaStream_t>(cuda_stream), q_pos));
 }
 
 fbk_status fbk_prefix_partial_static_scratch(const fbk_shape *shape, const void *q_blk,

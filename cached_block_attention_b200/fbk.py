@@ -34,7 +34,7 @@ DEVERR_TIMEOUT = 8
 EXPORTS = ("fbk_prefix_workspace_bytes", "fbk_default_num_splits", "fbk_prefix_partial",
            "fbk_block_attn_merge", "fbk_commit_block_rope_append", "fbk_full_ref_attn",
            "fbk_status_string", "fbk_prefix_partial_static_scratch", "fbk_decode_block",
-           "fbk_fp8_group_quant", "fbk_facache_unchanged_rows")
+           "fbk_fp8_group_quant", "fbk_facache_unchanged_rows", "fbk_prefix_partial_at")
 
 STATIC_SCRATCH_BYTES = 32 << 20  # FBK_STATIC_SCRATCH_BYTES
 
@@ -90,6 +90,9 @@ _lib.fbk_fp8_group_quant.restype = ctypes.c_int
 _lib.fbk_facache_unchanged_rows.argtypes = [_P(_Shape), ctypes.c_int32, _vp, _P(_Partial), _vp, _vp, _vp, _vp,
                                             _vp, _vp]
 _lib.fbk_facache_unchanged_rows.restype = ctypes.c_int
+_lib.fbk_prefix_partial_at.argtypes = [_P(_Shape), _vp, _vp, _P(_Cache), _P(_Partial), _vp, ctypes.c_size_t,
+                                       ctypes.c_int32, _vp]
+_lib.fbk_prefix_partial_at.restype = ctypes.c_int
 _lib.fbk_status_string.argtypes = [ctypes.c_int]
 _lib.fbk_status_string.restype = ctypes.c_char_p
 
@@ -196,6 +199,15 @@ def prefix_partial(shape: Shape, q_blk: torch.Tensor, cache: KVCache, out: Parti
     _check(_lib.fbk_prefix_partial(ctypes.byref(cs), _ptr(q_blk), ctypes.byref(cc), ctypes.byref(po),
                                    _ptr(ws), ws.numel() * ws.element_size(), num_splits,
                                    _stream(stream)), "fbk_prefix_partial")
+
+
+def prefix_partial_at(shape: Shape, q_blk: torch.Tensor, q_pos: torch.Tensor, cache: KVCache, out: Partial,
+                      ws: torch.Tensor, num_splits: int = 0, stream=None) -> None:
+    """prefix_partial with the block's rows rotated at q_pos[b] + t (q_pos int32 [b] on the device)."""
+    cs, cc, po = shape.c(), cache.c(), out.c()
+    _check(_lib.fbk_prefix_partial_at(ctypes.byref(cs), _ptr(q_blk), _ptr(q_pos), ctypes.byref(cc), ctypes.byref(po),
+                                      _ptr(ws), ws.numel() * ws.element_size(), num_splits, _stream(stream)),
+           "fbk_prefix_partial_at")
 
 
 def prefix_partial_static_scratch(shape: Shape, q_blk: torch.Tensor, cache: KVCache, out: Partial,

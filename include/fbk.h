@@ -117,7 +117,7 @@ typedef struct fbk_partial {
  * fp32 for the per-share states plus b*Hkv * 128*ceil(G*B/128) * d bf16 for the
  * rotated query rows, each region rounded up to 256 bytes. Depends only on b,
  * Hkv, G*B, d and the share count, not on the prefix lengths. Returns 0 for an
- * invalid shape. */
+ * invalid shape; B up to 256 is valid here (fbk_prefix_partial_at's blocks). */
 size_t fbk_prefix_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache,
                                   int32_t num_splits);
 
@@ -182,6 +182,20 @@ fbk_status fbk_commit_block_rope_append(const fbk_shape *shape, const void *k_bl
 fbk_status fbk_full_ref_attn(const fbk_shape *shape, const void *q_blk, const void *k_blk,
                              const void *v_blk, const fbk_kv_cache *cache, void *out,
                              float *lse, void *cuda_stream);
+
+/* fbk_prefix_partial with the block's query rows rotated at q_pos[b] + t
+ * instead of prefix_lens[b] + t (q_pos: int32 [b] on the device, required).
+ * The cached keys are still rows 0 .. prefix_lens[b]-1 of the cache, stored
+ * after RoPE at whatever positions they hold. This lets the block's rows meet
+ * keys that lie after the block, such as a masked suffix in full-sequence
+ * decoding (LaCache §3.3.1: U holds the prompt and the masked suffix). It also
+ * lets any run of rows with consecutive positions stand in as the "block",
+ * for instance a chunk of U's rows when FACache's cached state of U over U's
+ * keys is computed (LaCache §3.3.3). The block length may exceed 64 here: B is
+ * limited only by G*B <= 256. Otherwise as fbk_prefix_partial. */
+fbk_status fbk_prefix_partial_at(const fbk_shape *shape, const void *q_blk, const int32_t *q_pos,
+                                 const fbk_kv_cache *cache, const fbk_partial *out, void *ws, size_t ws_bytes,
+                                 int32_t num_splits, void *cuda_stream);
 
 /* Size of the library's built-in scratch array (per device) used by
  * fbk_prefix_partial_static_scratch: 32 MiB. */

@@ -71,7 +71,8 @@ def test_shape_validation(fbk, kw, code):
                                       ctypes.c_void_p(0x70000), ctypes.c_void_p(0x30000), ctypes.byref(p),
                                       ctypes.c_void_p(0x90000), None, None)
     assert st == code
-    assert fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), ctypes.byref(c), 4) == 0
+    if kw != dict(block_len=65):  # B in (64, 256] with G*B <= 256 is a valid prefix shape (fbk_prefix_partial_at)
+        assert fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), ctypes.byref(c), 4) == 0
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -266,3 +267,16 @@ int main(void) {
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+def test_prefix_partial_at_argument_checks(fbk):
+    """fbk_prefix_partial_at: q_pos is required; blocks longer than 64 are accepted while G*B <= 256."""
+    c = _cache(fbk)
+    p = fbk.CPartial(0x40000, 0x50000, 0x60000)
+    f = fbk.lib.fbk_prefix_partial_at
+    q, pos, ws = ctypes.c_void_p(0x70000), ctypes.c_void_p(0x30000), ctypes.c_void_p(0x80000)
+    s = _shape(fbk, n_q_heads=2, n_kv_heads=2, block_len=256)           # G*B = 256
+    assert f(ctypes.byref(s), q, None, ctypes.byref(c), ctypes.byref(p), ws, 1 << 30, 4, None) == -1
+    assert f(ctypes.byref(s), q, pos, ctypes.byref(c), ctypes.byref(p), None, 0, 4, None) == -4
+    s2 = _shape(fbk, n_q_heads=4, n_kv_heads=2, block_len=129)          # G*B = 258
+    assert f(ctypes.byref(s2), q, pos, ctypes.byref(c), ctypes.byref(p), ws, 1 << 30, 4, None) == -2
+    assert fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), ctypes.byref(c), 4) > 0
