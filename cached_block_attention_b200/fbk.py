@@ -34,7 +34,8 @@ DEVERR_TIMEOUT = 8
 EXPORTS = ("fbk_prefix_workspace_bytes", "fbk_default_num_splits", "fbk_prefix_partial",
            "fbk_block_attn_merge", "fbk_commit_block_rope_append", "fbk_full_ref_attn",
            "fbk_status_string", "fbk_prefix_partial_static_scratch", "fbk_decode_block",
-           "fbk_fp8_group_quant", "fbk_facache_unchanged_rows", "fbk_prefix_partial_at")
+           "fbk_fp8_group_quant", "fbk_facache_unchanged_rows", "fbk_prefix_partial_at",
+           "fbk_facache_workspace_bytes", "fbk_facache_refresh", "fbk_facache_step")
 
 STATIC_SCRATCH_BYTES = 32 << 20  # FBK_STATIC_SCRATCH_BYTES
 
@@ -93,6 +94,14 @@ _lib.fbk_facache_unchanged_rows.restype = ctypes.c_int
 _lib.fbk_prefix_partial_at.argtypes = [_P(_Shape), _vp, _vp, _P(_Cache), _P(_Partial), _vp, ctypes.c_size_t,
                                        ctypes.c_int32, _vp]
 _lib.fbk_prefix_partial_at.restype = ctypes.c_int
+_lib.fbk_facache_workspace_bytes.argtypes = [_P(_Shape), ctypes.c_int32, ctypes.c_int32]
+_lib.fbk_facache_workspace_bytes.restype = ctypes.c_size_t
+_lib.fbk_facache_refresh.argtypes = [_P(_Shape), ctypes.c_int32, _vp, _P(ctypes.c_int32), _P(_Cache), _P(_Partial),
+                                     _vp, ctypes.c_size_t, ctypes.c_int32, _vp]
+_lib.fbk_facache_refresh.restype = ctypes.c_int
+_lib.fbk_facache_step.argtypes = [_P(_Shape), ctypes.c_int32, _vp, _P(_Partial), _vp, _vp, _vp, _vp, _P(_Cache), _vp,
+                                  _vp, _vp, _vp, _vp, ctypes.c_size_t, ctypes.c_int32, _vp]
+_lib.fbk_facache_step.restype = ctypes.c_int
 _lib.fbk_status_string.argtypes = [ctypes.c_int]
 _lib.fbk_status_string.restype = ctypes.c_char_p
 
@@ -300,6 +309,32 @@ def facache_unchanged_rows(shape: Shape, q_u: torch.Tensor, state: Partial, k_bl
     _check(_lib.fbk_facache_unchanged_rows(ctypes.byref(cs), q_u.shape[1], _ptr(q_u), ctypes.byref(ps),
                                            _ptr(k_blk), _ptr(v_blk), _ptr(block_pos), _ptr(out), _ptr(lse),
                                            _stream(stream)), "fbk_facache_unchanged_rows")
+
+
+def facache_workspace_bytes(shape: Shape, n_rows: int, num_splits: int = 0) -> int:
+    cs = shape.c()
+    return int(_lib.fbk_facache_workspace_bytes(ctypes.byref(cs), n_rows, num_splits))
+
+
+def facache_refresh(shape: Shape, q_u_raw: torch.Tensor, block_pos_host, u_cache: KVCache, state: Partial,
+                    ws: torch.Tensor, num_splits: int = 0, stream=None) -> None:
+    """FACache's state of U's rows over U's keys: q_u_raw [b, U, Hq, d] before RoPE,
+    block_pos_host a host sequence of c0 per sequence, state [b, Hq, U, d] / [b, Hq, U]."""
+    pos = (ctypes.c_int32 * shape.batch)(*[int(c) for c in block_pos_host])
+    cs, cc, ps = shape.c(), u_cache.c(), state.c()
+    _check(_lib.fbk_facache_refresh(ctypes.byref(cs), q_u_raw.shape[1], _ptr(q_u_raw), pos, ctypes.byref(cc),
+                                    ctypes.byref(ps), _ptr(ws), ws.numel() * ws.element_size(), num_splits,
+                                    _stream(stream)), "fbk_facache_refresh")
+
+
+def facache_step(shape: Shape, q_u_rot, state: Partial, q_blk, k_blk, v_blk, block_pos, u_cache: KVCache, out_u,
+                 out_blk, ws: torch.Tensor, lse_u=None, lse_blk=None, num_splits: int = 0, stream=None) -> None:
+    """One denoising step of FACache over a whole sequence: U's rows and the block's rows."""
+    cs, cc, ps = shape.c(), u_cache.c(), state.c()
+    _check(_lib.fbk_facache_step(ctypes.byref(cs), q_u_rot.shape[1], _ptr(q_u_rot), ctypes.byref(ps), _ptr(q_blk),
+                                 _ptr(k_blk), _ptr(v_blk), _ptr(block_pos), ctypes.byref(cc), _ptr(out_u),
+                                 _ptr(lse_u), _ptr(out_blk), _ptr(lse_blk), _ptr(ws), ws.numel() * ws.element_size(),
+                                 num_splits, _stream(stream)), "fbk_facache_step")
 
 
 # raw handles for tests of the C ABI itself

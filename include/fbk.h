@@ -339,6 +339,48 @@ fbk_status fbk_facache_unchanged_rows(const fbk_shape *shape, int32_t n_rows, co
                                       const fbk_partial *state, const void *k_blk, const void *v_blk,
                                       const int32_t *block_pos, void *out, float *lse, void *cuda_stream);
 
+/* FACache over a whole sequence as two calls (LaCache §3.3.1-§3.3.3, App. J).
+ * The sequence's rows outside the current block (U: prompt, earlier blocks,
+ * masked suffix; n_rows per sequence, in sequence order with the block
+ * removed) keep their state over U's keys for the whole block:
+ * fbk_facache_refresh computes it once per block, and fbk_facache_step uses it
+ * at every denoising step. A step's outputs equal attention over the whole
+ * sequence. Both calls use a workspace of fbk_facache_workspace_bytes(shape,
+ * n_rows, num_splits) bytes (256-byte aligned, contents irrelevant on entry).
+ * The shape rules are those of the block path (B <= 64, G*B <= 256).
+ *
+ * u_cache: U's K (after RoPE, at the rows' own positions) and V, contiguous
+ *   [b, Hkv, capacity >= n_rows, d], with prefix_lens[b] = n_rows on the device.
+ *
+ * fbk_facache_refresh:
+ *  q_u_raw: bf16 [b, n_rows, Hq, d], U's queries BEFORE RoPE.
+ *  block_pos_host: int32 [b] on the HOST: c0, 0 <= c0 <= n_rows. Row i of U
+ *           sits at position i (i < c0) or i + B.
+ *  state:   the output, o_unnorm fp32 [b, Hq, n_rows, d] (16-byte aligned),
+ *           m and l fp32 [b, Hq, n_rows].
+ *  The rows are processed in chunks of up to 256/G rows that do not cross the
+ *  block, one prefix computation each, whose states are copied into place.
+ *
+ * fbk_facache_step (FBK_BF16 only):
+ *  q_u_rot: bf16 [b, n_rows, Hq, d], U's queries AFTER RoPE (RoPECache).
+ *  state:   from fbk_facache_refresh.
+ *  q_blk, k_blk, v_blk: the block, bf16 [b, B, Hq|Hkv, d], Q and K before RoPE.
+ *  block_pos: int32 [b] on the device: c0.
+ *  out_u: bf16 [b, n_rows, Hq, d]; lse_u fp32 [b, Hq, n_rows] or NULL.
+ *  out_blk: bf16 [b, B, Hq, d]; lse_blk fp32 [b, Hq, B] or NULL.
+ *  Launches: fbk_facache_unchanged_rows's kernel for U's rows; for the block's
+ *  rows, the prefix computation over U's keys with the rows rotated at c0 + t,
+ *  then fbk_block_attn_merge's kernel. */
+size_t fbk_facache_workspace_bytes(const fbk_shape *shape, int32_t n_rows, int32_t num_splits);
+fbk_status fbk_facache_refresh(const fbk_shape *shape, int32_t n_rows, const void *q_u_raw,
+                               const int32_t *block_pos_host, const fbk_kv_cache *u_cache,
+                               const fbk_partial *state, void *ws, size_t ws_bytes, int32_t num_splits,
+                               void *cuda_stream);
+fbk_status fbk_facache_step(const fbk_shape *shape, int32_t n_rows, const void *q_u_rot, const fbk_partial *state,
+                            const void *q_blk, const void *k_blk, const void *v_blk, const int32_t *block_pos,
+                            const fbk_kv_cache *u_cache, void *out_u, float *lse_u, void *out_blk, float *lse_blk,
+                            void *ws, size_t ws_bytes, int32_t num_splits, void *cuda_stream);
+
 /* Static text for a status code. */
 const char *fbk_status_string(fbk_status status);
 

@@ -153,3 +153,37 @@ def test_full_step_equals_full_sequence_attention(cfg):
                                             f(seq["v"][bi:bi + 1]), hkv, tau)
         H.assert_close(H.host_f64(out_u[bi:bi + 1]), ref[:, seq["up"][bi]], "bf16", f"U rows, sequence {bi}")
         H.assert_close(H.host_f64(out_c[bi:bi + 1]), ref[:, seq["cp"][bi]], "bf16", f"block rows, sequence {bi}")
+
+
+@pytest.mark.parametrize("cfg", CASES)
+def test_refresh_and_step_entry_points(cfg):
+    """The same step through fbk_facache_refresh and fbk_facache_step: the state
+    equals the chunk-by-chunk composition's, and both halves of the output equal
+    full-sequence attention."""
+    from cached_block_attention_b200 import fbk
+    b, hq, hkv, d, blk, n, c0s, base, tau = cfg
+    seq = make_sequence(b, hq, hkv, d, blk, n, c0s, base, seed=200 + CASES.index(cfg))
+    nu = n - blk
+    shape = fbk.Shape(b, hq, hkv, d, blk, tau, base)
+    cache = u_cache(seq, hkv, d)
+    ws = torch.empty(fbk.facache_workspace_bytes(shape, nu, 0), dtype=torch.uint8, device="cuda")
+    st = fbk.Partial(torch.empty(b, hq, nu, d, device="cuda"), torch.empty(b, hq, nu, device="cuda"),
+                     torch.empty(b, hq, nu, device="cuda"))
+    fbk.facache_refresh(shape, H.dev_bf16(seq["qu_raw"]), list(c0s), cache, st, ws)
+    ref_st = state_by_chunks(seq, hq, hkv, d, blk, list(c0s), tau, base)
+    for x, y in ((st.o_unnorm, ref_st.o_unnorm), (st.m, ref_st.m), (st.l, ref_st.l)):
+        assert torch.equal(x, y)
+    pos = torch.tensor(list(c0s), dtype=torch.int32, device="cuda")
+    out_u = torch.empty(b, nu, hq, d, dtype=torch.bfloat16, device="cuda")
+    out_c = torch.empty(b, blk, hq, d, dtype=torch.bfloat16, device="cuda")
+    fbk.facache_step(shape, H.dev_bf16(seq["qu_rot"]), st, H.dev_bf16(seq["qc"]), H.dev_bf16(seq["kc"]),
+                     H.dev_bf16(seq["vc"]), pos, cache, out_u, out_c, ws)
+    torch.cuda.synchronize()
+    f = orc.bits_to_f64
+    for bi in range(b):
+        pos_all = np.arange(n)[None, :, None]
+        ref, _ = fc.full_sequence_attention(orc.rope(f(seq["q"][bi:bi + 1]), pos_all, base),
+                                            orc.rope(f(seq["k"][bi:bi + 1]), pos_all, base),
+                                            f(seq["v"][bi:bi + 1]), hkv, tau)
+        H.assert_close(H.host_f64(out_u[bi:bi + 1]), ref[:, seq["up"][bi]], "bf16", f"U rows, sequence {bi}")
+        H.assert_close(H.host_f64(out_c[bi:bi + 1]), ref[:, seq["cp"][bi]], "bf16", f"block rows, sequence {bi}")
