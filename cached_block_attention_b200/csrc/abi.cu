@@ -12,6 +12,7 @@
 #include "facache_rows.h"
 #include "launch.h"
 #include "prefix_at.h"
+#include "sparse_prefix.h"
 
 namespace fbk {
 
@@ -587,6 +588,72 @@ fbk_status fbk_facache_step(const fbk_shape *shape, int32_t n_rows, const void *
     return FBK_ERR_CUDA;
   return from_cuda(enqueue_merge(shape, merge_geometry(shape, block_pos), q_blk, k_blk, v_blk, part, out_blk,
                                  lse_blk, s));
+}
+
+fbk_status fbk_page_means(const fbk_shape *shape, const fbk_kv_cache *cache, float *means, void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if ((st = check_cache(shape, cache)) != FBK_OK) return st;
+  if (!cache->paged) return FBK_ERR_UNSUPPORTED;
+  if (!means) return FBK_ERR_INVALID_ARG;
+  return from_cuda(launch_page_means(make_geometry(shape, cache), means, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+size_t fbk_select_pages_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache) {
+  if (check_shape(shape) != FBK_OK || !cache || !cache->paged || cache->max_pages_per_seq < 1) return 0;
+  const size_t qrot = (size_t)shape->batch * shape->block_len * shape->n_q_heads * shape->head_dim * 4;
+  return align256(qrot) + align256((size_t)shape->batch * cache->max_pages_per_seq * 4);
+}
+
+fbk_status fbk_select_pages(const fbk_shape *shape, const void *q_blk, const fbk_kv_cache *cache, const float *means,
+                            int32_t k, int32_t *kept_table, int32_t *kept_lens, void *ws, size_t ws_bytes,
+                            void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if ((st = check_cache(shape, cache)) != FBK_OK) return st;
+  if (!cache->paged) return FBK_ERR_UNSUPPORTED;
+  if (!q_blk || !means || !kept_table || !kept_lens || k < 1) return FBK_ERR_INVALID_ARG;
+  if ((size_t)cache->max_pages_per_seq * 8 > 200 * 1024) return FBK_ERR_UNSUPPORTED;  // scores + flags in smem
+  const size_t need = fbk_select_pages_workspace_bytes(shape, cache);
+  if (!ws || ws_bytes < need) return FBK_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return FBK_ERR_UNSUPPORTED;
+  const int sms = default_shares();
+  if (sms < 1) return FBK_ERR_CUDA;
+  float *qrot = static_cast<float *>(ws);
+  float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) +
+                                            align256((size_t)shape->batch * shape->block_len * shape->n_q_heads *
+                                                     shape->head_dim * 4));
+  return from_cuda(launch_select_pages(make_geometry(shape, cache), static_cast<const __nv_bfloat16 *>(q_blk), means,
+                                       k, qrot, scores, kept_table, kept_lens, sms,
+                                       static_cast<cudaStream_t>(cuda_stream)));
+}
+
+fbk_status fbk_residual_capture(const fbk_shape *shape, const fbk_partial *dense, const fbk_partial *sparse,
+                                float *r_o, float *r_lse, void *cuda_stream) {
+  fbk_status st = check_shape(shape, true, 256);
+  if (st != FBK_OK) return st;
+  if (!dense || !sparse || !dense->o_unnorm || !dense->m || !dense->l || !sparse->o_unnorm || !sparse->m ||
+      !sparse->l || !r_o || !r_lse)
+    return FBK_ERR_INVALID_ARG;
+  const int sms = default_shares();
+  if (sms < 1) return FBK_ERR_CUDA;
+  const int rows = shape->batch * shape->n_q_heads * shape->block_len;
+  return from_cuda(launch_residual_capture(rows, shape->head_dim, *dense, *sparse, r_o, r_lse, sms,
+                                           static_cast<cudaStream_t>(cuda_stream)));
+}
+
+fbk_status fbk_residual_apply(const fbk_shape *shape, const fbk_partial *sparse, const float *r_o,
+                              const float *r_lse, const fbk_partial *ext, void *cuda_stream) {
+  fbk_status st = check_shape(shape, true, 256);
+  if (st != FBK_OK) return st;
+  if (!sparse || !ext || !sparse->o_unnorm || !sparse->m || !sparse->l || !ext->o_unnorm || !ext->m || !ext->l ||
+      !r_o || !r_lse)
+    return FBK_ERR_INVALID_ARG;
+  const int sms = default_shares();
+  if (sms < 1) return FBK_ERR_CUDA;
+  const int rows = shape->batch * shape->n_q_heads * shape->block_len;
+  return from_cuda(launch_residual_apply(rows, shape->head_dim, *sparse, r_o, r_lse, *ext, sms,
+                                         static_cast<cudaStream_t>(cuda_stream)));
 }
 
 const char *fbk_status_string(fbk_status status) {

@@ -381,6 +381,37 @@ fbk_status fbk_facache_step(const fbk_shape *shape, int32_t n_rows, const void *
                             const fbk_kv_cache *u_cache, void *out_u, float *lse_u, void *out_blk, float *lse_blk,
                             void *ws, size_t ws_bytes, int32_t num_splits, void *cuda_stream);
 
+/* Sparse block-external attention with a cached residual (FlashBlock,
+ * Abstract: cached block-external attention combined with sparse attention as
+ * residual reuse). Reading: pages of the prefix (the paged cache's pages) are
+ * scored by the largest tau <RoPE(q_t, L_b + t), kbar> over the block's rows
+ * and query heads, kbar the page's mean key; the top k pages per sequence form
+ * a page table of their own for fbk_prefix_partial_at (queries rotated at the
+ * true L_b + t); at a dense step the residual (O~/l, lse) dense minus sparse
+ * is captured; at later steps the sparse state plus the residual becomes the
+ * state fbk_block_attn_merge merges. Paged caches only.
+ *
+ * fbk_page_means: means fp32 [b, max_pages_per_seq, Hkv, d], the mean key of
+ *   every logical page of the prefix (pages past prefix_lens untouched).
+ * fbk_select_pages: q_blk bf16 [b, B, Hq, d] before RoPE; k >= 1 pages kept;
+ *   kept_table int32 [b, k] (physical page ids in increasing logical order,
+ *   -1 past the kept count) and kept_lens int32 [b] (their token count, the
+ *   partial last page included), both on the device; workspace of
+ *   fbk_select_pages_workspace_bytes bytes, 256-byte aligned.
+ * fbk_residual_capture: r_o fp32 [b, Hq, B, d] and r_lse fp32 [b, Hq, B] from
+ *   the dense and the sparse state of the same queries (r_lse = -inf marks a
+ *   row with no prefix).
+ * fbk_residual_apply: ext = ((O~/l)_sparse + r_o, lse_sparse + r_lse, 1). */
+fbk_status fbk_page_means(const fbk_shape *shape, const fbk_kv_cache *cache, float *means, void *cuda_stream);
+size_t fbk_select_pages_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache);
+fbk_status fbk_select_pages(const fbk_shape *shape, const void *q_blk, const fbk_kv_cache *cache, const float *means,
+                            int32_t k, int32_t *kept_table, int32_t *kept_lens, void *ws, size_t ws_bytes,
+                            void *cuda_stream);
+fbk_status fbk_residual_capture(const fbk_shape *shape, const fbk_partial *dense, const fbk_partial *sparse,
+                                float *r_o, float *r_lse, void *cuda_stream);
+fbk_status fbk_residual_apply(const fbk_shape *shape, const fbk_partial *sparse, const float *r_o,
+                              const float *r_lse, const fbk_partial *ext, void *cuda_stream);
+
 /* Static text for a status code. */
 const char *fbk_status_string(fbk_status status);
 
