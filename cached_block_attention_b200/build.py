@@ -23,7 +23,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfbk.so")
 
 SOURCES = ["abi.cu", "prefix_tc.cu", "prefix_fp32.cu", "split_reduce.cu", "block_merge.cu",
-           "commit.cu", "full_ref.cu", "fp8_quant.cu", "facache_rows.cu"]
+           "commit.cu", "full_ref.cu", "fp8_quant.cu", "facache_rows.cu", "sparse_prefix.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

@@ -4,12 +4,15 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
 #include <initializer_list>
 #include <mutex>
 #include <vector>
 
 #include "facache_rows.h"
 #include "launch.h"
+#include "prefix_at.h"
+#include "sparse_prefix.h"
 
 namespace fbk {
 
@@ -24,7 +27,7 @@ bool is_pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
 
 // rows_limit: the block path keeps a kv-head's G*B query rows in at most two
 // 128-row tiles; entry points whose rows are not the block's skip that limit.
-fbk_status check_shape(const fbk_shape *s, bool rows_limit = true) {
+fbk_status check_shape(const fbk_shape *s, bool rows_limit = true, int max_block = 64) {
   if (!s) return FBK_ERR_INVALID_ARG;
   if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_heads < 1 || s->block_len < 1 || s->head_dim < 1)
     return FBK_ERR_INVALID_ARG;
@@ -34,7 +37,7 @@ fbk_status check_shape(const fbk_shape *s, bool rows_limit = true) {
     return FBK_ERR_INVALID_ARG;
   if (s->head_dim != 64 && s->head_dim != 128) return FBK_ERR_UNSUPPORTED;
   if (s->n_q_heads % s->n_kv_heads != 0) return FBK_ERR_UNSUPPORTED;
-  if (s->block_len > 64) return FBK_ERR_UNSUPPORTED;
+  if (s->block_len > max_block) return FBK_ERR_UNSUPPORTED;
   if (rows_limit && (long long)(s->n_q_heads / s->n_kv_heads) * s->block_len > 256) return FBK_ERR_UNSUPPORTED;
   if (s->batch > MAX_BATCH) return FBK_ERR_UNSUPPORTED;
   return FBK_OK;
@@ -138,6 +141,44 @@ Workspace carve(const WsLayout &l, void *base) {
 
 fbk_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FBK_OK : FBK_ERR_CUDA; }
 
+// Workspace of FACache over a whole sequence: a prefix workspace big enough
+// for a chunk of U's rows (b = 1, cmax rows per query head) and for the
+// block's rows (the step), one state buffer for either, and the chunks'
+// rotation bases.
+struct FacSeqLayout {
+  int cmax;
+  long long nchunks;  // per sequence
+  size_t part_o, part_m, part_l, pos, total;
+};
+
+FacSeqLayout fac_layout(const fbk_shape *s, int n_rows, int shares) {
+  FacSeqLayout L;
+  const int G = s->n_q_heads / s->n_kv_heads;
+  L.cmax = 256 / G;
+  fbk_shape chunk = *s;
+  chunk.batch = 1;
+  chunk.block_len = L.cmax;
+  const size_t pfx = std::max(ws_layout(&chunk, shares).total, ws_layout(s, shares).total);
+  const size_t rows = std::max((size_t)s->n_q_heads * L.cmax, (size_t)s->batch * s->n_q_heads * s->block_len);
+  size_t off = align256(pfx);
+  L.part_o = off;
+  off = align256(off + rows * s->head_dim * sizeof(float));
+  L.part_m = off;
+  off = align256(off + rows * sizeof(float));
+  L.part_l = off;
+  off = align256(off + rows * sizeof(float));
+  L.nchunks = ((long long)n_rows + L.cmax - 1) / L.cmax + 1;  // the block may cut one chunk in two
+  L.pos = off;
+  L.total = align256(off + (size_t)L.nchunks * sizeof(int));
+  return L;
+}
+
+fbk_partial fac_part(const FacSeqLayout &L, void *ws) {
+  char *p = static_cast<char *>(ws);
+  return fbk_partial{reinterpret_cast<float *>(p + L.part_o), reinterpret_cast<float *>(p + L.part_m),
+                     reinterpret_cast<float *>(p + L.part_l)};
+}
+
 bool misaligned16(std::initializer_list<const void *> ptrs) {
   uintptr_t bits = 0;
   for (const void *p : ptrs) bits |= reinterpret_cast<uintptr_t>(p);
@@ -180,12 +221,13 @@ fbk_status check_workspace(const fbk_shape *shape, int32_t num_splits, const voi
 }
 
 // The launches of one prefix computation: query rotation and share kernel (or
-// the fp32 share kernel), then the fixed-order split reduction.
+// the fp32 share kernel), then the fixed-order split reduction. qpos: NULL, or
+// the rotation base of the block's rows per sequence.
 cudaError_t enqueue_prefix(const fbk_shape *shape, const Geometry &g, const void *q_blk, const Workspace &w,
-                           int shares, const fbk_partial &out, cudaStream_t s) {
+                           int shares, const fbk_partial &out, cudaStream_t s, const int *qpos = nullptr) {
   const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_blk);
-  cudaError_t e = shape->mode == FBK_BF16 ? launch_prefix_tc(g, q, w, shares, s)
-                                          : launch_prefix_fp32(g, q, w, shares, s);
+  cudaError_t e = shape->mode == FBK_BF16 ? launch_prefix_tc_at(g, q, qpos, w, shares, s)
+                                          : launch_prefix_fp32_at(g, q, qpos, w, shares, s);
   if (e != cudaSuccess) return e;
   return launch_split_reduce(g, w, shares, out, s);
 }
@@ -246,7 +288,8 @@ int32_t fbk_default_num_splits(void) { return default_shares(); }
 
 size_t fbk_prefix_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache, int32_t num_splits) {
   (void)cache;
-  if (check_shape(shape) != FBK_OK || num_splits < 0) return 0;
+  // any shape a prefix computation accepts (fbk_prefix_partial_at allows B > 64)
+  if (check_shape(shape, true, 256) != FBK_OK || num_splits < 0) return 0;
   const int shares = num_splits ? num_splits : default_shares();
   if (shares < 1) return 0;
   return ws_layout(shape, shares).total;
@@ -302,6 +345,21 @@ fbk_status fbk_full_ref_attn(const fbk_shape *shape, const void *q_blk, const vo
                                    static_cast<const __nv_bfloat16 *>(k_blk),
                                    static_cast<const __nv_bfloat16 *>(v_blk), out, lse,
                                    shape->mode == FBK_FP32_CHECK, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+fbk_status fbk_prefix_partial_at(const fbk_shape *shape, const void *q_blk, const int32_t *q_pos,
+                                 const fbk_kv_cache *cache, const fbk_partial *out, void *ws, size_t ws_bytes,
+                                 int32_t num_splits, void *cuda_stream) {
+  fbk_status st = check_shape(shape, true, 256);  // G*B <= 256 rows per kv-head, B up to 256
+  if (st != FBK_OK) return st;
+  if ((st = check_cache(shape, cache)) != FBK_OK) return st;
+  if (num_splits < 0 || !q_pos) return FBK_ERR_INVALID_ARG;
+  if ((st = check_prefix_ptrs(q_blk, out)) != FBK_OK) return st;
+  int shares;
+  WsLayout lay;
+  if ((st = check_workspace(shape, num_splits, ws, ws_bytes, &shares, &lay)) != FBK_OK) return st;
+  return from_cuda(enqueue_prefix(shape, make_geometry(shape, cache), q_blk, carve(lay, ws), shares, *out,
+                                  static_cast<cudaStream_t>(cuda_stream), q_pos));
 }
 
 fbk_status fbk_prefix_partial_static_scratch(const fbk_shape *shape, const void *q_blk,
@@ -421,6 +479,181 @@ fbk_status fbk_facache_unchanged_rows(const fbk_shape *shape, int32_t n_rows, co
   a.n_rows = n_rows;
   a.ctas_per_unit = 1;
   return from_cuda(launch_facache_rows(make_geometry(shape, nullptr), a, sms, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+size_t fbk_facache_workspace_bytes(const fbk_shape *shape, int32_t n_rows, int32_t num_splits) {
+  if (check_shape(shape) != FBK_OK || n_rows < 0 || num_splits < 0) return 0;
+  const int shares = num_splits ? num_splits : default_shares();
+  if (shares < 1) return 0;
+  return fac_layout(shape, n_rows, shares).total;
+}
+
+fbk_status fbk_facache_refresh(const fbk_shape *shape, int32_t n_rows, const void *q_u_raw,
+                               const int32_t *block_pos_host, const fbk_kv_cache *u_cache,
+                               const fbk_partial *state, void *ws, size_t ws_bytes, int32_t num_splits,
+                               void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if ((st = check_cache(shape, u_cache)) != FBK_OK) return st;
+  if (u_cache->paged) return FBK_ERR_UNSUPPORTED;
+  if (n_rows < 0 || num_splits < 0 || !block_pos_host) return FBK_ERR_INVALID_ARG;
+  if (n_rows == 0) return FBK_OK;
+  if (u_cache->capacity_tokens < n_rows) return FBK_ERR_CAPACITY;
+  if ((st = check_prefix_ptrs(q_u_raw, state)) != FBK_OK) return st;
+  for (int32_t bi = 0; bi < shape->batch; ++bi)
+    if (block_pos_host[bi] < 0 || block_pos_host[bi] > n_rows) return FBK_ERR_INVALID_ARG;
+  const int shares = num_splits ? num_splits : default_shares();
+  if (shares < 1) return FBK_ERR_CUDA;
+  const FacSeqLayout L = fac_layout(shape, n_rows, shares);
+  if (!ws || ws_bytes < L.total) return FBK_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return FBK_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const fbk_partial part = fac_part(L, ws);
+  int *pos = reinterpret_cast<int *>(static_cast<char *>(ws) + L.pos);
+  const size_t hq = shape->n_q_heads, d = shape->head_dim, U = n_rows;
+  for (int32_t bi = 0; bi < shape->batch; ++bi) {
+    const int c0 = block_pos_host[bi];
+    const int n_before = (c0 + L.cmax - 1) / L.cmax, n_after = (n_rows - c0 + L.cmax - 1) / L.cmax;
+    if (launch_chunk_positions(pos, n_before, n_after, c0, L.cmax, shape->block_len, s) != cudaSuccess)
+      return FBK_ERR_CUDA;
+    fbk_kv_cache one = *u_cache;  // this sequence's keys
+    const size_t seq_elems = (size_t)shape->n_kv_heads * u_cache->capacity_tokens * d;
+    one.k = static_cast<char *>(u_cache->k) + bi * seq_elems * 2;
+    one.v = static_cast<char *>(u_cache->v) + bi * seq_elems * 2;
+    one.prefix_lens = u_cache->prefix_lens + bi;
+    int k = 0;
+    const int bounds[3] = {0, c0, n_rows};
+    for (int side = 0; side < 2; ++side) {
+      for (int i0 = bounds[side]; i0 < bounds[side + 1]; i0 += L.cmax, ++k) {
+        fbk_shape cs = *shape;
+        cs.batch = 1;
+        cs.block_len = std::min(L.cmax, bounds[side + 1] - i0);
+        const Geometry g = make_geometry(&cs, &one);
+        const Workspace w = carve(ws_layout(&cs, shares), ws);
+        const void *q = static_cast<const char *>(q_u_raw) + ((size_t)bi * U + i0) * hq * d * 2;
+        if (enqueue_prefix(&cs, g, q, w, shares, part, s, pos + k) != cudaSuccess) return FBK_ERR_CUDA;
+        // the chunk's rows into the state: [Hq, rows, d] -> [b, Hq, U, d] at row i0
+        const size_t rows = cs.block_len;
+        float *o_dst = state->o_unnorm + ((size_t)bi * hq * U + i0) * d;
+        if (cudaMemcpy2DAsync(o_dst, U * d * 4, part.o_unnorm, rows * d * 4, rows * d * 4, hq,
+                              cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+            cudaMemcpy2DAsync(state->m + (size_t)bi * hq * U + i0, U * 4, part.m, rows * 4, rows * 4, hq,
+                              cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+            cudaMemcpy2DAsync(state->l + (size_t)bi * hq * U + i0, U * 4, part.l, rows * 4, rows * 4, hq,
+                              cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+          return FBK_ERR_CUDA;
+      }
+    }
+  }
+  return FBK_OK;
+}
+
+fbk_status fbk_facache_step(const fbk_shape *shape, int32_t n_rows, const void *q_u_rot, const fbk_partial *state,
+                            const void *q_blk, const void *k_blk, const void *v_blk, const int32_t *block_pos,
+                            const fbk_kv_cache *u_cache, void *out_u, float *lse_u, void *out_blk, float *lse_blk,
+                            void *ws, size_t ws_bytes, int32_t num_splits, void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if (shape->mode != FBK_BF16) return FBK_ERR_UNSUPPORTED;
+  if ((st = check_cache(shape, u_cache)) != FBK_OK) return st;
+  if (n_rows < 0 || num_splits < 0) return FBK_ERR_INVALID_ARG;
+  if ((long long)shape->batch * n_rows * shape->n_q_heads > 0x7fffffffll) return FBK_ERR_CAPACITY;
+  if ((st = check_merge_ptrs(q_blk, k_blk, v_blk, block_pos, state, out_blk)) != FBK_OK) return st;
+  if (n_rows > 0 && (st = check_merge_ptrs(q_u_rot, k_blk, v_blk, block_pos, state, out_u)) != FBK_OK) return st;
+  const int shares = num_splits ? num_splits : default_shares();
+  if (shares < 1) return FBK_ERR_CUDA;
+  const FacSeqLayout L = fac_layout(shape, n_rows, shares);
+  if (!ws || ws_bytes < L.total) return FBK_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return FBK_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  if (n_rows > 0) {  // U's rows: their cached state merged with the block's keys
+    FacRowsArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(q_u_rot);
+    a.state = *state;
+    a.kb = static_cast<const __nv_bfloat16 *>(k_blk);
+    a.vb = static_cast<const __nv_bfloat16 *>(v_blk);
+    a.block_pos = block_pos;
+    a.out = static_cast<__nv_bfloat16 *>(out_u);
+    a.lse = lse_u;
+    a.n_rows = n_rows;
+    a.ctas_per_unit = 1;
+    const int sms = default_shares();
+    if (sms < 1) return FBK_ERR_CUDA;
+    if (launch_facache_rows(make_geometry(shape, nullptr), a, sms, s) != cudaSuccess) return FBK_ERR_CUDA;
+  }
+  // the block's rows: their state over U's keys (rotated at c0 + t), then the step kernel
+  const fbk_partial part = fac_part(L, ws);
+  if (enqueue_prefix(shape, make_geometry(shape, u_cache), q_blk, carve(ws_layout(shape, shares), ws), shares, part,
+                     s, block_pos) != cudaSuccess)
+    return FBK_ERR_CUDA;
+  return from_cuda(enqueue_merge(shape, merge_geometry(shape, block_pos), q_blk, k_blk, v_blk, part, out_blk,
+                                 lse_blk, s));
+}
+
+fbk_status fbk_page_means(const fbk_shape *shape, const fbk_kv_cache *cache, float *means, void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if ((st = check_cache(shape, cache)) != FBK_OK) return st;
+  if (!cache->paged) return FBK_ERR_UNSUPPORTED;
+  if (!means) return FBK_ERR_INVALID_ARG;
+  return from_cuda(launch_page_means(make_geometry(shape, cache), means, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+size_t fbk_select_pages_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache) {
+  if (check_shape(shape) != FBK_OK || !cache || !cache->paged || cache->max_pages_per_seq < 1) return 0;
+  const size_t qrot = (size_t)shape->batch * shape->block_len * shape->n_q_heads * shape->head_dim * 4;
+  return align256(qrot) + align256((size_t)shape->batch * cache->max_pages_per_seq * 4);
+}
+
+fbk_status fbk_select_pages(const fbk_shape *shape, const void *q_blk, const fbk_kv_cache *cache, const float *means,
+                            int32_t k, int32_t *kept_table, int32_t *kept_lens, void *ws, size_t ws_bytes,
+                            void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if ((st = check_cache(shape, cache)) != FBK_OK) return st;
+  if (!cache->paged) return FBK_ERR_UNSUPPORTED;
+  if (!q_blk || !means || !kept_table || !kept_lens || k < 1) return FBK_ERR_INVALID_ARG;
+  if ((size_t)cache->max_pages_per_seq * 8 > 200 * 1024) return FBK_ERR_UNSUPPORTED;  // scores + flags in smem
+  const size_t need = fbk_select_pages_workspace_bytes(shape, cache);
+  if (!ws || ws_bytes < need) return FBK_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return FBK_ERR_UNSUPPORTED;
+  const int sms = default_shares();
+  if (sms < 1) return FBK_ERR_CUDA;
+  float *qrot = static_cast<float *>(ws);
+  float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) +
+                                            align256((size_t)shape->batch * shape->block_len * shape->n_q_heads *
+                                                     shape->head_dim * 4));
+  return from_cuda(launch_select_pages(make_geometry(shape, cache), static_cast<const __nv_bfloat16 *>(q_blk), means,
+                                       k, qrot, scores, kept_table, kept_lens, sms,
+                                       static_cast<cudaStream_t>(cuda_stream)));
+}
+
+fbk_status fbk_residual_capture(const fbk_shape *shape, const fbk_partial *dense, const fbk_partial *sparse,
+                                float *r_o, float *r_lse, void *cuda_stream) {
+  fbk_status st = check_shape(shape, true, 256);
+  if (st != FBK_OK) return st;
+  if (!dense || !sparse || !dense->o_unnorm || !dense->m || !dense->l || !sparse->o_unnorm || !sparse->m ||
+      !sparse->l || !r_o || !r_lse)
+    return FBK_ERR_INVALID_ARG;
+  const int sms = default_shares();
+  if (sms < 1) return FBK_ERR_CUDA;
+  const int rows = shape->batch * shape->n_q_heads * shape->block_len;
+  return from_cuda(launch_residual_capture(rows, shape->head_dim, *dense, *sparse, r_o, r_lse, sms,
+                                           static_cast<cudaStream_t>(cuda_stream)));
+}
+
+fbk_status fbk_residual_apply(const fbk_shape *shape, const fbk_partial *sparse, const float *r_o,
+                              const float *r_lse, const fbk_partial *ext, void *cuda_stream) {
+  fbk_status st = check_shape(shape, true, 256);
+  if (st != FBK_OK) return st;
+  if (!sparse || !ext || !sparse->o_unnorm || !sparse->m || !sparse->l || !ext->o_unnorm || !ext->m || !ext->l ||
+      !r_o || !r_lse)
+    return FBK_ERR_INVALID_ARG;
+  const int sms = default_shares();
+  if (sms < 1) return FBK_ERR_CUDA;
+  const int rows = shape->batch * shape->n_q_heads * shape->block_len;
+  return from_cuda(launch_residual_apply(rows, shape->head_dim, *sparse, r_o, r_lse, *ext, sms,
+                                         static_cast<cudaStream_t>(cuda_stream)));
 }
 
 const char *fbk_status_string(fbk_status status) {

@@ -277,7 +277,23 @@ cudaError_t launch_d(const Geometry &g, const FacRowsArgs &a0, int sms, cudaStre
   return launch_pdl(kern, dim3((unsigned)ctas), dim3(FR_WARPS * 32), lay.bytes, st, g, a);
 }
 
+// Rotation base of every chunk of U's rows for one sequence: the chunks before
+// the block start at positions 0, cmax, 2 cmax, ...; those after it at
+// c0 + B + j cmax (U's row c0 + j cmax sits at that position).
+__global__ void chunk_positions_kernel(int *pos, int n_before, int n_after, int c0, int cmax, int blk) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k < n_before) pos[k] = k * cmax;
+  else if (k < n_before + n_after) pos[k] = c0 + (k - n_before) * cmax + blk;
+}
+
 }  // namespace
+
+cudaError_t launch_chunk_positions(int *pos, int n_before, int n_after, int c0, int cmax, int blk, cudaStream_t st) {
+  const int n = n_before + n_after;
+  if (n == 0) return cudaSuccess;
+  chunk_positions_kernel<<<(n + 255) / 256, 256, 0, st>>>(pos, n_before, n_after, c0, cmax, blk);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_facache_rows(const Geometry &g, const FacRowsArgs &a, int sms, cudaStream_t st) {
   return g.d == 128 ? launch_d<128>(g, a, sms, st) : launch_d<64>(g, a, sms, st);

@@ -23,4 +23,8 @@ struct FacRowsArgs {
 // One launch; sms = the device's SM count.
 cudaError_t launch_facache_rows(const Geometry &g, const FacRowsArgs &a, int sms, cudaStream_t st);
 
+// Writes the rotation base of each chunk of U's rows of one sequence (kernel
+// parameters only; see facache_rows.cu).
+cudaError_t launch_chunk_positions(int *pos, int n_before, int n_after, int c0, int cmax, int blk, cudaStream_t st);
+
 }  // namespace fbk

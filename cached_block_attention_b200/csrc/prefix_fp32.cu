@@ -8,6 +8,7 @@
 // indexing and merge logic from tensor-core rounding. Query rows are handled
 // 32 at a time; each 32-row chunk re-reads the piece's tiles (from L2).
 #include "launch.h"
+#include "prefix_at.h"
 
 namespace fbk {
 namespace {
@@ -30,7 +31,8 @@ struct Smem {
 template <int D>
 __global__ void __launch_bounds__(THREADS) prefix_fp32_kernel(Geometry g,
                                                               const __nv_bfloat16 *__restrict__ q,
-                                                              Workspace ws, int shares) {
+                                                              Workspace ws, int shares,
+                                                              const int *__restrict__ qpos) {
   extern __shared__ float4 smem_f4[];
   float *sm = reinterpret_cast<float *>(smem_f4);
   using S = Smem<D>;
@@ -52,6 +54,7 @@ __global__ void __launch_bounds__(THREADS) prefix_fp32_kernel(Geometry g,
   Piece p;
   while (walk.next(g, p)) {
     const long long slot = (long long)blockIdx.x + p.u;
+    const int pos0 = qpos ? qpos[p.b] : p.L;  // rotation base of the block's rows
     for (int r0 = 0; r0 < g.rows; r0 += ROWS_PER_PASS) {
       __syncthreads();  // previous users of Qf are done
       for (int idx = threadIdx.x; idx < ROWS_PER_PASS * (D / 2); idx += THREADS) {
@@ -61,7 +64,7 @@ __global__ void __launch_bounds__(THREADS) prefix_fp32_kernel(Geometry g,
           const int hl = r / g.blk, t = r % g.blk, h = p.kvh * g.group + hl;
           const __nv_bfloat16 *src = q + (((long long)p.b * g.blk + t) * g.hq + h) * D;
           const float x1 = __bfloat162float(src[i]), x2 = __bfloat162float(src[i + D / 2]);
-          const float2 cs = rope_cs_f32(p.L + t, freq_over_pi(i, D, g.log2_base));
+          const float2 cs = rope_cs_f32(pos0 + t, freq_over_pi(i, D, g.log2_base));
           y1 = x1 * cs.x - x2 * cs.y;
           y2 = x2 * cs.x + x1 * cs.y;
         }
@@ -152,20 +155,25 @@ __global__ void __launch_bounds__(THREADS) prefix_fp32_kernel(Geometry g,
 }
 
 template <int D>
-cudaError_t launch_d(const Geometry &g, const __nv_bfloat16 *q, const Workspace &ws, int shares,
+cudaError_t launch_d(const Geometry &g, const __nv_bfloat16 *q, const int *qpos, const Workspace &ws, int shares,
                      cudaStream_t st) {
   const size_t bytes = sizeof(float) * Smem<D>::FLOATS;
   cudaError_t e = cudaFuncSetAttribute(prefix_fp32_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
-  return launch_pdl(prefix_fp32_kernel<D>, dim3(shares), dim3(THREADS), bytes, st, g, q, ws, shares);
+  return launch_pdl(prefix_fp32_kernel<D>, dim3(shares), dim3(THREADS), bytes, st, g, q, ws, shares, qpos);
 }
 
 }  // namespace
 
+cudaError_t launch_prefix_fp32_at(const Geometry &g, const __nv_bfloat16 *q, const int *qpos, const Workspace &ws,
+                                  int shares, cudaStream_t st) {
+  return g.d == 128 ? launch_d<128>(g, q, qpos, ws, shares, st) : launch_d<64>(g, q, qpos, ws, shares, st);
+}
+
 cudaError_t launch_prefix_fp32(const Geometry &g, const __nv_bfloat16 *q, const Workspace &ws,
                                int shares, cudaStream_t st) {
-  return g.d == 128 ? launch_d<128>(g, q, ws, shares, st) : launch_d<64>(g, q, ws, shares, st);
+  return launch_prefix_fp32_at(g, q, nullptr, ws, shares, st);
 }
 
 }  // namespace fbk

@@ -41,6 +41,7 @@
 #include <algorithm>
 
 #include "launch.h"
+#include "prefix_at.h"
 #include "tc.cuh"
 
 namespace fbk {
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
 // G*B are zero. One thread per 8 rotation pairs (chunk c of each half of a row).
 template <int D, int MT>
 __global__ void __launch_bounds__(256) rope_q_kernel(Geometry g, const __nv_bfloat16 *__restrict__ q,
-                                                    __nv_bfloat16 *__restrict__ qrot) {
+                                                    __nv_bfloat16 *__restrict__ qrot, const int *__restrict__ qpos) {
   constexpr int HALF = D / 2, KI = D / 16, ROWS = MT * 128;
   __shared__ double theta[HALF];
   for (int i = threadIdx.x; i < HALF; i += blockDim.x) theta[i] = freq_over_pi(i, D, g.log2_base);
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(256) rope_q_kernel(Geometry g, const __nv_bflo
     uint4 y1 = make_uint4(0, 0, 0, 0), y2 = make_uint4(0, 0, 0, 0);
     if (r < g.rows) {
       const int t = r % g.blk, h = kvh * g.group + r / g.blk;
-      const int L = prefix_len(g, b);
+      const int L = qpos ? qpos[b] : prefix_len(g, b);  // rotation base of the block's rows
       const uint4 *src = reinterpret_cast<const uint4 *>(q + (((long long)b * g.blk + t) * g.hq + h) * D);
       const uint4 a = src[c], bq = src[c + KI];
       const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {bq.x, bq.y, bq.z, bq.w};
@@ -547,7 +548,7 @@ bool make_map(CUtensorMap *m, const void *base, long long rows, int d, int boxh)
 }
 
 template <int D, int MT>
-cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const Workspace &ws, int shares,
+cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const int *qpos, const Workspace &ws, int shares,
                        cudaStream_t st) {
   using C = Cfg<D, MT>;
   const long long rows = g.paged ? g.num_pages * g.hkv * g.page_size : (long long)g.batch * g.hkv * g.cap;
@@ -563,7 +564,7 @@ cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const Workspac
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long items = qrows * (D / 16);
   const int rq_ctas = (int)std::min<long long>((items + 255) / 256, 8ll * sms);
-  cudaError_t e = launch_pdl(rope_q_kernel<D, MT>, dim3(rq_ctas), dim3(256), 0, st, g, q, ws.qrot);
+  cudaError_t e = launch_pdl(rope_q_kernel<D, MT>, dim3(rq_ctas), dim3(256), 0, st, g, q, ws.qrot, qpos);
   if (e != cudaSuccess) return e;
   auto kern = prefix_tc_kernel<D, MT>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -573,12 +574,17 @@ cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const Workspac
 
 }  // namespace
 
-cudaError_t launch_prefix_tc(const Geometry &g, const __nv_bfloat16 *q, const Workspace &ws,
-                             int shares, cudaStream_t st) {
+cudaError_t launch_prefix_tc_at(const Geometry &g, const __nv_bfloat16 *q, const int *qpos, const Workspace &ws,
+                                int shares, cudaStream_t st) {
   const bool two = g.rows > 128;
   if (g.d == 128)
-    return two ? launch_cfg<128, 2>(g, q, ws, shares, st) : launch_cfg<128, 1>(g, q, ws, shares, st);
-  return two ? launch_cfg<64, 2>(g, q, ws, shares, st) : launch_cfg<64, 1>(g, q, ws, shares, st);
+    return two ? launch_cfg<128, 2>(g, q, qpos, ws, shares, st) : launch_cfg<128, 1>(g, q, qpos, ws, shares, st);
+  return two ? launch_cfg<64, 2>(g, q, qpos, ws, shares, st) : launch_cfg<64, 1>(g, q, qpos, ws, shares, st);
+}
+
+cudaError_t launch_prefix_tc(const Geometry &g, const __nv_bfloat16 *q, const Workspace &ws,
+                             int shares, cudaStream_t st) {
+  return launch_prefix_tc_at(g, q, nullptr, ws, shares, st);
 }
 
 }  // namespace fbk

@@ -34,7 +34,9 @@ DEVERR_TIMEOUT = 8
 EXPORTS = ("fbk_prefix_workspace_bytes", "fbk_default_num_splits", "fbk_prefix_partial",
            "fbk_block_attn_merge", "fbk_commit_block_rope_append", "fbk_full_ref_attn",
            "fbk_status_string", "fbk_prefix_partial_static_scratch", "fbk_decode_block",
-           "fbk_fp8_group_quant", "fbk_facache_unchanged_rows")
+           "fbk_fp8_group_quant", "fbk_facache_unchanged_rows", "fbk_prefix_partial_at",
+           "fbk_facache_workspace_bytes", "fbk_facache_refresh", "fbk_facache_step", "fbk_page_means",
+           "fbk_select_pages_workspace_bytes", "fbk_select_pages", "fbk_residual_capture", "fbk_residual_apply")
 
 STATIC_SCRATCH_BYTES = 32 << 20  # FBK_STATIC_SCRATCH_BYTES
 
@@ -90,6 +92,27 @@ _lib.fbk_fp8_group_quant.restype = ctypes.c_int
 _lib.fbk_facache_unchanged_rows.argtypes = [_P(_Shape), ctypes.c_int32, _vp, _P(_Partial), _vp, _vp, _vp, _vp,
                                             _vp, _vp]
 _lib.fbk_facache_unchanged_rows.restype = ctypes.c_int
+_lib.fbk_prefix_partial_at.argtypes = [_P(_Shape), _vp, _vp, _P(_Cache), _P(_Partial), _vp, ctypes.c_size_t,
+                                       ctypes.c_int32, _vp]
+_lib.fbk_prefix_partial_at.restype = ctypes.c_int
+_lib.fbk_facache_workspace_bytes.argtypes = [_P(_Shape), ctypes.c_int32, ctypes.c_int32]
+_lib.fbk_facache_workspace_bytes.restype = ctypes.c_size_t
+_lib.fbk_facache_refresh.argtypes = [_P(_Shape), ctypes.c_int32, _vp, _P(ctypes.c_int32), _P(_Cache), _P(_Partial),
+                                     _vp, ctypes.c_size_t, ctypes.c_int32, _vp]
+_lib.fbk_facache_refresh.restype = ctypes.c_int
+_lib.fbk_facache_step.argtypes = [_P(_Shape), ctypes.c_int32, _vp, _P(_Partial), _vp, _vp, _vp, _vp, _P(_Cache), _vp,
+                                  _vp, _vp, _vp, _vp, ctypes.c_size_t, ctypes.c_int32, _vp]
+_lib.fbk_facache_step.restype = ctypes.c_int
+_lib.fbk_page_means.argtypes = [_P(_Shape), _P(_Cache), _vp, _vp]
+_lib.fbk_page_means.restype = ctypes.c_int
+_lib.fbk_select_pages_workspace_bytes.argtypes = [_P(_Shape), _P(_Cache)]
+_lib.fbk_select_pages_workspace_bytes.restype = ctypes.c_size_t
+_lib.fbk_select_pages.argtypes = [_P(_Shape), _vp, _P(_Cache), _vp, ctypes.c_int32, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.fbk_select_pages.restype = ctypes.c_int
+_lib.fbk_residual_capture.argtypes = [_P(_Shape), _P(_Partial), _P(_Partial), _vp, _vp, _vp]
+_lib.fbk_residual_capture.restype = ctypes.c_int
+_lib.fbk_residual_apply.argtypes = [_P(_Shape), _P(_Partial), _vp, _vp, _P(_Partial), _vp]
+_lib.fbk_residual_apply.restype = ctypes.c_int
 _lib.fbk_status_string.argtypes = [ctypes.c_int]
 _lib.fbk_status_string.restype = ctypes.c_char_p
 
@@ -198,6 +221,15 @@ def prefix_partial(shape: Shape, q_blk: torch.Tensor, cache: KVCache, out: Parti
                                    _stream(stream)), "fbk_prefix_partial")
 
 
+def prefix_partial_at(shape: Shape, q_blk: torch.Tensor, q_pos: torch.Tensor, cache: KVCache, out: Partial,
+                      ws: torch.Tensor, num_splits: int = 0, stream=None) -> None:
+    """prefix_partial with the block's rows rotated at q_pos[b] + t (q_pos int32 [b] on the device)."""
+    cs, cc, po = shape.c(), cache.c(), out.c()
+    _check(_lib.fbk_prefix_partial_at(ctypes.byref(cs), _ptr(q_blk), _ptr(q_pos), ctypes.byref(cc), ctypes.byref(po),
+                                      _ptr(ws), ws.numel() * ws.element_size(), num_splits, _stream(stream)),
+           "fbk_prefix_partial_at")
+
+
 def prefix_partial_static_scratch(shape: Shape, q_blk: torch.Tensor, cache: KVCache, out: Partial,
                                   num_splits: int = 0, stream=None) -> None:
     """prefix_partial using the library's built-in per-device scratch array
@@ -288,6 +320,61 @@ def facache_unchanged_rows(shape: Shape, q_u: torch.Tensor, state: Partial, k_bl
     _check(_lib.fbk_facache_unchanged_rows(ctypes.byref(cs), q_u.shape[1], _ptr(q_u), ctypes.byref(ps),
                                            _ptr(k_blk), _ptr(v_blk), _ptr(block_pos), _ptr(out), _ptr(lse),
                                            _stream(stream)), "fbk_facache_unchanged_rows")
+
+
+def facache_workspace_bytes(shape: Shape, n_rows: int, num_splits: int = 0) -> int:
+    cs = shape.c()
+    return int(_lib.fbk_facache_workspace_bytes(ctypes.byref(cs), n_rows, num_splits))
+
+
+def facache_refresh(shape: Shape, q_u_raw: torch.Tensor, block_pos_host, u_cache: KVCache, state: Partial,
+                    ws: torch.Tensor, num_splits: int = 0, stream=None) -> None:
+    """FACache's state of U's rows over U's keys: q_u_raw [b, U, Hq, d] before RoPE,
+    block_pos_host a host sequence of c0 per sequence, state [b, Hq, U, d] / [b, Hq, U]."""
+    pos = (ctypes.c_int32 * shape.batch)(*[int(c) for c in block_pos_host])
+    cs, cc, ps = shape.c(), u_cache.c(), state.c()
+    _check(_lib.fbk_facache_refresh(ctypes.byref(cs), q_u_raw.shape[1], _ptr(q_u_raw), pos, ctypes.byref(cc),
+                                    ctypes.byref(ps), _ptr(ws), ws.numel() * ws.element_size(), num_splits,
+                                    _stream(stream)), "fbk_facache_refresh")
+
+
+def facache_step(shape: Shape, q_u_rot, state: Partial, q_blk, k_blk, v_blk, block_pos, u_cache: KVCache, out_u,
+                 out_blk, ws: torch.Tensor, lse_u=None, lse_blk=None, num_splits: int = 0, stream=None) -> None:
+    """One denoising step of FACache over a whole sequence: U's rows and the block's rows."""
+    cs, cc, ps = shape.c(), u_cache.c(), state.c()
+    _check(_lib.fbk_facache_step(ctypes.byref(cs), q_u_rot.shape[1], _ptr(q_u_rot), ctypes.byref(ps), _ptr(q_blk),
+                                 _ptr(k_blk), _ptr(v_blk), _ptr(block_pos), ctypes.byref(cc), _ptr(out_u),
+                                 _ptr(lse_u), _ptr(out_blk), _ptr(lse_blk), _ptr(ws), ws.numel() * ws.element_size(),
+                                 num_splits, _stream(stream)), "fbk_facache_step")
+
+
+def page_means(shape: Shape, cache: KVCache, means: torch.Tensor, stream=None) -> None:
+    cs, cc = shape.c(), cache.c()
+    _check(_lib.fbk_page_means(ctypes.byref(cs), ctypes.byref(cc), _ptr(means), _stream(stream)), "fbk_page_means")
+
+
+def select_pages_workspace_bytes(shape: Shape, cache: KVCache) -> int:
+    cs, cc = shape.c(), cache.c()
+    return int(_lib.fbk_select_pages_workspace_bytes(ctypes.byref(cs), ctypes.byref(cc)))
+
+
+def select_pages(shape: Shape, q_blk, cache: KVCache, means, k: int, kept_table, kept_lens, ws, stream=None) -> None:
+    cs, cc = shape.c(), cache.c()
+    _check(_lib.fbk_select_pages(ctypes.byref(cs), _ptr(q_blk), ctypes.byref(cc), _ptr(means), k, _ptr(kept_table),
+                                 _ptr(kept_lens), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "fbk_select_pages")
+
+
+def residual_capture(shape: Shape, dense: Partial, sparse: Partial, r_o, r_lse, stream=None) -> None:
+    cs, pd, ps = shape.c(), dense.c(), sparse.c()
+    _check(_lib.fbk_residual_capture(ctypes.byref(cs), ctypes.byref(pd), ctypes.byref(ps), _ptr(r_o), _ptr(r_lse),
+                                     _stream(stream)), "fbk_residual_capture")
+
+
+def residual_apply(shape: Shape, sparse: Partial, r_o, r_lse, ext: Partial, stream=None) -> None:
+    cs, ps, pe = shape.c(), sparse.c(), ext.c()
+    _check(_lib.fbk_residual_apply(ctypes.byref(cs), ctypes.byref(ps), _ptr(r_o), _ptr(r_lse), ctypes.byref(pe),
+                                   _stream(stream)), "fbk_residual_apply")
 
 
 # raw handles for tests of the C ABI itself

@@ -117,7 +117,7 @@ typedef struct fbk_partial {
  * fp32 for the per-share states plus b*Hkv * 128*ceil(G*B/128) * d bf16 for the
  * rotated query rows, each region rounded up to 256 bytes. Depends only on b,
  * Hkv, G*B, d and the share count, not on the prefix lengths. Returns 0 for an
- * invalid shape. */
+ * invalid shape; B up to 256 is valid here (fbk_prefix_partial_at's blocks). */
 size_t fbk_prefix_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache,
                                   int32_t num_splits);
 
@@ -183,6 +183,20 @@ fbk_status fbk_full_ref_attn(const fbk_shape *shape, const void *q_blk, const vo
                              const void *v_blk, const fbk_kv_cache *cache, void *out,
                              float *lse, void *cuda_stream);
 
+/* fbk_prefix_partial with the block's query rows rotated at q_pos[b] + t
+ * instead of prefix_lens[b] + t (q_pos: int32 [b] on the device, required).
+ * The cached keys are still rows 0 .. prefix_lens[b]-1 of the cache, stored
+ * after RoPE at whatever positions they hold. This lets the block's rows meet
+ * keys that lie after the block, such as a masked suffix in full-sequence
+ * decoding (LaCache §3.3.1: U holds the prompt and the masked suffix). It also
+ * lets any run of rows with consecutive positions stand in as the "block",
+ * for instance a chunk of U's rows when FACache's cached state of U over U's
+ * keys is computed (LaCache §3.3.3). The block length may exceed 64 here: B is
+ * limited only by G*B <= 256. Otherwise as fbk_prefix_partial. */
+fbk_status fbk_prefix_partial_at(const fbk_shape *shape, const void *q_blk, const int32_t *q_pos,
+                                 const fbk_kv_cache *cache, const fbk_partial *out, void *ws, size_t ws_bytes,
+                                 int32_t num_splits, void *cuda_stream);
+
 /* Size of the library's built-in scratch array (per device) used by
  * fbk_prefix_partial_static_scratch: 32 MiB. */
 #define FBK_STATIC_SCRATCH_BYTES (32u << 20)
@@ -200,6 +214,14 @@ fbk_status fbk_full_ref_attn(const fbk_shape *shape, const void *q_blk, const vo
  * allocates nothing either: its scratch is a fixed array of
  * FBK_STATIC_SCRATCH_BYTES bytes in the library's own device image, one per
  * device, created when the CUDA module is loaded.
+ *
+ * Footprint. The array lives in a device module of its own (it holds no
+ * kernel), and a device that loads that module holds the 32 MiB until the
+ * process exits. With lazy module loading (the CUDA default,
+ * CUDA_MODULE_LOADING=LAZY) only the address lookup of this entry point's
+ * first call loads it, so a process that never calls it pays nothing; with
+ * CUDA_MODULE_LOADING=EAGER every device the process initialises pays it when
+ * the library loads, whether or not this entry point is ever called.
  *
  * Arguments are those of fbk_prefix_partial minus ws and ws_bytes.
  *
@@ -324,6 +346,79 @@ fbk_status fbk_fp8_group_quant(const void *x, int64_t rows, int64_t cols, void *
 fbk_status fbk_facache_unchanged_rows(const fbk_shape *shape, int32_t n_rows, const void *q_u,
                                       const fbk_partial *state, const void *k_blk, const void *v_blk,
                                       const int32_t *block_pos, void *out, float *lse, void *cuda_stream);
+
+/* FACache over a whole sequence as two calls (LaCache §3.3.1-§3.3.3, App. J).
+ * The sequence's rows outside the current block (U: prompt, earlier blocks,
+ * masked suffix; n_rows per sequence, in sequence order with the block
+ * removed) keep their state over U's keys for the whole block:
+ * fbk_facache_refresh computes it once per block, and fbk_facache_step uses it
+ * at every denoising step. A step's outputs equal attention over the whole
+ * sequence. Both calls use a workspace of fbk_facache_workspace_bytes(shape,
+ * n_rows, num_splits) bytes (256-byte aligned, contents irrelevant on entry).
+ * The shape rules are those of the block path (B <= 64, G*B <= 256).
+ *
+ * u_cache: U's K (after RoPE, at the rows' own positions) and V, contiguous
+ *   [b, Hkv, capacity >= n_rows, d], with prefix_lens[b] = n_rows on the device.
+ *
+ * fbk_facache_refresh:
+ *  q_u_raw: bf16 [b, n_rows, Hq, d], U's queries BEFORE RoPE.
+ *  block_pos_host: int32 [b] on the HOST: c0, 0 <= c0 <= n_rows. Row i of U
+ *           sits at position i (i < c0) or i + B.
+ *  state:   the output, o_unnorm fp32 [b, Hq, n_rows, d] (16-byte aligned),
+ *           m and l fp32 [b, Hq, n_rows].
+ *  The rows are processed in chunks of up to 256/G rows that do not cross the
+ *  block, one prefix computation each, whose states are copied into place.
+ *
+ * fbk_facache_step (FBK_BF16 only):
+ *  q_u_rot: bf16 [b, n_rows, Hq, d], U's queries AFTER RoPE (RoPECache).
+ *  state:   from fbk_facache_refresh.
+ *  q_blk, k_blk, v_blk: the block, bf16 [b, B, Hq|Hkv, d], Q and K before RoPE.
+ *  block_pos: int32 [b] on the device: c0.
+ *  out_u: bf16 [b, n_rows, Hq, d]; lse_u fp32 [b, Hq, n_rows] or NULL.
+ *  out_blk: bf16 [b, B, Hq, d]; lse_blk fp32 [b, Hq, B] or NULL.
+ *  Launches: fbk_facache_unchanged_rows's kernel for U's rows; for the block's
+ *  rows, the prefix computation over U's keys with the rows rotated at c0 + t,
+ *  then fbk_block_attn_merge's kernel. */
+size_t fbk_facache_workspace_bytes(const fbk_shape *shape, int32_t n_rows, int32_t num_splits);
+fbk_status fbk_facache_refresh(const fbk_shape *shape, int32_t n_rows, const void *q_u_raw,
+                               const int32_t *block_pos_host, const fbk_kv_cache *u_cache,
+                               const fbk_partial *state, void *ws, size_t ws_bytes, int32_t num_splits,
+                               void *cuda_stream);
+fbk_status fbk_facache_step(const fbk_shape *shape, int32_t n_rows, const void *q_u_rot, const fbk_partial *state,
+                            const void *q_blk, const void *k_blk, const void *v_blk, const int32_t *block_pos,
+                            const fbk_kv_cache *u_cache, void *out_u, float *lse_u, void *out_blk, float *lse_blk,
+                            void *ws, size_t ws_bytes, int32_t num_splits, void *cuda_stream);
+
+/* Sparse block-external attention with a cached residual (FlashBlock,
+ * Abstract: cached block-external attention combined with sparse attention as
+ * residual reuse). Reading: pages of the prefix (the paged cache's pages) are
+ * scored by the largest tau <RoPE(q_t, L_b + t), kbar> over the block's rows
+ * and query heads, kbar the page's mean key; the top k pages per sequence form
+ * a page table of their own for fbk_prefix_partial_at (queries rotated at the
+ * true L_b + t); at a dense step the residual (O~/l, lse) dense minus sparse
+ * is captured; at later steps the sparse state plus the residual becomes the
+ * state fbk_block_attn_merge merges. Paged caches only.
+ *
+ * fbk_page_means: means fp32 [b, max_pages_per_seq, Hkv, d], the mean key of
+ *   every logical page of the prefix (pages past prefix_lens untouched).
+ * fbk_select_pages: q_blk bf16 [b, B, Hq, d] before RoPE; k >= 1 pages kept;
+ *   kept_table int32 [b, k] (physical page ids in increasing logical order,
+ *   -1 past the kept count) and kept_lens int32 [b] (their token count, the
+ *   partial last page included), both on the device; workspace of
+ *   fbk_select_pages_workspace_bytes bytes, 256-byte aligned.
+ * fbk_residual_capture: r_o fp32 [b, Hq, B, d] and r_lse fp32 [b, Hq, B] from
+ *   the dense and the sparse state of the same queries (r_lse = -inf marks a
+ *   row with no prefix).
+ * fbk_residual_apply: ext = ((O~/l)_sparse + r_o, lse_sparse + r_lse, 1). */
+fbk_status fbk_page_means(const fbk_shape *shape, const fbk_kv_cache *cache, float *means, void *cuda_stream);
+size_t fbk_select_pages_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache);
+fbk_status fbk_select_pages(const fbk_shape *shape, const void *q_blk, const fbk_kv_cache *cache, const float *means,
+                            int32_t k, int32_t *kept_table, int32_t *kept_lens, void *ws, size_t ws_bytes,
+                            void *cuda_stream);
+fbk_status fbk_residual_capture(const fbk_shape *shape, const fbk_partial *dense, const fbk_partial *sparse,
+                                float *r_o, float *r_lse, void *cuda_stream);
+fbk_status fbk_residual_apply(const fbk_shape *shape, const fbk_partial *sparse, const float *r_o,
+                              const float *r_lse, const fbk_partial *ext, void *cuda_stream);
 
 /* Static text for a status code. */
 const char *fbk_status_string(fbk_status status);

@@ -71,7 +71,8 @@ def test_shape_validation(fbk, kw, code):
                                       ctypes.c_void_p(0x70000), ctypes.c_void_p(0x30000), ctypes.byref(p),
                                       ctypes.c_void_p(0x90000), None, None)
     assert st == code
-    assert fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), ctypes.byref(c), 4) == 0
+    if kw != dict(block_len=65):  # B in (64, 256] with G*B <= 256 is a valid prefix shape (fbk_prefix_partial_at)
+        assert fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), ctypes.byref(c), 4) == 0
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -266,3 +267,41 @@ int main(void) {
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+def test_prefix_partial_at_argument_checks(fbk):
+    """fbk_prefix_partial_at: q_pos is required; blocks longer than 64 are accepted while G*B <= 256."""
+    c = _cache(fbk)
+    p = fbk.CPartial(0x40000, 0x50000, 0x60000)
+    f = fbk.lib.fbk_prefix_partial_at
+    q, pos, ws = ctypes.c_void_p(0x70000), ctypes.c_void_p(0x30000), ctypes.c_void_p(0x80000)
+    s = _shape(fbk, n_q_heads=2, n_kv_heads=2, block_len=256)           # G*B = 256
+    assert f(ctypes.byref(s), q, None, ctypes.byref(c), ctypes.byref(p), ws, 1 << 30, 4, None) == -1
+    assert f(ctypes.byref(s), q, pos, ctypes.byref(c), ctypes.byref(p), None, 0, 4, None) == -4
+    s2 = _shape(fbk, n_q_heads=4, n_kv_heads=2, block_len=129)          # G*B = 258
+    assert f(ctypes.byref(s2), q, pos, ctypes.byref(c), ctypes.byref(p), ws, 1 << 30, 4, None) == -2
+    assert fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), ctypes.byref(c), 4) > 0
+
+
+def test_facache_refresh_and_step_argument_checks(fbk):
+    """Host checks of fbk_facache_refresh and fbk_facache_step; none reach a CUDA call."""
+    s = _shape(fbk)
+    p = fbk.CPartial(0x40000, 0x50000, 0x60000)
+    ptr = ctypes.c_void_p
+    pos = (ctypes.c_int32 * 1)(10)
+    bad_pos = (ctypes.c_int32 * 1)(101)
+    c = _cache(fbk)
+    paged = _cache(fbk, paged=1, page_size=64, max_pages_per_seq=4, num_pages=8, page_table=0x1000)
+    r = fbk.lib.fbk_facache_refresh
+    assert r(ctypes.byref(s), 100, ptr(0x70000), pos, ctypes.byref(paged), ctypes.byref(p), None, 0, 4, None) == -2
+    assert r(ctypes.byref(s), 100, ptr(0x70000), bad_pos, ctypes.byref(c), ctypes.byref(p), None, 0, 4, None) == -1
+    assert r(ctypes.byref(s), 100, ptr(0x70000), None, ctypes.byref(c), ctypes.byref(p), None, 0, 4, None) == -1
+    assert r(ctypes.byref(s), 0, None, pos, ctypes.byref(c), None, None, 0, 4, None) == 0
+    assert r(ctypes.byref(s), 100, ptr(0x70000), pos, ctypes.byref(c), ctypes.byref(p), None, 0, 4, None) == -4
+    n = fbk.lib.fbk_facache_workspace_bytes(ctypes.byref(s), 100, 4)
+    assert n > fbk.lib.fbk_prefix_workspace_bytes(ctypes.byref(s), None, 4)
+    st = fbk.lib.fbk_facache_step
+    args = [ptr(0x70000), ctypes.byref(p), ptr(0x71000), ptr(0x72000), ptr(0x73000), ptr(0x30000), ctypes.byref(c),
+            ptr(0x90000), None, ptr(0x91000), None]
+    assert st(ctypes.byref(_shape(fbk, mode=1)), 100, *args, ptr(0x100000), n, 4, None) == -2
+    assert st(ctypes.byref(s), 100, *args, ptr(0x100000), n - 1, 4, None) == -4
+    assert st(ctypes.byref(s), 100, *args, ptr(0x100010), n, 4, None) == -2

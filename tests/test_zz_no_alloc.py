@@ -2,9 +2,13 @@
 built-in scratch array instead of a caller workspace.
 
 The GPU tests call it through the C ABI twice in a row and compare each result
-with fbk_prefix_partial (caller workspace) on the same inputs, within the
-parity tolerance. This file is named to be collected last, so it also runs
-after every other test has used the library in the same process.
+with fbk_prefix_partial (caller workspace) on the same inputs. Both calls run
+the same kernels with the same share count and a fixed-order reduction, so the
+states must be bit-identical: a scratch-aliasing fault that moved a value by
+less than the parity tolerance would still fail. Each result is also checked
+within the parity tolerance, as the other tests check states. This file is
+named to be collected last, so it also runs after every other test has used
+the library in the same process.
 """
 import ctypes
 
@@ -31,8 +35,13 @@ def _call_static(fbk, case, q, out, num_splits=0):
 
 
 def _compare(got, ref, mname, what):
-    """States compared as the parity tests compare them: empty rows exactly
-    (0, -inf, 0), the rest through O~/l, m + log l and m."""
+    """Bit equality of O~, m and l with the workspace call, then the parity
+    tests' comparison: empty rows exactly (0, -inf, 0), the rest through O~/l,
+    m + log l and m."""
+    for name in ("o_unnorm", "m", "l"):
+        a, b = getattr(got, name), getattr(ref, name)
+        assert torch.equal(a, b), f"{what}: {name} differs from the workspace call " \
+            f"({int((a != b).sum())} elements)"
     H.check_partial(H.partial_to_host(got), H.partial_to_host(ref), mname, what)
 
 
