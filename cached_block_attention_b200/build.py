@@ -6,6 +6,11 @@ Compiles every csrc/*.cu with nvcc for sm_100a only and links them into
 cached_block_attention_b200/libfbk.so (CUDA runtime linked statically, no
 libcuda link: the tensor-map encoder is fetched through the runtime's driver
 entry-point query). Objects go to _build/ at the repository root.
+
+It also links libfbk_testhooks.so, the test build: the same objects except
+the prefix kernel's, which is compiled with FBK_TEST_HOOKS so that a test
+can shorten the kernel's bounded waits and withhold one of its loads
+(include/fbk_test_hooks.h). Only the bounded-wait test loads it.
 """
 from __future__ import annotations
 
@@ -21,6 +26,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfbk.so")
+TEST_LIB = os.path.join(PKG, "libfbk_testhooks.so")
+HOOKED = "prefix_tc.cu"  # the one source the test build compiles differently
 
 SOURCES = ["abi.cu", "prefix_tc.cu", "prefix_fp32.cu", "split_reduce.cu", "block_merge.cu",
            "commit.cu", "full_ref.cu", "fp8_quant.cu", "facache_rows.cu", "sparse_prefix.cu"]
@@ -47,32 +54,40 @@ def _newer(target: str, deps) -> bool:
 def build(verbose: bool = False, force: bool = False, ptxas_info: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
-    headers.append(os.path.join(INCLUDE, "fbk.h"))
+    headers += [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
     cc = nvcc()
 
-    def compile_one(src):
+    def compile_one(job):
+        src, hooks = job
         path = os.path.join(CSRC, src)
-        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
+        obj = os.path.join(BUILD, src.replace(".cu", "_hooks.o" if hooks else ".o"))
         if not force and not ptxas_info and _newer(obj, [path] + headers):
             return obj, ""
-        cmd = [cc] + FLAGS + (["-Xptxas", "-v"] if ptxas_info else []) + ["-c", path, "-o", obj]
+        cmd = ([cc] + FLAGS + (["-DFBK_TEST_HOOKS"] if hooks else []) + (["-Xptxas", "-v"] if ptxas_info else [])
+               + ["-c", path, "-o", obj])
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
         return obj, r.stderr
 
+    jobs = [(src, False) for src in SOURCES] + [(HOOKED, True)]
     with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        results = list(ex.map(compile_one, SOURCES))
-    objs = [o for o, _ in results]
+        results = list(ex.map(compile_one, jobs))
+    objs = {job: o for job, (o, _) in zip(jobs, results)}
     if verbose or ptxas_info:
-        for src, (_, log) in zip(SOURCES, results):
-            if log.strip():
+        for (src, hooks), (_, log) in zip(jobs, results):
+            if log.strip() and not hooks:
                 print(f"--- {src}\n{log}")
-    if force or not _newer(LIB, objs):
-        cmd = [cc] + ARCH + ["-shared", "-o", LIB] + objs
-        r = subprocess.run(cmd, capture_output=True, text=True)
-        if r.returncode != 0:
-            raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+
+    def link(target, parts):
+        if force or not _newer(target, parts):
+            cmd = [cc] + ARCH + ["-shared", "-o", target] + parts
+            r = subprocess.run(cmd, capture_output=True, text=True)
+            if r.returncode != 0:
+                raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+
+    link(LIB, [objs[(s, False)] for s in SOURCES])
+    link(TEST_LIB, [objs[(s, s == HOOKED)] for s in SOURCES])
     return LIB
 
 

@@ -32,9 +32,6 @@ struct TmaMaps;  // defined in prefix_tc.cu
 cudaError_t launch_prefix_fp32(const Geometry &g, const __nv_bfloat16 *q, const Workspace &ws,
                                int shares, cudaStream_t st);
 
-// tcgen05 / TMA prefix kernel (FBK_BF16): one CTA per share.
-cudaError_t launch_prefix_tc(const Geometry &g, const __nv_bfloat16 *q, const Workspace &ws,
-                             int shares, cudaStream_t st);
 
 // Fixed-order LSE reduction of the per-share states into the prefix state.
 cudaError_t launch_split_reduce(const Geometry &g, const Workspace &ws, int shares,

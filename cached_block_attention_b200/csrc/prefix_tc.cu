@@ -72,7 +72,8 @@ struct Cfg {
   static constexpr int B_ODONE = B_PFULL + 2 * MT;
   static constexpr int B_OFREE = B_ODONE + MT;
   static constexpr int B_DRAIN = B_OFREE + MT;  // [2]: S issuer, PV issuer
-  static constexpr int NBAR = B_DRAIN + 2;
+  static constexpr int B_VTAIL = B_DRAIN + 2;   // a partial V tile's own loads landed (V producer only)
+  static constexpr int NBAR = B_VTAIL + 1;
   static constexpr int LEN_OFF = BAR_OFF + NBAR * 8;  // [MAX_BATCH] int: validated L_b
   static constexpr int SCAN_OFF = LEN_OFF + MAX_BATCH * 4;  // [MAX_BATCH] int: tile scan
   static constexpr int MISC_OFF = SCAN_OFF + MAX_BATCH * 4;
@@ -89,7 +90,7 @@ struct Cfg {
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   const long long t0 = clock64();
   while (!mbar_test(bar, parity))
-    if (clock64() - t0 > WAIT_LIMIT_CLOCKS) return false;
+    if (clock64() - t0 > wait_limit()) return false;
   return true;
 }
 
@@ -98,20 +99,35 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t *>(&v);
 }
 
+// Keys of list tile j of piece p that exist (the unit's last tile may be partial).
+__device__ __forceinline__ int tile_keys(const Piece &p, int j) { return min(KV_TILE, p.L - j * KV_TILE); }
+
+// Rows a tile load brings in for n valid keys: whole boxes of boxh rows, then
+// 8-row boxes for the rest, so up to 7 rows past the unit's last key may be
+// loaded (their K only meets masked scores; their V rows are zeroed before the
+// P~ V product reads them).
+__device__ __forceinline__ int tile_rows(int n, int boxh) {
+  const int full = n / boxh * boxh;
+  return full + ((n - full + 7) & ~7);
+}
+
+// TMA loads of the n valid keys of tile j into a stage (each 64-column block
+// of the stage holds KV_TILE rows of 128 bytes, 128B swizzle). Rows past the
+// unit's keys are never requested in whole boxes: they may lie in memory the
+// caller never wrote.
 template <int D>
-__device__ __forceinline__ void load_kv_tile(const Geometry &g, const CUtensorMap *map, uint32_t dst,
-                                             const Piece &p, int j, int boxh, uint32_t bar,
+__device__ __forceinline__ void load_kv_tile(const Geometry &g, const CUtensorMap *map, const CUtensorMap *map8,
+                                             uint32_t dst, const Piece &p, int j, int n, int boxh, uint32_t bar,
                                              uint64_t pol) {
-  for (int rb = 0; rb < KV_TILE / boxh; ++rb) {
-    const long long pos = (long long)j * KV_TILE + (long long)rb * boxh;
-    long long row = 0;  // rows at or past L are masked later; any valid row will do
-    if (pos < p.L) {
-      row = cache_row(g, p.b, p.kvh, pos);
-      if (row < 0) row = 0;
-    }
+  int r = 0;
+  while (r < n) {
+    const bool whole = n - r >= boxh;
+    long long row = cache_row(g, p.b, p.kvh, (long long)j * KV_TILE + r);
+    if (row < 0) row = 0;  // bad page id: flagged; any row keeps the arithmetic going
 #pragma unroll
     for (int cb = 0; cb < D / 64; ++cb)
-      tma_load_2d(dst + cb * (KV_TILE * 128) + rb * boxh * 128, map, cb * 64, (int)row, bar, pol);
+      tma_load_2d(dst + cb * (KV_TILE * 128) + r * 128, whole ? map : map8, cb * 64, (int)row, bar, pol);
+    r += whole ? boxh : 8;
   }
 }
 
@@ -119,7 +135,8 @@ template <int D, int MT>
 __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     prefix_tc_kernel(const __grid_constant__ Geometry g, const __nv_bfloat16 *__restrict__ q,
                      const Workspace ws, const int shares, const __grid_constant__ CUtensorMap tmk,
-                     const __grid_constant__ CUtensorMap tmv, const int boxh,
+                     const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmk8,
+                     const __grid_constant__ CUtensorMap tmv8, const int boxh,
                      const __grid_constant__ CUtensorMap tmq) {
   using C = Cfg<D, MT>;
   extern __shared__ uint8_t smem_raw[];
@@ -136,6 +153,12 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::MISC_OFF);
 
   // ---- before the wait: nothing another kernel writes is touched here
+  // The V ring starts at zero: a stage only ever holds these zeros, rows of
+  // committed keys, or rows zeroed after a partial load, so every V row that
+  // meets a zero weight in O += P~ V is finite.
+  for (int o = threadIdx.x * 16; o < C::NS * C::KV_BYTES; o += C::THREADS * 16)
+    *reinterpret_cast<uint4 *>(smem + C::V_OFF + o) = make_uint4(0, 0, 0, 0);
+  fence_proxy_async();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar(C::B_KFULL + s), 1);
@@ -156,6 +179,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     }
     mbar_init(bar(C::B_DRAIN), 1);
     mbar_init(bar(C::B_DRAIN + 1), 1);
+    mbar_init(bar(C::B_VTAIL), 1);
     *abort_flag = 0;
     mbar_fence_init();
     prefetch_tmap(&tmk);
@@ -193,20 +217,49 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
     if (lane == 0) {
       const bool is_k = warp == 0;
       const CUtensorMap *map = is_k ? &tmk : &tmv;
+      const CUtensorMap *map8 = is_k ? &tmk8 : &tmv8;
       const int b_full = is_k ? C::B_KFULL : C::B_VFULL, b_empty = is_k ? C::B_KEMPTY : C::B_VEMPTY;
       const uint32_t ring = sb + (is_k ? C::K_OFF : C::V_OFF);
       const uint64_t pol = policy_evict_first();
       PieceWalker walk;
       walk.init(g, s_len, s_scan, blockIdx.x, T, shares);
       Piece p;
-      int i = 0;
+      int i = 0, ntail = 0;
       bool ok = true;
       while (ok && walk.next(g, p)) {
         for (int j = p.tile_begin; j < p.tile_end; ++j, ++i) {
           const int st = i % C::NS;
           if (!mbar_wait(bar(b_empty + st), ((i / C::NS) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(bar(b_full + st), C::KV_BYTES);
-          load_kv_tile<D>(g, map, ring + st * C::KV_BYTES, p, j, boxh, bar(b_full + st), pol);
+#ifdef FBK_TEST_HOOKS
+          if (is_k && blockIdx.x == 0 && i == g_test_withhold_stage) continue;  // a tile that never lands
+#endif
+          const int n = tile_keys(p, j), nrows = tile_rows(n, boxh);
+          const uint32_t bytes = (uint32_t)nrows * 128u * (D / 64);
+          if (is_k || nrows == n) {
+            mbar_expect_tx(bar(b_full + st), bytes);
+            load_kv_tile<D>(g, map, map8, ring + st * C::KV_BYTES, p, j, n, boxh, bar(b_full + st), pol);
+          } else {
+            // a partial V tile (once per unit): its loads land on a barrier of
+            // their own, the up to 7 rows past the unit's last key are zeroed,
+            // and only then is the stage marked full for O += P~ V
+            mbar_expect_tx(bar(C::B_VTAIL), bytes);
+            load_kv_tile<D>(g, map, map8, ring + st * C::KV_BYTES, p, j, n, boxh, bar(C::B_VTAIL), pol);
+            if (!mbar_wait(bar(C::B_VTAIL), ntail & 1, abort_flag)) {
+              mbar_wait_drain(bar(C::B_VTAIL), ntail & 1);  // no TMA write may be in flight when the CTA leaves
+              ok = false;
+              break;
+            }
+            ++ntail;
+            uint8_t *stage = smem + C::V_OFF + st * C::KV_BYTES;
+            for (int rr = n; rr < nrows; ++rr)
+#pragma unroll
+              for (int cb = 0; cb < D / 64; ++cb)
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                  *reinterpret_cast<uint4 *>(stage + cb * (KV_TILE * 128) + rr * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+            fence_proxy_async();
+            mbar_arrive(bar(b_full + st));
+          }
         }
       }
       // no TMA write may be in flight when the CTA leaves
@@ -553,8 +606,9 @@ cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const int *qpo
   using C = Cfg<D, MT>;
   const long long rows = g.paged ? g.num_pages * g.hkv * g.page_size : (long long)g.batch * g.hkv * g.cap;
   const int boxh = g.paged ? min(g.page_size, KV_TILE) : KV_TILE;
-  CUtensorMap mk, mv;
-  if (!make_map(&mk, g.kc, rows, D, boxh) || !make_map(&mv, g.vc, rows, D, boxh))
+  CUtensorMap mk, mv, mk8, mv8;  // whole tiles; 8-row boxes for a unit's partial last tile
+  if (!make_map(&mk, g.kc, rows, D, boxh) || !make_map(&mv, g.vc, rows, D, boxh) ||
+      !make_map(&mk8, g.kc, rows, D, 8) || !make_map(&mv8, g.vc, rows, D, 8))
     return cudaErrorInvalidValue;
   // the rotated query rows: [units * MT * 128, D], boxes of 64 columns x 128 rows
   CUtensorMap mq;
@@ -569,7 +623,8 @@ cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const int *qpo
   auto kern = prefix_tc_kernel<D, MT>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(shares), dim3(C::THREADS), C::SMEM, st, g, q, ws, shares, mk, mv, boxh, mq);
+  return launch_pdl(kern, dim3(shares), dim3(C::THREADS), C::SMEM, st, g, q, ws, shares, mk, mv, mk8, mv8, boxh,
+                    mq);
 }
 
 }  // namespace
@@ -588,3 +643,12 @@ cudaError_t launch_prefix_tc(const Geometry &g, const __nv_bfloat16 *q, const Wo
 }
 
 }  // namespace fbk
+
+#ifdef FBK_TEST_HOOKS
+// Test build only: see include/fbk_test_hooks.h.
+extern "C" int fbk_test_set_wait_fault(long long wait_limit_clocks, int withhold_stage) {
+  cudaError_t e = cudaMemcpyToSymbol(fbk::tc::g_test_wait_limit, &wait_limit_clocks, sizeof(long long));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(fbk::tc::g_test_withhold_stage, &withhold_stage, sizeof(int));
+  return (int)e;
+}
+#endif

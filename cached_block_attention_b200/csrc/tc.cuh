@@ -14,6 +14,17 @@ namespace tc {
 // error shows up as a flag instead of a hung GPU.
 constexpr long long WAIT_LIMIT_CLOCKS = 2000000000ll;
 
+#ifdef FBK_TEST_HOOKS
+// Test build only (libfbk_testhooks.so, which the bounded-wait test loads):
+// the wait limit, and one K stage that block 0 leaves unloaded, are device
+// variables set by fbk_test_set_wait_fault. The library proper has neither.
+static __device__ long long g_test_wait_limit = WAIT_LIMIT_CLOCKS;
+static __device__ int g_test_withhold_stage = -1;
+__device__ __forceinline__ long long wait_limit() { return g_test_wait_limit; }
+#else
+__device__ __forceinline__ long long wait_limit() { return WAIT_LIMIT_CLOCKS; }
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
@@ -36,16 +47,18 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
                : "memory");
 }
 
-// One try: the thread may sleep in hardware (up to ~0.1 ms, the suspend-time
-// hint) until the phase completes, so waiting warps take no issue slots.
+// One try: the thread may sleep in hardware for a system-dependent time
+// until the phase completes, so waiting warps take few issue slots. (No
+// suspend-time hint: measured on B200, a two-warp mbarrier ping-pong takes
+// ~155 clocks per round trip this way against ~200 with a long hint.)
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(100000u)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -97,7 +110,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   while (true) {
     if (mbar_test(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > WAIT_LIMIT_CLOCKS) {
+    if (clock64() - t0 > wait_limit()) {
       *abort = 1;
       return false;
     }
@@ -216,6 +229,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
       "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]),
       "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 

@@ -203,8 +203,8 @@ fbk_status fbk_prefix_partial_at(const fbk_shape *shape, const void *q_blk, cons
 
 /* fbk_prefix_partial without a caller-supplied workspace. The pages have no
  * counterpart to this call: it is an interface convenience only, and it
- * computes exactly what fbk_prefix_partial computes, with the same two
- * kernels and the same results.
+ * computes exactly what fbk_prefix_partial computes, with the same kernels
+ * and the same results.
  *
  * Who it is for. Some callers cannot hand over scratch memory. Examples are a
  * plain C host with no device allocator of its own, or a plug-in inside another

@@ -18,8 +18,8 @@ def fbk():
     return m
 
 
-def declared_entry_points():
-    text = open(os.path.join(ROOT, "include", "fbk.h")).read()
+def declared_entry_points(header="fbk.h"):
+    text = open(os.path.join(ROOT, "include", header)).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(fbk_[a-z0-9_]+)\s*\(", text)))
 
@@ -30,6 +30,19 @@ def test_exports_every_declared_symbol(fbk):
     for n in names:
         assert hasattr(fbk.lib, n), n
     assert set(fbk.EXPORTS) == set(names)
+
+
+def test_test_build_exports_its_hook_and_the_library_does_not(fbk):
+    """libfbk_testhooks.so exports every fbk.h entry point plus the hook of
+    include/fbk_test_hooks.h; the library proper has no hook."""
+    from cached_block_attention_b200 import build
+    hooks = ctypes.CDLL(build.TEST_LIB)
+    hook_names = declared_entry_points("fbk_test_hooks.h")
+    assert hook_names == ["fbk_test_set_wait_fault"]
+    for n in declared_entry_points() + hook_names:
+        assert hasattr(hooks, n), n
+    for n in hook_names:
+        assert not hasattr(fbk.lib, n), n
 
 
 def test_status_strings(fbk):

@@ -412,3 +412,38 @@ def test_workload_parity_check_mode(name):
         full, _ = orc.full_attention(q, k, v, kp, vp, case.lens, case.hkv, 1.0, case.base)
         H.assert_close(H.host_f64(out), full, "fp32", f"{wl.name} step {s + 1} vs uncached")
     assert int(case.dev["cache"].error_flags.item()) == 0
+
+
+@pytest.mark.parametrize("mode,mname", MODES)
+@pytest.mark.parametrize("page_size", [0, 16, 64])
+def test_memory_past_the_prefix_is_never_read(page_size, mode, mname):
+    """Cache slots past each sequence's committed length hold NaN bit patterns
+    (a cache allocated without initialisation may hold anything there). The
+    prefix lengths are not multiples of 8, so the last tile of every unit is
+    partial: the state and the step output must still be finite and match the
+    oracle, which never looks past L_b."""
+    case = H.make_case(3, 8, 2, 128, 32, (77, 203, 1001), page_size, 1.0, seed=131, mode=mode,
+                       cap_extra=200).upload()
+    cache = case.dev["cache"]
+    nan = torch.tensor(0x7FC1, dtype=torch.int16).view(torch.bfloat16)
+    for bi, L in enumerate(case.lens):
+        if page_size:
+            table = cache.page_table[bi].cpu().numpy()
+            for lp, pid in enumerate(table):
+                if pid < 0:
+                    continue
+                lo = max(0, int(L) - lp * page_size)  # first unused slot of this page
+                if lo < page_size:
+                    cache.k[pid, :, lo:] = nan
+                    cache.v[pid, :, lo:] = nan
+        else:
+            cache.k[bi, :, int(L):] = nan
+            cache.v[bi, :, int(L):] = nan
+    pfx = H.run_prefix(case, case.dev["steps"][0][0])
+    got = H.partial_to_host(pfx)
+    assert np.isfinite(got[0]).all() and np.isfinite(got[2]).all()
+    ref = orc.prefix_partial(case.step_f64(0)[0], case.k_pfx(), case.v_pfx(), case.lens, case.hkv, 1.0, case.base)
+    H.check_partial(got, ref, mname, f"page {page_size}")
+    out, _ = H.run_step(case, pfx, 0)
+    H.assert_close(H.host_f64(out), oracle_full(case, 0)[0], mname, f"page {page_size} step")
+    assert int(cache.error_flags.item()) == 0
