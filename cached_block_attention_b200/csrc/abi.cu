@@ -224,12 +224,14 @@ fbk_status check_workspace(const fbk_shape *shape, int32_t num_splits, const voi
 // the fp32 share kernel), then the fixed-order split reduction. qpos: NULL, or
 // the rotation base of the block's rows per sequence.
 cudaError_t enqueue_prefix(const fbk_shape *shape, const Geometry &g, const void *q_blk, const Workspace &w,
-                           int shares, const fbk_partial &out, cudaStream_t s, const int *qpos = nullptr) {
+                           int shares, const fbk_partial &out, cudaStream_t s, const int *qpos = nullptr,
+                           const PrefixGate *gate = nullptr) {
   const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(q_blk);
-  cudaError_t e = shape->mode == FBK_BF16 ? launch_prefix_tc_at(g, q, qpos, w, shares, s)
+  if (gate && shape->mode != FBK_BF16) return cudaErrorInvalidValue;  // gated launches: bf16 path only
+  cudaError_t e = shape->mode == FBK_BF16 ? launch_prefix_tc_at(g, q, qpos, w, shares, s, gate)
                                           : launch_prefix_fp32_at(g, q, qpos, w, shares, s);
   if (e != cudaSuccess) return e;
-  return launch_split_reduce(g, w, shares, out, s);
+  return launch_split_reduce(g, w, shares, out, s, gate ? gate->gate : nullptr);
 }
 
 // Geometry of the step kernel: no cache, only the prefix lengths.
@@ -427,6 +429,78 @@ fbk_status fbk_decode_block(const fbk_shape *shape, const fbk_layer_block *layer
       float *lse = L.lse ? L.lse + step * lse_step : nullptr;
       if (enqueue_merge(shape, gm, q, at(L.k, step * kv_step * 2), at(L.v, step * kv_step * 2), L.prefix, out, lse,
                         s) != cudaSuccess)
+        return FBK_ERR_CUDA;
+    }
+  }
+  if (commit) {
+    for (int32_t l = 0; l < n_layers; ++l) {
+      const fbk_layer_block &L = layers[l];
+      const size_t last = (size_t)(steps - 1) * kv_step * 2;
+      if (enqueue_commit(geo[l], at(L.k, last), at(L.v, last), &L.cache, s) != cudaSuccess) return FBK_ERR_CUDA;
+    }
+  }
+  return FBK_OK;
+}
+
+fbk_status fbk_decode_block_adaptive(const fbk_shape *shape, const fbk_layer_block *layers, int32_t n_layers,
+                                     int32_t steps, int32_t commit, const fbk_drift_policy *policy, void *ws,
+                                     size_t ws_bytes, int32_t num_splits, void *cuda_stream) {
+  fbk_status st = check_shape(shape);
+  if (st != FBK_OK) return st;
+  if (!layers || n_layers < 1 || steps < 1 || num_splits < 0 || !policy) return FBK_ERR_INVALID_ARG;
+  if (shape->mode != FBK_BF16) return FBK_ERR_UNSUPPORTED;
+  if (!(policy->threshold >= 0.f) || !policy->flags || !policy->last_refresh || !policy->drift ||
+      !policy->refreshed)  // (a NaN threshold fails the first test)
+    return FBK_ERR_INVALID_ARG;
+  if ((long long)n_layers * steps > 0x7fffffffll) return FBK_ERR_CAPACITY;
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const fbk_layer_block &L = layers[l];
+    if ((st = check_cache(shape, &L.cache)) != FBK_OK) return st;
+    if ((st = check_prefix_ptrs(L.q, &L.prefix)) != FBK_OK) return st;
+    if ((st = check_merge_ptrs(L.q, L.k, L.v, L.cache.prefix_lens, &L.prefix, L.out)) != FBK_OK) return st;
+    if (commit) {
+      for (int32_t j = 0; j < l; ++j)
+        if (layers[j].cache.prefix_lens == L.cache.prefix_lens) return FBK_ERR_INVALID_ARG;
+    }
+  }
+  const size_t b = shape->batch, B = shape->block_len, d = shape->head_dim;
+  const size_t q_step = b * B * shape->n_q_heads * d, kv_step = b * B * shape->n_kv_heads * d;
+  const size_t out_step_bytes = q_step * 2;
+  const size_t lse_step = b * shape->n_q_heads * B;
+  if ((size_t)steps > ((size_t)1 << 62) / (out_step_bytes * 2)) return FBK_ERR_CAPACITY;
+  int shares;
+  WsLayout lay;
+  if ((st = check_workspace(shape, num_splits, ws, ws_bytes, &shares, &lay)) != FBK_OK) return st;
+  const Workspace w = carve(lay, ws);
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  std::vector<Geometry> geo(n_layers);
+  for (int32_t l = 0; l < n_layers; ++l) geo[l] = make_geometry(shape, &layers[l].cache);
+  Geometry gm = make_geometry(shape, nullptr);
+  auto at = [](const void *p, size_t bytes) { return static_cast<const char *>(p) + bytes; };
+  int32_t *flags = policy->flags;  // [2][n_layers]: requests for even and odd steps
+
+  if (launch_adaptive_init(flags, policy->last_refresh, policy->drift, policy->refreshed, n_layers, steps, s) !=
+      cudaSuccess)
+    return FBK_ERR_CUDA;
+  for (int32_t step = 0; step < steps; ++step) {
+    int32_t *cur = flags + (step & 1) * n_layers, *nxt = flags + ((step + 1) & 1) * n_layers;
+    for (int32_t l = 0; l < n_layers; ++l) {
+      const fbk_layer_block &L = layers[l];
+      const void *q = at(L.q, step * q_step * 2);
+      const size_t cell = (size_t)step * n_layers + l;
+      const PrefixGate gate{cur + l, policy->refreshed + cell, policy->last_refresh + l, step};
+      if (enqueue_prefix(shape, geo[l], q, w, shares, L.prefix, s, nullptr, &gate) != cudaSuccess)
+        return FBK_ERR_CUDA;
+      const DriftArgs dr{static_cast<const __nv_bfloat16 *>(L.q), (long long)q_step, policy->last_refresh + l,
+                         step + 1 < steps ? step + 1 : -1, cur + l, nxt + l, n_layers - l, policy->threshold,
+                         policy->drift + cell};
+      gm.lens = L.cache.prefix_lens;
+      void *out = static_cast<char *>(L.out) + step * out_step_bytes;
+      float *lse = L.lse ? L.lse + step * lse_step : nullptr;
+      if (launch_block_merge(gm, static_cast<const __nv_bfloat16 *>(q),
+                             reinterpret_cast<const __nv_bfloat16 *>(at(L.k, step * kv_step * 2)),
+                             reinterpret_cast<const __nv_bfloat16 *>(at(L.v, step * kv_step * 2)), L.prefix, out, lse,
+                             false, s, &dr) != cudaSuccess)
         return FBK_ERR_CUDA;
     }
   }

@@ -75,8 +75,8 @@ constexpr int STEP_ROWS = 16;  // query rows of one row tile: one m16 MMA tile
 template <int D, int WPT, int RT>
 struct StepLayout {  // byte offsets in shared memory, all 16-byte aligned
   static constexpr int RS = D * 2 + 16;  // padded bf16 row: the 8 rows of an ldmatrix hit distinct banks
-  int bpad, ps_stride, ks, vs, qs, ps, red, cs, bytes;
-  __host__ __device__ StepLayout(int blk) {
+  int bpad, ps_stride, ks, vs, qs, ps, red, cs, dq, dc, bytes;
+  __host__ __device__ StepLayout(int blk, bool drift = false) {
     bpad = (blk + 15) & ~15;
     ps_stride = bpad * 2 + 16;
     ks = 0;
@@ -85,7 +85,11 @@ struct StepLayout {  // byte offsets in shared memory, all 16-byte aligned
     ps = qs + RT * STEP_ROWS * RS;
     red = ps + (WPT > 1 ? RT * STEP_ROWS * ps_stride : 0);     // P~ of each row tile (bf16)
     cs = red + (WPT > 1 ? 2 * RT * WPT * STEP_ROWS * 4 : 0);   // [2][RT][WPT][16] fp32 max, sum
-    bytes = cs + blk * (D / 2) * 8;                           // [blk][D/2] (cos, sin)
+    dq = cs + blk * (D / 2) * 8;                              // [blk][D/2] (cos, sin)
+    // adaptive refresh only: the query rows of the next step and of the
+    // state's step ([2][rows][RS]), then 1 - cos per row (fp32)
+    dc = dq + (drift ? 2 * RT * STEP_ROWS * RS : 0);
+    bytes = dc + (drift ? RT * STEP_ROWS * 4 : 0);
   }
 };
 
@@ -113,7 +117,7 @@ template <int D, int WPT, int RT>
 __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
     Geometry g, const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kb,
     const __nv_bfloat16 *__restrict__ vb, fbk_partial pfx, __nv_bfloat16 *__restrict__ out,
-    float *__restrict__ lse, int tiles) {
+    float *__restrict__ lse, int tiles, DriftArgs dr) {
   using L = StepLayout<D, WPT, RT>;
   constexpr int CTA_ROWS = RT * STEP_ROWS, NTHREADS = RT * WPT * 32;
   constexpr int HALF = D / 2, CH = D / 8, RS = L::RS;
@@ -121,7 +125,8 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
   extern __shared__ float4 smem_f4[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(smem_f4);
   const int blk = g.blk;
-  const L lay(blk);
+  const bool drift = dr.q_base != nullptr && dr.next_step >= 0;
+  const L lay(blk, dr.q_base != nullptr);
   const int bpad = lay.bpad, NT = bpad / 8, PSS = lay.ps_stride;
   uint8_t *Ks = sm + lay.ks, *Vs = sm + lay.vs, *Qs = sm + lay.qs, *Ps = sm + lay.ps;
   float *red_max = reinterpret_cast<float *>(sm + lay.red);
@@ -151,6 +156,7 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
   }
   pdl_wait();
   pdl_release();
+  if (dr.clear && blockIdx.x == 0 && tid == 0) *dr.clear = 0;  // this step's refresh request is used up
 
   // ---- 1. every global read of the CTA, issued at once
   const long long kv_row0 = (long long)b * blk * g.hkv + kvh;  // token t: row kv_row0 + t*hkv
@@ -164,6 +170,17 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
     const int rr = idx / CH, c = idx % CH, r = r0 + rr;
     const int t = r % blk, h = kvh * g.group + r / blk;
     cp_async16(Qs + rr * RS + c * 16, q + (((long long)b * blk + t) * g.hq + h) * D + c * 8);
+  }
+  if (drift) {  // the rows of the next step's queries and of the state's queries
+    const __nv_bfloat16 *qn = dr.q_base + (long long)dr.next_step * dr.q_stride;
+    const __nv_bfloat16 *qr = dr.q_base + (long long)(*dr.last_refresh) * dr.q_stride;
+    for (int idx = tid; idx < rows_cta * CH; idx += NTHREADS) {
+      const int rr = idx / CH, c = idx % CH, r = r0 + rr;
+      const int t = r % blk, h = kvh * g.group + r / blk;
+      const long long off = (((long long)b * blk + t) * g.hq + h) * D + c * 8;
+      cp_async16(sm + lay.dq + rr * RS + c * 16, qn + off);
+      cp_async16(sm + lay.dq + (CTA_ROWS + rr) * RS + c * 16, qr + off);
+    }
   }
   // padding key rows and query rows must be finite zeros
   for (int idx = tid; idx < (bpad - blk) * CH; idx += NTHREADS) {
@@ -195,6 +212,39 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
   if (vbr) { m1b = __ldg(pfx.m + pb); l1b = __ldg(pfx.l + pb); }
   cp_async_wait_all();
   __syncthreads();
+
+  if (drift) {
+    // 1 - cos between the next step's and the state's query row, as
+    // |q/|q| - r/|r||^2 / 2 (exactly 0 for equal rows; 0 if a row is zero):
+    // one warp per row, lanes over the columns
+    float *dcos = reinterpret_cast<float *>(sm + lay.dc);
+    for (int rr = tid >> 5; rr < rows_cta; rr += NTHREADS / 32) {
+      const uint8_t *rq = sm + lay.dq + rr * RS, *rf = sm + lay.dq + (CTA_ROWS + rr) * RS;
+      float x[D / 32], y[D / 32], nx = 0.f, ny = 0.f;
+#pragma unroll
+      for (int e = 0; e < D / 32; ++e) {
+        const int col = lane + 32 * e;
+        x[e] = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(rq)[col]);
+        y[e] = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(rf)[col]);
+        nx += x[e] * x[e];
+        ny += y[e] * y[e];
+      }
+      nx = warp_sum(nx);
+      ny = warp_sum(ny);
+      float dd = 0.f;
+      if (nx > 0.f && ny > 0.f) {
+        const float ix = rsqrtf(nx), iy = rsqrtf(ny);
+#pragma unroll
+        for (int e = 0; e < D / 32; ++e) {
+          // rounded products (no fused multiply-add), so equal rows give exactly 0
+          const float t = __fsub_rn(__fmul_rn(x[e], ix), __fmul_rn(y[e], iy));
+          dd += t * t;
+        }
+      }
+      dd = warp_sum(dd);
+      if (lane == 0) dcos[rr] = 0.5f * dd;
+    }
+  }
 
   // ---- 2. rotate block K and the query rows in place at their block offsets, 8 pairs per item
   for (int idx = tid; idx < (blk + rows_cta) * (D / 16); idx += NTHREADS) {
@@ -413,13 +463,27 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
     if (va) lse[pa] = Ma + logf(lta);
     if (vbr) lse[pb] = Mb + logf(ltb);
   }
+  if (drift) {
+    // drift statistic: the prefix's share of the row's softmax mass times the
+    // row's 1 - cos; the maximum over the CTA's rows, then over the grid
+    const float *dcos = reinterpret_cast<const float *>(sm + lay.dc);
+    float dm = 0.f;
+    if (va) dm = fmaxf(dm, w1a * l1a / lta * dcos[tr0 + lr]);
+    if (vbr) dm = fmaxf(dm, w1b * l1b / ltb * dcos[tr0 + lr + 8]);
+    dm = warp_max(dm);
+    if (lane == 0 && dm > 0.f) {
+      atomicMax(reinterpret_cast<int *>(dr.drift_out), __float_as_int(dm));  // non-negative floats order as ints
+      if (dm > dr.theta)
+        for (int j = 0; j < dr.n_next; ++j) dr.next_flags[j] = 1;  // this layer and every deeper one
+    }
+  }
 }
 
 template <int D, int WPT, int RT>
 cudaError_t launch_mma_cfg(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
                            const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
-                           cudaStream_t st) {
-  const StepLayout<D, WPT, RT> lay(g.blk);
+                           cudaStream_t st, const DriftArgs &da) {
+  const StepLayout<D, WPT, RT> lay(g.blk, da.q_base != nullptr);
   auto kern = block_merge_mma_kernel<D, WPT, RT>;
   if (lay.bytes > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.bytes);
@@ -429,7 +493,7 @@ cudaError_t launch_mma_cfg(const Geometry &g, const __nv_bfloat16 *q, const __nv
   const long long ctas = (long long)g.batch * g.hkv * tiles;
   if (ctas > 0x7fffffffll) return cudaErrorInvalidConfiguration;
   return launch_pdl(kern, dim3((unsigned)ctas), dim3(RT * WPT * 32), lay.bytes, st, g, q, kb, vb, pfx,
-                    static_cast<__nv_bfloat16 *>(out), lse, tiles);
+                    static_cast<__nv_bfloat16 *>(out), lse, tiles, da);
 }
 
 // Layout choice from the number of 16-row tiles n = units * ceil(G*B / 16),
@@ -441,18 +505,18 @@ cudaError_t launch_mma_cfg(const Geometry &g, const __nv_bfloat16 *q, const __nv
 template <int D>
 cudaError_t launch_mma(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfloat16 *kb,
                        const __nv_bfloat16 *vb, const fbk_partial &pfx, void *out, float *lse,
-                       cudaStream_t st) {
+                       cudaStream_t st, const DriftArgs &da) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long units = (long long)g.batch * g.hkv, t16 = (g.rows + STEP_ROWS - 1) / STEP_ROWS;
-  if (units * t16 >= 4ll * sms) return launch_mma_cfg<D, 1, 4>(g, q, kb, vb, pfx, out, lse, st);
+  if (units * t16 >= 4ll * sms) return launch_mma_cfg<D, 1, 4>(g, q, kb, vb, pfx, out, lse, st, da);
   int rt = 1;
   for (int c = 4; c > 1; c >>= 1)
     if (c <= t16 && units * ((t16 + c - 1) / c) * 20 >= 17ll * sms) { rt = c; break; }
   switch (rt) {
-    case 4: return launch_mma_cfg<D, 4, 4>(g, q, kb, vb, pfx, out, lse, st);
-    case 2: return launch_mma_cfg<D, 4, 2>(g, q, kb, vb, pfx, out, lse, st);
-    default: return launch_mma_cfg<D, 4, 1>(g, q, kb, vb, pfx, out, lse, st);
+    case 4: return launch_mma_cfg<D, 4, 4>(g, q, kb, vb, pfx, out, lse, st, da);
+    case 2: return launch_mma_cfg<D, 4, 2>(g, q, kb, vb, pfx, out, lse, st, da);
+    default: return launch_mma_cfg<D, 4, 1>(g, q, kb, vb, pfx, out, lse, st, da);
   }
 }
 
@@ -648,12 +712,15 @@ cudaError_t launch_f32(const Geometry &g, const __nv_bfloat16 *q, const __nv_bfl
 cudaError_t launch_block_merge(const Geometry &g, const __nv_bfloat16 *q,
                                const __nv_bfloat16 *kb, const __nv_bfloat16 *vb,
                                const fbk_partial &pfx, void *out, float *lse, bool f32_out,
-                               cudaStream_t st) {
-  if (f32_out)
+                               cudaStream_t st, const DriftArgs *drift) {
+  if (f32_out) {
+    if (drift) return cudaErrorInvalidValue;  // the adaptive refresh runs on the bf16 path
     return g.d == 128 ? launch_f32<128>(g, q, kb, vb, pfx, out, lse, st)
                       : launch_f32<64>(g, q, kb, vb, pfx, out, lse, st);
-  return g.d == 128 ? launch_mma<128>(g, q, kb, vb, pfx, out, lse, st)
-                    : launch_mma<64>(g, q, kb, vb, pfx, out, lse, st);
+  }
+  const DriftArgs da = drift ? *drift : DriftArgs{nullptr, 0, nullptr, -1, nullptr, nullptr, 0, 0.f, nullptr};
+  return g.d == 128 ? launch_mma<128>(g, q, kb, vb, pfx, out, lse, st, da)
+                    : launch_mma<64>(g, q, kb, vb, pfx, out, lse, st, da);
 }
 
 }  // namespace fbk

@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
                      const Workspace ws, const int shares, const __grid_constant__ CUtensorMap tmk,
                      const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmk8,
                      const __grid_constant__ CUtensorMap tmv8, const int boxh,
-                     const __grid_constant__ CUtensorMap tmq) {
+                     const __grid_constant__ CUtensorMap tmq, const int *gate) {
   using C = Cfg<D, MT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -192,6 +192,13 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
   }
   pdl_wait();
   pdl_release();
+  if (gate && *gate == 0) {  // no refresh of this state at this step (the same for every thread)
+    fence_before_sync();
+    __syncthreads();  // the allocation's address is in shared memory
+    fence_after_sync();
+    if (warp == 1) tmem_dealloc(*tmem_slot, C::TMEM_COLS);  // nothing was issued on it
+    return;
+  }
   fence_before_sync();
   const long long T = load_tile_scan(g, s_len, s_scan);  // reads prefix_lens; two CTA barriers
   fence_after_sync();
@@ -535,13 +542,21 @@ __global__ void __launch_bounds__(Cfg<D, MT>::THREADS, 1)
 // G*B are zero. One thread per 8 rotation pairs (chunk c of each half of a row).
 template <int D, int MT>
 __global__ void __launch_bounds__(256) rope_q_kernel(Geometry g, const __nv_bfloat16 *__restrict__ q,
-                                                    __nv_bfloat16 *__restrict__ qrot, const int *__restrict__ qpos) {
+                                                    __nv_bfloat16 *__restrict__ qrot, const int *__restrict__ qpos,
+                                                    PrefixGate gate) {
   constexpr int HALF = D / 2, KI = D / 16, ROWS = MT * 128;
   __shared__ double theta[HALF];
   for (int i = threadIdx.x; i < HALF; i += blockDim.x) theta[i] = freq_over_pi(i, D, g.log2_base);
   __syncthreads();
   pdl_wait();
   pdl_release();
+  if (gate.gate) {  // the adaptive refresh: run only when asked, and record that it ran
+    if (*gate.gate == 0) return;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      *gate.mark = 1;
+      *gate.last = gate.step;
+    }
+  }
   const long long n_items = (long long)g.batch * g.hkv * ROWS * KI;
   for (long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x; item < n_items;
        item += (long long)gridDim.x * blockDim.x) {
@@ -602,7 +617,8 @@ bool make_map(CUtensorMap *m, const void *base, long long rows, int d, int boxh)
 
 template <int D, int MT>
 cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const int *qpos, const Workspace &ws, int shares,
-                       cudaStream_t st) {
+                       cudaStream_t st, const PrefixGate *pg) {
+  const PrefixGate gate = pg ? *pg : PrefixGate{nullptr, nullptr, nullptr, 0};
   using C = Cfg<D, MT>;
   const long long rows = g.paged ? g.num_pages * g.hkv * g.page_size : (long long)g.batch * g.hkv * g.cap;
   const int boxh = g.paged ? min(g.page_size, KV_TILE) : KV_TILE;
@@ -618,23 +634,49 @@ cudaError_t launch_cfg(const Geometry &g, const __nv_bfloat16 *q, const int *qpo
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long items = qrows * (D / 16);
   const int rq_ctas = (int)std::min<long long>((items + 255) / 256, 8ll * sms);
-  cudaError_t e = launch_pdl(rope_q_kernel<D, MT>, dim3(rq_ctas), dim3(256), 0, st, g, q, ws.qrot, qpos);
+  cudaError_t e = launch_pdl(rope_q_kernel<D, MT>, dim3(rq_ctas), dim3(256), 0, st, g, q, ws.qrot, qpos, gate);
   if (e != cudaSuccess) return e;
   auto kern = prefix_tc_kernel<D, MT>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(shares), dim3(C::THREADS), C::SMEM, st, g, q, ws, shares, mk, mv, mk8, mv8, boxh,
-                    mq);
+                    mq, gate.gate);
 }
 
 }  // namespace
 
 cudaError_t launch_prefix_tc_at(const Geometry &g, const __nv_bfloat16 *q, const int *qpos, const Workspace &ws,
-                                int shares, cudaStream_t st) {
+                                int shares, cudaStream_t st, const PrefixGate *gate) {
   const bool two = g.rows > 128;
   if (g.d == 128)
-    return two ? launch_cfg<128, 2>(g, q, qpos, ws, shares, st) : launch_cfg<128, 1>(g, q, qpos, ws, shares, st);
-  return two ? launch_cfg<64, 2>(g, q, qpos, ws, shares, st) : launch_cfg<64, 1>(g, q, qpos, ws, shares, st);
+    return two ? launch_cfg<128, 2>(g, q, qpos, ws, shares, st, gate)
+               : launch_cfg<128, 1>(g, q, qpos, ws, shares, st, gate);
+  return two ? launch_cfg<64, 2>(g, q, qpos, ws, shares, st, gate)
+             : launch_cfg<64, 1>(g, q, qpos, ws, shares, st, gate);
+}
+
+namespace {
+__global__ void adaptive_init_kernel(int *flags, int *last_refresh, float *drift, int *refreshed, int n, int steps) {
+  pdl_wait();
+  pdl_release();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < steps * n; i += gridDim.x * blockDim.x) {
+    drift[i] = 0.f;
+    refreshed[i] = 0;
+    if (i < n) {
+      flags[i] = 1;      // step 0 computes every layer's state
+      flags[n + i] = 0;  // no request for step 1 yet
+      last_refresh[i] = 0;
+    }
+  }
+}
+}  // namespace
+
+cudaError_t launch_adaptive_init(int *flags, int *last_refresh, float *drift, int *refreshed, int n_layers,
+                                 int steps, cudaStream_t st) {
+  const long long items = (long long)n_layers * steps;
+  const int ctas = (int)std::min<long long>((items + 255) / 256, 1024);
+  return launch_pdl(adaptive_init_kernel, dim3(ctas), dim3(256), 0, st, flags, last_refresh, drift, refreshed,
+                    n_layers, steps);
 }
 
 cudaError_t launch_prefix_tc(const Geometry &g, const __nv_bfloat16 *q, const Workspace &ws,

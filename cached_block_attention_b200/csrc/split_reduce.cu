@@ -21,7 +21,7 @@ constexpr int NCH = 8;            // pieces whose O~ rows are in flight at once
 
 template <int D, int ROWS_PER_WARP>
 __global__ void __launch_bounds__(WARPS * 32) split_reduce_kernel(Geometry g, Workspace ws, int shares,
-                                                                 fbk_partial out) {
+                                                                 fbk_partial out, const int *gate) {
   constexpr int CPL = D / 32, CTA_ROWS = WARPS * ROWS_PER_WARP;
   const int u = blockIdx.x, b = u / g.hkv, kvh = u % g.hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(WARPS * 32) split_reduce_kernel(Geometry g, Wo
   __shared__ int s_n;
   pdl_wait();
   pdl_release();
+  if (gate && *gate == 0) return;  // no refresh of this state at this step
 
   // list positions before sequence b and in total: parallel loads, block reduction
   long long before = 0, T = 0;
@@ -166,20 +167,21 @@ __global__ void __launch_bounds__(WARPS * 32) split_reduce_kernel(Geometry g, Wo
 // shorter chains).
 template <int D, int RPW>
 cudaError_t launch_rpw(const Geometry &g, const Workspace &ws, int shares, const fbk_partial &out,
-                       cudaStream_t st) {
+                       cudaStream_t st, const int *gate) {
   dim3 grid(g.batch * g.hkv, (g.rows + WARPS * RPW - 1) / (WARPS * RPW));
-  return launch_pdl(split_reduce_kernel<D, RPW>, grid, dim3(WARPS * 32), 0, st, g, ws, shares, out);
+  return launch_pdl(split_reduce_kernel<D, RPW>, grid, dim3(WARPS * 32), 0, st, g, ws, shares, out, gate);
 }
 
 }  // namespace
 
 cudaError_t launch_split_reduce(const Geometry &g, const Workspace &ws, int shares,
-                                const fbk_partial &out, cudaStream_t st) {
+                                const fbk_partial &out, cudaStream_t st, const int *gate) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const bool four = (long long)g.batch * g.hkv * g.rows >= 4ll * WARPS * sms;
-  if (g.d == 128) return four ? launch_rpw<128, 4>(g, ws, shares, out, st) : launch_rpw<128, 1>(g, ws, shares, out, st);
-  return four ? launch_rpw<64, 4>(g, ws, shares, out, st) : launch_rpw<64, 1>(g, ws, shares, out, st);
+  if (g.d == 128)
+    return four ? launch_rpw<128, 4>(g, ws, shares, out, st, gate) : launch_rpw<128, 1>(g, ws, shares, out, st, gate);
+  return four ? launch_rpw<64, 4>(g, ws, shares, out, st, gate) : launch_rpw<64, 1>(g, ws, shares, out, st, gate);
 }
 
 }  // namespace fbk

@@ -36,7 +36,8 @@ EXPORTS = ("fbk_prefix_workspace_bytes", "fbk_default_num_splits", "fbk_prefix_p
            "fbk_status_string", "fbk_prefix_partial_static_scratch", "fbk_decode_block",
            "fbk_fp8_group_quant", "fbk_facache_unchanged_rows", "fbk_prefix_partial_at",
            "fbk_facache_workspace_bytes", "fbk_facache_refresh", "fbk_facache_step", "fbk_page_means",
-           "fbk_select_pages_workspace_bytes", "fbk_select_pages", "fbk_residual_capture", "fbk_residual_apply")
+           "fbk_select_pages_workspace_bytes", "fbk_select_pages", "fbk_residual_capture", "fbk_residual_apply",
+           "fbk_decode_block_adaptive")
 
 STATIC_SCRATCH_BYTES = 32 << 20  # FBK_STATIC_SCRATCH_BYTES
 
@@ -87,6 +88,17 @@ _lib.fbk_prefix_partial_static_scratch.restype = ctypes.c_int
 _lib.fbk_decode_block.argtypes = [_P(_Shape), _P(_LayerBlock), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                   _vp, ctypes.c_size_t, ctypes.c_int32, _vp]
 _lib.fbk_decode_block.restype = ctypes.c_int
+
+
+class _DriftPolicy(ctypes.Structure):
+    _fields_ = [("threshold", ctypes.c_float), ("flags", ctypes.c_void_p), ("last_refresh", ctypes.c_void_p),
+                ("drift", ctypes.c_void_p), ("refreshed", ctypes.c_void_p)]
+
+
+_lib.fbk_decode_block_adaptive.argtypes = [_P(_Shape), _P(_LayerBlock), ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_int32, _P(_DriftPolicy), _vp, ctypes.c_size_t, ctypes.c_int32,
+                                           _vp]
+_lib.fbk_decode_block_adaptive.restype = ctypes.c_int
 _lib.fbk_fp8_group_quant.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
 _lib.fbk_fp8_group_quant.restype = ctypes.c_int
 _lib.fbk_facache_unchanged_rows.argtypes = [_P(_Shape), ctypes.c_int32, _vp, _P(_Partial), _vp, _vp, _vp, _vp,
@@ -298,6 +310,44 @@ def decode_block(shape: Shape, layers, ws: torch.Tensor, commit: bool = True, nu
            "fbk_decode_block")
 
 
+@dataclass
+class DriftPolicy:
+    """fbk_drift_policy: threshold and the device arrays (int32 flags [2, n_layers]
+    and last_refresh [n_layers] scratch; fp32 drift and int32 refreshed
+    [steps, n_layers] outputs)."""
+    threshold: float
+    flags: torch.Tensor
+    last_refresh: torch.Tensor
+    drift: torch.Tensor
+    refreshed: torch.Tensor
+
+    @staticmethod
+    def empty(threshold: float, n_layers: int, steps: int, device="cuda") -> "DriftPolicy":
+        i32 = dict(dtype=torch.int32, device=device)
+        return DriftPolicy(threshold, torch.empty(2, n_layers, **i32), torch.empty(n_layers, **i32),
+                           torch.empty(steps, n_layers, dtype=torch.float32, device=device),
+                           torch.empty(steps, n_layers, **i32))
+
+    def c(self) -> _DriftPolicy:
+        return _DriftPolicy(self.threshold, self.flags.data_ptr(), self.last_refresh.data_ptr(),
+                            self.drift.data_ptr(), self.refreshed.data_ptr())
+
+
+def decode_block_adaptive(shape: Shape, layers, policy: DriftPolicy, ws: torch.Tensor, commit: bool = True,
+                          num_splits: int = 0, stream=None) -> None:
+    """decode_block with the drift-triggered, depth-aware refresh of
+    fbk_decode_block_adaptive (the layers' refresh_interval is ignored)."""
+    steps = {int(L.q.shape[0]) for L in layers}
+    if len(steps) != 1:
+        raise ValueError(f"layers disagree on the number of steps: {sorted(steps)}")
+    arr = (_LayerBlock * len(layers))(*[L.c() for L in layers])
+    cs, cp = shape.c(), policy.c()
+    _check(_lib.fbk_decode_block_adaptive(ctypes.byref(cs), arr, len(layers), steps.pop(), 1 if commit else 0,
+                                          ctypes.byref(cp), _ptr(ws), ws.numel() * ws.element_size(), num_splits,
+                                          _stream(stream)),
+           "fbk_decode_block_adaptive")
+
+
 FP8_GROUP = 128  # FBK_FP8_GROUP
 
 
@@ -380,3 +430,4 @@ def residual_apply(shape: Shape, sparse: Partial, r_o, r_lse, ext: Partial, stre
 # raw handles for tests of the C ABI itself
 lib = _lib
 CShape, CCache, CPartial, CLayerBlock = _Shape, _Cache, _Partial, _LayerBlock
+CDriftPolicy = _DriftPolicy

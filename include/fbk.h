@@ -295,6 +295,51 @@ fbk_status fbk_decode_block(const fbk_shape *shape, const fbk_layer_block *layer
                             int32_t steps, int32_t commit, void *ws, size_t ws_bytes,
                             int32_t num_splits, void *cuda_stream);
 
+/* Scratch and outputs of fbk_decode_block_adaptive, all device memory owned
+ * by the caller; the call initialises every array itself.
+ *  threshold:    theta >= 0 (may be +inf; FBK_ERR_INVALID_ARG for NaN or < 0).
+ *  flags:        int32 [2, n_layers] scratch: refresh requests for the even
+ *                and the odd steps.
+ *  last_refresh: int32 [n_layers] scratch: each layer's last refresh step.
+ *  drift:        fp32 [steps, n_layers] out: delta_s of every layer-step (the
+ *                last step's row is 0: it decides nothing).
+ *  refreshed:    int32 [steps, n_layers] out: 1 where the layer recomputed its
+ *                prefix state at that step. */
+typedef struct fbk_drift_policy {
+  float threshold;
+  int32_t *flags;
+  int32_t *last_refresh;
+  float *drift;
+  int32_t *refreshed;
+} fbk_drift_policy;
+
+/* fbk_decode_block with an adaptive, depth-aware refresh in place of the
+ * fixed intervals (Elastic-Cache, Abstract: an attention-aware drift test
+ * decides when to refresh, and the refresh recomputes from the triggering
+ * layer onward; the rule below is this library's reading of it). The layers'
+ * refresh_interval fields are ignored.
+ *
+ * Step 0 computes every layer's prefix state. At every step s < steps - 1 the
+ * step kernel of layer l computes
+ *   delta_s = max over the block's query rows of
+ *             pi_ext * (1 - cos(q_{s+1}, q_ref)),
+ * pi_ext the share of the row's softmax mass on the prefix at step s, q_{s+1}
+ * the row's pre-RoPE queries of step s + 1 (in the layer's step-major q) and
+ * q_ref those of the step the layer's state was computed from; 1 - cos is
+ * |q/|q| - r/|r||^2 / 2 (0 for equal rows and for zero rows). When
+ * delta_s > threshold, layer l and every deeper layer recompute their state at
+ * step s + 1. threshold = 0 refreshes every layer whose next queries differ
+ * from its state's; threshold = +inf is FlashBlock's reuse of step 0's state.
+ *
+ * The decisions are taken on the device, so the whole block is still only
+ * enqueued (one CUDA graph can hold it): every layer-step enqueues the prefix
+ * launches, which return at once when no refresh is due. FBK_BF16 mode only
+ * (FBK_ERR_UNSUPPORTED otherwise). Other arguments and errors as for
+ * fbk_decode_block. */
+fbk_status fbk_decode_block_adaptive(const fbk_shape *shape, const fbk_layer_block *layers, int32_t n_layers,
+                                     int32_t steps, int32_t commit, const fbk_drift_policy *policy, void *ws,
+                                     size_t ws_bytes, int32_t num_splits, void *cuda_stream);
+
 /* Elements per quantisation group of fbk_fp8_group_quant (1 x 128). */
 #define FBK_FP8_GROUP 128
 

@@ -197,6 +197,30 @@ def test_decode_block_argument_checks(fbk):
     assert _decode(fbk, ok, ws=0x100010, ws_bytes=n) == -2          # workspace not 256-byte aligned
 
 
+def test_decode_block_adaptive_argument_checks(fbk):
+    """fbk_decode_block_adaptive: the policy is checked with the layers, before
+    any launch; a missing workspace (-4) is the last check."""
+    ok = [_layer(fbk, lens=0x30000), _layer(fbk, lens=0x31000, interval=0)]  # intervals are ignored
+    pol = fbk.CDriftPolicy(0.1, 0x80000, 0x81000, 0x82000, 0x83000)
+
+    def call(layers=ok, policy=pol, steps=4, shape=None):
+        s = shape or _shape(fbk)
+        arr = (fbk.CLayerBlock * max(1, len(layers)))(*layers)
+        return fbk.lib.fbk_decode_block_adaptive(ctypes.byref(s), arr if layers else None, len(layers), steps, 1,
+                                                 ctypes.byref(policy) if policy else None, None, 0, 4, None)
+
+    assert call() == -4
+    assert call(policy=None) == -1
+    assert call(layers=[]) == -1
+    assert call(steps=0) == -1
+    for theta in (-1.0, float("nan")):
+        assert call(policy=fbk.CDriftPolicy(theta, 0x80000, 0x81000, 0x82000, 0x83000)) == -1
+    assert call(policy=fbk.CDriftPolicy(float("inf"), 0x80000, 0x81000, 0x82000, 0x83000)) == -4
+    assert call(policy=fbk.CDriftPolicy(0.1, None, 0x81000, 0x82000, 0x83000)) == -1
+    assert call(policy=fbk.CDriftPolicy(0.1, 0x80000, 0x81000, 0x82000, None)) == -1
+    assert call(shape=_shape(fbk, mode=1)) == -2  # the adaptive refresh runs on the bf16 path
+
+
 def test_fp8_group_quant_argument_checks(fbk):
     """Host checks of fbk_fp8_group_quant; none of these reach a CUDA call."""
     q = fbk.lib.fbk_fp8_group_quant
