@@ -42,12 +42,19 @@ def parse():
     ap.add_argument("--workload", default="long131k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="attention", choices=["attention", "fp8_group_quant", "facache_rows"],
+    ap.add_argument("--keep", type=float, default=0.125,
+                    help="--op sparse_prefix: fraction of each sequence's prefix pages kept (top-k)")
+    ap.add_argument("--op", default="attention",
+                    choices=["attention", "fp8_group_quant", "facache_rows", "sparse_prefix"],
                     help="attention: the cached block attention block (default); fp8_group_quant: the "
                          "per-group FP8 activation quantisation on the FP8_WORKLOADS shapes; facache_rows: "
                          "the FACache step of a whole sequence's unchanged rows (FACACHE_WORKLOADS)")
     ap.add_argument("--layers", type=int, default=1,
                     help="attention layers per block; > 1 runs the whole block through fbk_decode_block")
+    ap.add_argument("--adaptive", default="",
+                    help="with --layers: comma-separated drift thresholds; each is also timed through "
+                         "fbk_decode_block_adaptive (drift-triggered, depth-aware refresh) and reported in "
+                         "adaptive_sweep")
     ap.add_argument("--refresh-interval", default="",
                     help="cache update interval(s) for --layers, comma-separated; the first is the "
                          "reported value, every one is timed and its error against interval 1 reported "
@@ -755,6 +762,42 @@ def run_layers(args, wl, rank, world, local):
         ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
         sweep.append({"refresh_interval": r, "value": S / (ms * 1e-3), "unit": "denoising steps/s",
                       "ms_per_block": ms, "refreshes_per_layer": -(-S // r), **acc[r]})
+    # the adaptive refresh: one graph per threshold (the decisions are taken on
+    # the device, so the block stays one graph); refreshes and accuracy from a
+    # run of the same block
+    adaptive = []
+    thetas = [float(x) for x in args.adaptive.split(",")] if args.adaptive else []
+    for theta in thetas:
+        pol = fbk.DriftPolicy.empty(theta, N, S, dev)
+
+        def run_adaptive(pol=pol):
+            lens.copy_(lens0)
+            fbk.decode_block_adaptive(shape, blocks_for(1), pol, ws, commit=True)
+
+        run_adaptive()
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+        n_refresh = int(pol.refreshed.sum())
+        dmax = float(pol.drift.max())
+        run_block(1)
+        torch.cuda.synchronize()
+        exact = torch.stack(outs).float()
+        run_adaptive()
+        torch.cuda.synchronize()
+        diff = torch.stack(outs).float() - exact
+        ga = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(st):
+            with torch.cuda.graph(ga, stream=st, capture_error_mode="thread_local"):
+                run_adaptive()
+        torch.cuda.synchronize()
+        ev = timed(ga, max(3, args.steps // 2))
+        torch.cuda.synchronize()
+        ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+        adaptive.append({"threshold": theta, "value": S / (ms * 1e-3), "unit": "denoising steps/s",
+                         "ms_per_block": ms, "refreshes": n_refresh, "refreshes_per_layer": n_refresh / N,
+                         "max_drift": dmax, "max_abs_vs_interval_1": float(diff.abs().max()),
+                         "rel_l2_vs_interval_1": float(diff.norm() / exact.norm())})
+        del ga, exact, diff
     ev_p = timed(graphs[("prefix", 0)], max(3, args.steps // 2))
     ev_s = timed(graphs[("step", 0)], max(3, args.steps // 2))
     torch.cuda.synchronize()
@@ -826,6 +869,7 @@ def run_layers(args, wl, rank, world, local):
         "roofline": roofline,
         "prefix_us": pfx_launch_ms * 1e3, "step_us": step_launch_ms * 1e3,
         "interval_sweep": sweep,
+        **({"adaptive_sweep": adaptive} if adaptive else {}),
         "e2e": {"value": aggregate_steps_per_s(world, 1, S, e2e_ms), "unit": "denoising steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "one fbk_decode_block call per block; every layer's inputs H2D from pinned host and "
@@ -1173,6 +1217,145 @@ def run_facache(args, name, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ sparse prefix + cached residual
+
+SPARSE_METRIC = "sparse block-external attention with a cached residual: denoising steps/s (1×B200)"
+
+
+def run_sparse(args, wl, rank, world, local):
+    """One bench step = one block of the sparse schedule (FlashBlock, Abstract:
+    sparse attention with complementary residual reuse; the reading of
+    oracle/sparse_residual.py): at step 0 the page means, the top-k pages by
+    the block queries' scores, the dense and the sparse prefix state and the
+    residual between them; at every step the sparse state over the kept pages
+    with that step's queries, the residual applied, and the step kernel. One
+    CUDA graph per block, L2 flushed before it. Contiguous workloads are laid
+    out in 64-token pages for this (the page table is what the sparse state
+    reads through)."""
+    import dataclasses
+    import torch
+    from cached_block_attention_b200 import fbk, synth
+    if not wl.page_size:
+        wl = dataclasses.replace(wl, page_size=64, page_seed=4242)
+    dev = torch.device("cuda", local)
+    S = wl.steps
+    lens_np = wl.prefix_lens()
+    ks, vs = synth.gen_prefix(wl, lens_np)
+    kp, vp, table = synth.paged_cache(ks, vs, wl.n_kv_heads, wl.head_dim, wl.page_size, wl.block_len, wl.page_seed)
+    del ks, vs
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    lens = torch.from_numpy(lens_np.astype(np.int32)).to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    cache = fbk.KVCache(to(kp), to(vp), lens, torch.from_numpy(table).to(dev), err)
+    del kp, vp
+    shape = fbk.Shape(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.block_len, 1.0, wl.rope_base)
+    steps = [tuple(to(x) for x in synth.gen_step(wl, s)) for s in range(S)]
+    b, maxp = table.shape
+    pages = (lens_np + wl.page_size - 1) // wl.page_size
+    k = max(1, int(round(args.keep * float(pages.mean()))))
+    means = torch.zeros(b, maxp, wl.n_kv_heads, wl.head_dim, dtype=torch.float32, device=dev)
+    kept = torch.empty(b, k, dtype=torch.int32, device=dev)
+    kept_lens = torch.empty(b, dtype=torch.int32, device=dev)
+    sel_ws = torch.empty(fbk.select_pages_workspace_bytes(shape, cache), dtype=torch.uint8, device=dev)
+    sparse_cache = fbk.KVCache(cache.k, cache.v, kept_lens, kept, err)
+    ws = torch.empty(fbk.prefix_workspace_bytes(shape, cache, 0), dtype=torch.uint8, device=dev)
+    dense, sparse, ext = (fbk.Partial.empty(shape, dev) for _ in range(3))
+    r_o = torch.empty(b, wl.n_q_heads, wl.block_len, wl.head_dim, dtype=torch.float32, device=dev)
+    r_lse = torch.empty(b, wl.n_q_heads, wl.block_len, dtype=torch.float32, device=dev)
+    out = torch.empty(S, b, wl.block_len, wl.n_q_heads, wl.head_dim, dtype=torch.bfloat16, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    def seg_select():
+        fbk.page_means(shape, cache, means)
+        fbk.select_pages(shape, steps[0][0], cache, means, k, kept, kept_lens, sel_ws)
+
+    def seg_dense():
+        fbk.prefix_partial(shape, steps[0][0], cache, dense, ws)
+
+    def seg_sparse(s=0):
+        fbk.prefix_partial_at(shape, steps[s][0], lens, sparse_cache, sparse, ws)
+
+    def block():
+        seg_select()
+        seg_dense()
+        seg_sparse(0)
+        fbk.residual_capture(shape, dense, sparse, r_o, r_lse)
+        fbk.block_attn_merge(shape, steps[0][0], steps[0][1], steps[0][2], lens, dense, out[0])
+        for s in range(1, S):
+            seg_sparse(s)
+            fbk.residual_apply(shape, sparse, r_o, r_lse, ext)
+            fbk.block_attn_merge(shape, steps[s][0], steps[s][1], steps[s][2], lens, ext, out[s])
+
+    for _ in range(2):
+        block()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0, f"device error flags {int(err.item())}"
+    st = torch.cuda.Stream(dev)
+    st.wait_stream(torch.cuda.current_stream(dev))
+    graphs = {}
+    with torch.cuda.stream(st):
+        for name, fn in (("block", block), ("select", seg_select), ("dense", seg_dense), ("sparse", seg_sparse)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st, capture_error_mode="thread_local"):
+                fn()
+            graphs[name] = g
+    torch.cuda.synchronize()
+
+    def timed(g, n):
+        evs = []
+        with torch.cuda.stream(st):
+            for _ in range(n):
+                flush.zero_()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e[0].record(st)
+                g.replay()
+                e[1].record(st)
+                evs.append(e)
+        return evs
+
+    timed(graphs["block"], args.warmup)
+    barrier(world)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    evs = timed(graphs["block"], args.steps)
+    barrier(world)
+    clock_info = clocks.stop()
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), world)
+    part = {}
+    for name in ("select", "dense", "sparse"):
+        ev = timed(graphs[name], max(3, args.steps // 2))
+        torch.cuda.synchronize()
+        part[name] = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    kept_tokens = int(kept_lens.sum())
+    hbm_gbs, _, _, peak_kind = load_peaks()
+    sparse_bytes = 4 * wl.n_kv_heads * wl.head_dim * kept_tokens
+    achieved = sparse_bytes / (part["sparse"] * 1e-3) / 1e9
+    line = {
+        "metric": SPARSE_METRIC, "value": aggregate_steps_per_s(world, args.steps, S, total_ms),
+        "unit": "denoising steps/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "keep": args.keep, "kept_pages_per_sequence": k,
+                   "page_size": wl.page_size, "kept_tokens": kept_tokens, "prefix_tokens": int(lens_np.sum()),
+                   "bench_step": f"one block of the sparse schedule ({S} steps), one CUDA graph",
+                   "l2": "flushed (2x L2 memset) before every timed block, outside the events",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                     "frac": achieved / hbm_gbs, "peak_kind": f"{peak_kind} hbm_gbs", "traffic": None,
+                     "traffic_key": None, "kernel": "fbk_prefix_partial_at (kept pages)",
+                     "algorithmic_bytes_per_launch": sparse_bytes, "launch_us": part["sparse"] * 1e3},
+        "select_us": part["select"] * 1e3, "dense_prefix_us": part["dense"] * 1e3,
+        "sparse_prefix_us": part["sparse"] * 1e3,
+        "gpu_launches": None,
+        "clocks": clock_info,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    graphs.clear()
+
+
 def layer_mode(args):
     return args.layers > 1 or bool(args.refresh_interval)
 
@@ -1211,6 +1394,19 @@ def main():
                 dist.destroy_process_group()
         return
     wl = synth.WORKLOADS[args.workload]
+    if args.op == "sparse_prefix":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the sparse schedule has no timed oracle arm; "
+                                                                  "its oracle is exercised by the tests"}))
+            return
+        rank, world, local = dist_setup(args.gpus)
+        try:
+            run_sparse(args, wl, rank, world, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         if layer_mode(args):
