@@ -676,7 +676,7 @@ fbk_status fbk_page_means(const fbk_shape *shape, const fbk_kv_cache *cache, flo
 size_t fbk_select_pages_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache) {
   if (check_shape(shape) != FBK_OK || !cache || !cache->paged || cache->max_pages_per_seq < 1) return 0;
   const size_t qrot = (size_t)shape->batch * shape->block_len * shape->n_q_heads * shape->head_dim * 4;
-  return align256(qrot) + align256((size_t)shape->batch * cache->max_pages_per_seq * 4);
+  return align256(qrot) + align256((size_t)shape->batch * shape->n_kv_heads * cache->max_pages_per_seq * 4);
 }
 
 fbk_status fbk_select_pages(const fbk_shape *shape, const void *q_blk, const fbk_kv_cache *cache, const float *means,
@@ -687,6 +687,7 @@ fbk_status fbk_select_pages(const fbk_shape *shape, const void *q_blk, const fbk
   if ((st = check_cache(shape, cache)) != FBK_OK) return st;
   if (!cache->paged) return FBK_ERR_UNSUPPORTED;
   if (!q_blk || !means || !kept_table || !kept_lens || k < 1) return FBK_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(means) & 15u) return FBK_ERR_UNSUPPORTED;  // 16-byte vector loads
   if ((size_t)cache->max_pages_per_seq * 8 > 200 * 1024) return FBK_ERR_UNSUPPORTED;  // scores + flags in smem
   const size_t need = fbk_select_pages_workspace_bytes(shape, cache);
   if (!ws || ws_bytes < need) return FBK_ERR_WORKSPACE;

@@ -13,8 +13,9 @@
 //
 // The step moves a few MB and is latency-bound, so both variants are built
 // around one DRAM round trip: every input of the CTA is requested up front
-// (cp.async for block K/V and query rows, register loads for the prefix
-// state), and the rest runs from shared memory and registers.
+// (cp.async for block V, register loads for block K, the query rows and the
+// prefix state; K and Q are rotated in registers as they arrive and stored
+// once), and the rest runs from shared memory and registers.
 //  * FBK_BF16: a CTA holds RT tiles of 16 query rows of one (sequence,
 //    kv-head) unit and that unit's block K/V. S = Q^ K^T and O = P~ V are
 //    warp-level bf16 tensor-core MMAs (mma.sync m16n8k16, fp32 accumulation;
@@ -75,7 +76,7 @@ constexpr int STEP_ROWS = 16;  // query rows of one row tile: one m16 MMA tile
 template <int D, int WPT, int RT>
 struct StepLayout {  // byte offsets in shared memory, all 16-byte aligned
   static constexpr int RS = D * 2 + 16;  // padded bf16 row: the 8 rows of an ldmatrix hit distinct banks
-  int bpad, ps_stride, ks, vs, qs, ps, red, cs, dq, dc, bytes;
+  int bpad, ps_stride, ks, vs, qs, ps, red, cs, dq, dc, rq, bytes;
   __host__ __device__ StepLayout(int blk, bool drift = false) {
     bpad = (blk + 15) & ~15;
     ps_stride = bpad * 2 + 16;
@@ -89,7 +90,8 @@ struct StepLayout {  // byte offsets in shared memory, all 16-byte aligned
     // adaptive refresh only: the query rows of the next step and of the
     // state's step ([2][rows][RS]), then 1 - cos per row (fp32)
     dc = dq + (drift ? 2 * RT * STEP_ROWS * RS : 0);
-    bytes = dc + (drift ? RT * STEP_ROWS * 4 : 0);
+    rq = dc + (drift ? RT * STEP_ROWS * 4 : 0);
+    bytes = rq + RT * STEP_ROWS * 16;  // per query row: its offset in q (8 bytes) and token (4 bytes)
   }
 };
 
@@ -132,6 +134,8 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
   float *red_max = reinterpret_cast<float *>(sm + lay.red);
   float *red_sum = red_max + RT * WPT * STEP_ROWS;
   float2 *cs = reinterpret_cast<float2 *>(sm + lay.cs);
+  long long *s_qoff = reinterpret_cast<long long *>(sm + lay.rq);
+  int *s_tq = reinterpret_cast<int *>(sm + lay.rq + CTA_ROWS * 8);
 
   const int u = blockIdx.x / tiles, r0 = (blockIdx.x % tiles) * CTA_ROWS;
   const int b = u / g.hkv, kvh = u % g.hkv;
@@ -154,22 +158,39 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
     // chunks c = 0..7 of one row read 8 consecutive float4 (no bank conflict)
     cs[t * HALF + ((i >> 1) & 3) * (D / 8) + (i >> 3) * 2 + (i & 1)] = make_float2(c, sn);
   }
+  // each query row's token and the offset of its row in q (kernel parameters only)
+  for (int rr = tid; rr < rows_cta; rr += NTHREADS) {
+    const int r = r0 + rr, t = r % blk, h = kvh * g.group + r / blk;
+    s_tq[rr] = t;
+    s_qoff[rr] = (((long long)b * blk + t) * g.hq + h) * D;
+  }
+  __syncthreads();
   pdl_wait();
   pdl_release();
   if (dr.clear && blockIdx.x == 0 && tid == 0) *dr.clear = 0;  // this step's refresh request is used up
 
-  // ---- 1. every global read of the CTA, issued at once
+  // ---- 1. every global read of the CTA, issued at once: block V by cp.async
+  // into shared memory; block K and the query rows into registers, in pairs of
+  // 16-byte chunks (c, c + D/16) that hold the RoPE pairs (i, i + D/2), to be
+  // rotated there; the prefix state into registers (below)
   const long long kv_row0 = (long long)b * blk * g.hkv + kvh;  // token t: row kv_row0 + t*hkv
   for (int idx = tid; idx < blk * CH; idx += NTHREADS) {
     const int t = idx / CH, c = idx % CH;
-    const long long src = (kv_row0 + (long long)t * g.hkv) * D + c * 8;
-    cp_async16(Ks + t * RS + c * 16, kb + src);
-    cp_async16(Vs + t * RS + c * 16, vb + src);
+    cp_async16(Vs + t * RS + c * 16, vb + (kv_row0 + (long long)t * g.hkv) * D + c * 8);
   }
-  for (int idx = tid; idx < rows_cta * CH; idx += NTHREADS) {
-    const int rr = idx / CH, c = idx % CH, r = r0 + rr;
-    const int t = r % blk, h = kvh * g.group + r / blk;
-    cp_async16(Qs + rr * RS + c * 16, q + (((long long)b * blk + t) * g.hq + h) * D + c * 8);
+  // B <= 64 (the C ABI rejects longer blocks): MAXI items per thread cover every row
+  constexpr int PAIRS = D / 16, MAXI = ((64 + CTA_ROWS) * PAIRS + NTHREADS - 1) / NTHREADS;
+  const int nrot = (blk + rows_cta) * PAIRS;
+  uint4 xa[MAXI], xb[MAXI];
+#pragma unroll
+  for (int i = 0; i < MAXI; ++i) {
+    const int idx = tid + i * NTHREADS;
+    if (idx < nrot) {
+      const int rowi = idx / PAIRS, c = idx % PAIRS;
+      const __nv_bfloat16 *row = rowi < blk ? kb + (kv_row0 + (long long)rowi * g.hkv) * D : q + s_qoff[rowi - blk];
+      xa[i] = __ldg(reinterpret_cast<const uint4 *>(row) + c);
+      xb[i] = __ldg(reinterpret_cast<const uint4 *>(row + HALF) + c);
+    }
   }
   if (drift) {  // the rows of the next step's queries and of the state's queries
     const __nv_bfloat16 *qn = dr.q_base + (long long)dr.next_step * dr.q_stride;
@@ -210,6 +231,31 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
   }
   if (va) { m1a = __ldg(pfx.m + pa); l1a = __ldg(pfx.l + pa); }
   if (vbr) { m1b = __ldg(pfx.m + pb); l1b = __ldg(pfx.l + pb); }
+  // ---- 2. rotate block K and the query rows at their block offsets, 8 pairs per item, and store them
+#pragma unroll
+  for (int i = 0; i < MAXI; ++i) {
+    const int idx = tid + i * NTHREADS;
+    if (idx < nrot) {
+      const int rowi = idx / PAIRS, c = idx % PAIRS;
+      const bool is_k = rowi < blk;
+      const int t = is_k ? rowi : s_tq[rowi - blk];
+      uint8_t *row = is_k ? Ks + rowi * RS : Qs + (rowi - blk) * RS;
+      const uint4 a = xa[i], bq = xb[i];
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {bq.x, bq.y, bq.z, bq.w};
+      const float4 *cp = reinterpret_cast<const float4 *>(cs + t * HALF + 2 * c);  // + e * (D / 8) float2
+      uint32_t y1[4], y2[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4 c2 = cp[e * (D / 16)];  // (cos, sin) of pairs 8c + 2e and 8c + 2e + 1
+        const float x1l = __uint_as_float(aw[e] << 16), x1h = __uint_as_float(aw[e] & 0xffff0000u);
+        const float x2l = __uint_as_float(bw[e] << 16), x2h = __uint_as_float(bw[e] & 0xffff0000u);
+        y1[e] = pack2(x1l * c2.x - x2l * c2.y, x1h * c2.z - x2h * c2.w);
+        y2[e] = pack2(x2l * c2.x + x1l * c2.y, x2h * c2.z + x1h * c2.w);
+      }
+      *reinterpret_cast<uint4 *>(row + c * 16) = make_uint4(y1[0], y1[1], y1[2], y1[3]);
+      *reinterpret_cast<uint4 *>(row + D + c * 16) = make_uint4(y2[0], y2[1], y2[2], y2[3]);
+    }
+  }
   cp_async_wait_all();
   __syncthreads();
 
@@ -245,30 +291,6 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
       if (lane == 0) dcos[rr] = 0.5f * dd;
     }
   }
-
-  // ---- 2. rotate block K and the query rows in place at their block offsets, 8 pairs per item
-  for (int idx = tid; idx < (blk + rows_cta) * (D / 16); idx += NTHREADS) {
-    const int rowi = idx / (D / 16), c = idx % (D / 16);
-    const bool is_k = rowi < blk;
-    const int t = is_k ? rowi : (r0 + rowi - blk) % blk;
-    uint8_t *row = is_k ? Ks + rowi * RS : Qs + (rowi - blk) * RS;
-    uint4 *p1 = reinterpret_cast<uint4 *>(row + c * 16), *p2 = reinterpret_cast<uint4 *>(row + D + c * 16);
-    const uint4 a = *p1, bq = *p2;
-    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {bq.x, bq.y, bq.z, bq.w};
-    const float4 *cp = reinterpret_cast<const float4 *>(cs + t * HALF + 2 * c);  // + e * (D / 8) float2
-    uint32_t y1[4], y2[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float4 c2 = cp[e * (D / 16)];  // (cos, sin) of pairs 8c + 2e and 8c + 2e + 1
-      const float x1l = __uint_as_float(aw[e] << 16), x1h = __uint_as_float(aw[e] & 0xffff0000u);
-      const float x2l = __uint_as_float(bw[e] << 16), x2h = __uint_as_float(bw[e] & 0xffff0000u);
-      y1[e] = pack2(x1l * c2.x - x2l * c2.y, x1h * c2.z - x2h * c2.w);
-      y2[e] = pack2(x2l * c2.x + x1l * c2.y, x2h * c2.z + x1h * c2.w);
-    }
-    *p1 = make_uint4(y1[0], y1[1], y1[2], y1[3]);
-    *p2 = make_uint4(y2[0], y2[1], y2[2], y2[3]);
-  }
-  __syncthreads();
 
   const uint32_t qs_a = (uint32_t)__cvta_generic_to_shared(Qs + tr0 * RS),
                  ks_a = (uint32_t)__cvta_generic_to_shared(Ks), vs_a = (uint32_t)__cvta_generic_to_shared(Vs);
@@ -351,9 +373,11 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
     float *rmax = red_max + grp * WPT * STEP_ROWS, *rsum = red_sum + grp * WPT * STEP_ROWS;
     // ---- 3. S = Q^ K^T for key n-tiles warp and warp + 4 (16 rows x 8 keys each)
     const int b_row = lane & 7, b_col = 8 * ((lane >> 3) & 1);  // B fragment (k16 x n8)
-    float sacc[2][4];
+    float sacc[2][4], sacc2[2][4];  // even and odd kk: two chains of dependent MMAs
 #pragma unroll
-    for (int e = 0; e < 2; ++e) sacc[e][0] = sacc[e][1] = sacc[e][2] = sacc[e][3] = 0.f;
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+      for (int x = 0; x < 4; ++x) sacc[e][x] = sacc2[e][x] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       uint32_t a0, a1, a2, a3;
@@ -364,10 +388,15 @@ __global__ void __launch_bounds__(RT * WPT * 32) block_merge_mma_kernel(
         if (nt < NT) {
           uint32_t b0, b1;
           ldsm_x2(ks_a + (8 * nt + b_row) * RS + (16 * kk + b_col) * 2, b0, b1);
-          mma16816(sacc[e], a0, a1, a2, a3, b0, b1);
+          if (kk & 1) mma16816(sacc2[e], a0, a1, a2, a3, b0, b1);
+          else mma16816(sacc[e], a0, a1, a2, a3, b0, b1);
         }
       }
     }
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+      for (int x = 0; x < 4; ++x) sacc[e][x] += sacc2[e][x];
     // ---- 4. block softmax across the tile's warps (log2 units)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {

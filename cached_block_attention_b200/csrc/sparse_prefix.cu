@@ -24,9 +24,18 @@ namespace fbk {
 namespace {
 
 // Mean key of every logical page (b, lp) of every kv-head: [b, max_pages, Hkv, d]
-// fp32. One CTA per (b, lp); pages past the prefix are left untouched.
-__global__ void __launch_bounds__(256) page_means_kernel(Geometry g, float *__restrict__ means) {
+// fp32. One CTA per (b, lp); pages past the prefix are left untouched. The
+// page's keys of one kv-head are P rows of d bf16 in one run; the CTA reads a
+// kv-head's run in 16-byte chunks (thread: chunk c of rows s, s + NS, ...),
+// then sums the NS partial sums of each column in a fixed order.
+constexpr int MEAN_THREADS = 256;
+
+template <int D>
+__global__ void __launch_bounds__(MEAN_THREADS) page_means_kernel(Geometry g, float *__restrict__ means) {
+  constexpr int CPR = D / 8, NS = MEAN_THREADS / CPR;  // 16-byte chunks per row, row slots
+  __shared__ float part[NS][D + 4];
   const int b = blockIdx.x / g.max_pages, lp = blockIdx.x % g.max_pages;
+  const int c = threadIdx.x % CPR, slot = threadIdx.x / CPR;
   pdl_wait();
   pdl_release();
   const int L = prefix_len(g, b);
@@ -34,16 +43,33 @@ __global__ void __launch_bounds__(256) page_means_kernel(Geometry g, float *__re
   if (n <= 0) return;
   const int pid = g.page_table[(long long)b * g.max_pages + lp];
   if (pid < 0 || (long long)pid >= g.num_pages) {
-    raise_flag(g, FBK_DEVERR_PAGE_ID);
+    if (threadIdx.x == 0) raise_flag(g, FBK_DEVERR_PAGE_ID);
     return;
   }
-  const int cols = g.hkv * g.d;
-  for (int c = threadIdx.x; c < cols; c += blockDim.x) {
-    const int kvh = c / g.d, i = c % g.d;
-    const __nv_bfloat16 *src = g.kc + (((long long)pid * g.hkv + kvh) * g.page_size) * g.d + i;
-    float s = 0.f;
-    for (int t = 0; t < n; ++t) s += __bfloat162float(src[(long long)t * g.d]);
-    means[(((long long)b * g.max_pages + lp) * g.hkv + kvh) * g.d + i] = s / (float)n;
+  const float inv_n = 1.f / (float)n;
+  for (int kvh = 0; kvh < g.hkv; ++kvh) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(g.kc + ((long long)pid * g.hkv + kvh) * g.page_size * D) + c;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int t = slot; t < n; t += NS) {
+      const uint4 v = __ldg(src + (long long)t * CPR);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += __uint_as_float(w[e] << 16);
+        acc[2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[slot][8 * c + e] = acc[e];
+    __syncthreads();
+    for (int i = threadIdx.x; i < D; i += MEAN_THREADS) {
+      float s = 0.f;
+#pragma unroll
+      for (int k = 0; k < NS; ++k) s += part[k][i];
+      means[(((long long)b * g.max_pages + lp) * g.hkv + kvh) * D + i] = s * inv_n;
+    }
+    __syncthreads();  // part is rewritten by the next kv-head
   }
 }
 
@@ -67,68 +93,228 @@ __global__ void __launch_bounds__(256) rotate_queries_kernel(Geometry g, const _
   }
 }
 
-// Score of every logical page: one warp per (b, lp), the largest
-// tau <qrot[b, t, h], kbar[b, lp, kv(h)]> over t and h. Pages past the prefix
-// score -inf.
-__global__ void __launch_bounds__(256) page_scores_kernel(Geometry g, const float *__restrict__ qrot,
-                                                          const float *__restrict__ means,
-                                                          float *__restrict__ scores) {
+// Score of every logical page per kv-head: scores [b, Hkv, max_pages], the
+// largest tau <qrot[b, t, h], kbar[b, lp, kvh]> over the block's tokens t and
+// the query heads h of kv-head kvh (the page's score is the largest over the
+// kv-heads, taken by the selection). One CTA per (b, kvh, 64 pages): the mean
+// keys of its pages and then 64 query rows at a time are staged transposed in
+// shared memory ([d][64] each), and each thread forms a 4 x 4 block of dot
+// products in fp32 (rows 4rg.., pages 4pg..), 16 multiply-adds per two
+// 16-byte shared loads. Pages past the prefix are not written.
+constexpr int SCORE_PAGES = 64, SCORE_ROWS = 64, SCORE_THREADS = 256;
+
+constexpr int score_smem_bytes(int d) { return (d * (SCORE_PAGES + SCORE_ROWS) + SCORE_THREADS / 16 * SCORE_PAGES) * 4; }
+
+template <int D>
+__global__ void __launch_bounds__(SCORE_THREADS) page_scores_kernel(Geometry g, const float *__restrict__ qrot,
+                                                                    const float *__restrict__ means,
+                                                                    float *__restrict__ scores, int tiles) {
+  extern __shared__ float4 score_smem[];
+  float(*Kt)[SCORE_PAGES] = reinterpret_cast<float(*)[SCORE_PAGES]>(score_smem);
+  float(*Qt)[SCORE_ROWS] = reinterpret_cast<float(*)[SCORE_ROWS]>(&Kt[D][0]);
+  float(*red)[SCORE_PAGES] = reinterpret_cast<float(*)[SCORE_PAGES]>(&Qt[D][0]);
+  const int tile = blockIdx.x % tiles, u = blockIdx.x / tiles, b = u / g.hkv, kvh = u % g.hkv;
+  const int tid = threadIdx.x, pg = tid % 16, rg = tid / 16;
   pdl_wait();
   pdl_release();
-  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= (long long)g.batch * g.max_pages) return;
-  const int b = (int)(warp / g.max_pages), lp = (int)(warp % g.max_pages);
   const int L = prefix_len(g, b);
-  float best = -CUDART_INF_F;
-  if (lp * g.page_size < L) {
-    for (int h = 0; h < g.hq; ++h) {
-      const float *kbar = means + (((long long)b * g.max_pages + lp) * g.hkv + h / g.group) * g.d;
-      for (int t = 0; t < g.blk; ++t) {
-        const float *qv = qrot + (((long long)b * g.blk + t) * g.hq + h) * g.d;
-        float s = 0.f;
-        for (int i = lane; i < g.d; i += 32) s += qv[i] * kbar[i];
-        s = warp_sum(s);
-        best = fmaxf(best, g.tau * s);
-      }
-    }
+  const int n_pages = (L + g.page_size - 1) / g.page_size, p0 = tile * SCORE_PAGES;
+  if (p0 >= n_pages) return;
+  const int np = min(SCORE_PAGES, n_pages - p0), R = g.group * g.blk;  // rows of the kv-head: (head, token)
+  for (int idx = tid; idx < SCORE_PAGES * (D / 4); idx += SCORE_THREADS) {
+    const int p = idx % SCORE_PAGES, i4 = idx / SCORE_PAGES;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p < np)
+      v = __ldg(reinterpret_cast<const float4 *>(means + (((long long)b * g.max_pages + p0 + p) * g.hkv + kvh) * D) + i4);
+    Kt[4 * i4][p] = v.x;
+    Kt[4 * i4 + 1][p] = v.y;
+    Kt[4 * i4 + 2][p] = v.z;
+    Kt[4 * i4 + 3][p] = v.w;
   }
-  if (lane == 0) scores[warp] = best;
+  float best[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+  for (int r0 = 0; r0 < R; r0 += SCORE_ROWS) {
+    __syncthreads();  // the previous rows are consumed
+    for (int idx = tid; idx < SCORE_ROWS * (D / 4); idx += SCORE_THREADS) {
+      const int rr = idx % SCORE_ROWS, i4 = idx / SCORE_ROWS, r = r0 + rr;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < R) {
+        const int hl = r / g.blk, t = r % g.blk;
+        v = __ldg(reinterpret_cast<const float4 *>(qrot + (((long long)b * g.blk + t) * g.hq + kvh * g.group + hl) * D) + i4);
+      }
+      Qt[4 * i4][rr] = v.x;
+      Qt[4 * i4 + 1][rr] = v.y;
+      Qt[4 * i4 + 2][rr] = v.z;
+      Qt[4 * i4 + 3][rr] = v.w;
+    }
+    __syncthreads();
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < D; ++i) {
+      const float4 kv = *reinterpret_cast<const float4 *>(&Kt[i][4 * pg]);
+      const float4 qv = *reinterpret_cast<const float4 *>(&Qt[i][4 * rg]);
+      const float qa[4] = {qv.x, qv.y, qv.z, qv.w}, ka[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(qa[x], ka[y], acc[x][y]);
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+      if (r0 + 4 * rg + x < R)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) best[y] = fmaxf(best[y], g.tau * acc[x][y]);
+  }
+#pragma unroll
+  for (int y = 0; y < 4; ++y) red[rg][4 * pg + y] = best[y];
+  __syncthreads();
+  if (tid < np) {
+    float m = -CUDART_INF_F;
+#pragma unroll
+    for (int k = 0; k < SCORE_THREADS / 16; ++k) m = fmaxf(m, red[k][tid]);
+    scores[((long long)b * g.hkv + kvh) * g.max_pages + p0 + tid] = m;
+  }
 }
 
-// Top-k pages of each sequence (one CTA per sequence): a page is kept when
-// fewer than k pages beat it (higher score, or equal score and lower index).
-// Writes the kept physical pages in increasing logical order and their token
-// count (a partial last page counts its tokens; being the highest page, it
-// is last when kept).
-__global__ void __launch_bounds__(1024) select_pages_kernel(Geometry g, const float *__restrict__ scores, int k,
-                                                            int *__restrict__ kept_table, int *__restrict__ kept_lens) {
-  extern __shared__ float sel_smem[];
-  float *sc = sel_smem;
-  int *keep = reinterpret_cast<int *>(sc + g.max_pages);
-  const int b = blockIdx.x;
+// Top-k pages of each sequence (one CTA per sequence). A page's score is the
+// largest of its kv-heads' scores; the k best pages are kept, ties to the
+// lower page index. The k-th largest score is found by a radix select over the
+// scores' order-preserving 32-bit keys (four 8-bit digits, most significant
+// first, one shared-memory histogram each); the pages above it are kept, and
+// of the pages equal to it the lowest-indexed ones that complete the k. The
+// kept pages' physical ids go to kept_table in increasing logical order (their
+// positions from a block-wide scan of the keep flags, each thread owning a run
+// of consecutive pages), with their token count (a partial last page counts
+// its tokens; being the highest page, it is last when kept).
+constexpr int SEL_THREADS = 1024;
+
+__device__ __forceinline__ unsigned order_key(float f) {  // a < b  <=>  order_key(a) < order_key(b)
+  const unsigned u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive prefix sum of v over the CTA's threads in thread order; *total
+// gets the sum. Every thread of the CTA calls it.
+__device__ int block_exclusive_scan(int v, int *wsum, int *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < SEL_THREADS / 32 ? wsum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    wsum[lane] = t;
+  }
+  __syncthreads();
+  const int before = warp > 0 ? wsum[warp - 1] : 0;
+  *total = wsum[SEL_THREADS / 32 - 1];
+  __syncthreads();  // wsum is reused by the next call
+  return before + x - v;
+}
+
+__global__ void __launch_bounds__(SEL_THREADS) select_pages_kernel(Geometry g, const float *__restrict__ scores, int k,
+                                                                   int *__restrict__ kept_table,
+                                                                   int *__restrict__ kept_lens) {
+  extern __shared__ unsigned sel_key[];  // [max_pages]
+  __shared__ int hist[256];
+  __shared__ int wsum[32];
+  __shared__ unsigned s_prefix;
+  __shared__ int s_rem;
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
   pdl_release();
   const int L = prefix_len(g, b);
   const int n_pages = (L + g.page_size - 1) / g.page_size;
-  for (int p = threadIdx.x; p < n_pages; p += blockDim.x) sc[p] = scores[(long long)b * g.max_pages + p];
-  __syncthreads();
-  for (int p = threadIdx.x; p < n_pages; p += blockDim.x) {
-    int beaten = 0;
-    for (int o = 0; o < n_pages; ++o) beaten += (sc[o] > sc[p]) || (sc[o] == sc[p] && o < p);
-    keep[p] = beaten < k ? 1 : 0;
+  for (int p = tid; p < n_pages; p += SEL_THREADS) {
+    float m = -CUDART_INF_F;
+    for (int kvh = 0; kvh < g.hkv; ++kvh) m = fmaxf(m, scores[((long long)b * g.hkv + kvh) * g.max_pages + p]);
+    sel_key[p] = order_key(m);
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {  // n_pages is at most max_pages: a serial pass is short
-    int pos = 0, tokens = 0;
-    for (int p = 0; p < n_pages; ++p) {
-      if (!keep[p]) continue;
-      kept_table[(long long)b * k + pos++] = g.page_table[(long long)b * g.max_pages + p];
+  const bool keep_all = k >= n_pages;
+  unsigned prefix = 0u, mask = 0u;
+  int rem = keep_all ? n_pages : k;  // pages still to take among those matching prefix under mask
+  for (int shift = 24; shift >= 0 && !keep_all; shift -= 8) {
+    for (int i = tid; i < 256; i += SEL_THREADS) hist[i] = 0;
+    __syncthreads();  // keys written (first pass), histogram cleared
+    for (int p = tid; p < n_pages; p += SEL_THREADS) {
+      const unsigned key = sel_key[p];
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {  // lane l holds digits 255 - 8l down to 248 - 8l
+      int c[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = hist[255 - 8 * lane - j];
+        sum += c[j];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, incl >= rem);  // non-empty: the counts add up to >= rem
+      if (lane == __ffs(hit) - 1) {
+        int cum = incl - sum;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (cum + c[j] >= rem) {
+            s_prefix = prefix | ((unsigned)(255 - 8 * lane - j) << shift);
+            s_rem = rem - cum;
+            break;
+          }
+          cum += c[j];
+        }
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    rem = s_rem;
+    mask |= 255u << shift;
+  }
+  __syncthreads();  // keys visible (keep_all skipped the passes)
+  // prefix is now the k-th largest key; the rem lowest-indexed pages equal to it are kept
+  const int C = (n_pages + SEL_THREADS - 1) / SEL_THREADS, lo = min(tid * C, n_pages), hi = min(lo + C, n_pages);
+  int n_eq = 0;
+  for (int p = lo; p < hi && !keep_all; ++p) n_eq += sel_key[p] == prefix;
+  int total;
+  int eq_rank = block_exclusive_scan(n_eq, wsum, &total);
+  int n_keep = 0, tokens = 0;
+  for (int p = lo; p < hi; ++p) {
+    const unsigned key = sel_key[p];
+    bool keep = keep_all || key > prefix;
+    if (!keep_all && key == prefix) keep = eq_rank++ < rem;
+    if (keep) {
+      ++n_keep;
       tokens += min(g.page_size, L - p * g.page_size);
     }
-    for (; pos < k; ++pos) kept_table[(long long)b * k + pos] = -1;
-    kept_lens[b] = tokens;
   }
+  int kept_total;
+  int pos = block_exclusive_scan(n_keep, wsum, &kept_total);
+  int tok_total;
+  block_exclusive_scan(tokens, wsum, &tok_total);
+  eq_rank -= n_eq;  // this run's first rank among the equal pages, again
+  for (int p = lo; p < hi; ++p) {
+    const unsigned key = sel_key[p];
+    bool keep = keep_all || key > prefix;
+    if (!keep_all && key == prefix) keep = eq_rank++ < rem;
+    if (keep) kept_table[(long long)b * k + pos++] = g.page_table[(long long)b * g.max_pages + p];
+  }
+  for (int j = kept_total + tid; j < k; j += SEL_THREADS) kept_table[(long long)b * k + j] = -1;
+  if (tid == 0) kept_lens[b] = tok_total;
 }
 
 // Residual at a dense step, per row of [b, Hq, B]: R_O = (O~/l)_dense -
@@ -178,7 +364,8 @@ unsigned grid_for(long long n, int sms) {
 cudaError_t launch_page_means(const Geometry &g, float *means, cudaStream_t st) {
   const long long ctas = (long long)g.batch * g.max_pages;
   if (ctas > 0x7fffffffll) return cudaErrorInvalidConfiguration;
-  return launch_pdl(page_means_kernel, dim3((unsigned)ctas), dim3(256), 0, st, g, means);
+  if (g.d == 128) return launch_pdl(page_means_kernel<128>, dim3((unsigned)ctas), dim3(MEAN_THREADS), 0, st, g, means);
+  return launch_pdl(page_means_kernel<64>, dim3((unsigned)ctas), dim3(MEAN_THREADS), 0, st, g, means);
 }
 
 cudaError_t launch_select_pages(const Geometry &g, const __nv_bfloat16 *q, const float *means, int k, float *qrot,
@@ -186,16 +373,27 @@ cudaError_t launch_select_pages(const Geometry &g, const __nv_bfloat16 *q, const
   const long long nrot = (long long)g.batch * g.blk * g.hq * (g.d / 2);
   cudaError_t e = launch_pdl(rotate_queries_kernel, dim3(grid_for(nrot, sms)), dim3(256), 0, st, g, q, qrot);
   if (e != cudaSuccess) return e;
-  const long long warps = (long long)g.batch * g.max_pages;
-  e = launch_pdl(page_scores_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, st, g,
-                 (const float *)qrot, means, scores);
+  const int tiles = (g.max_pages + SCORE_PAGES - 1) / SCORE_PAGES;
+  const long long ctas = (long long)g.batch * g.hkv * tiles;
+  if (ctas > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+  if (g.d == 128) {
+    e = cudaFuncSetAttribute(page_scores_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, score_smem_bytes(128));
+    if (e == cudaSuccess)
+      e = launch_pdl(page_scores_kernel<128>, dim3((unsigned)ctas), dim3(SCORE_THREADS), score_smem_bytes(128), st, g,
+                     (const float *)qrot, means, scores, tiles);
+  } else {
+    e = cudaFuncSetAttribute(page_scores_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, score_smem_bytes(64));
+    if (e == cudaSuccess)
+      e = launch_pdl(page_scores_kernel<64>, dim3((unsigned)ctas), dim3(SCORE_THREADS), score_smem_bytes(64), st, g,
+                     (const float *)qrot, means, scores, tiles);
+  }
   if (e != cudaSuccess) return e;
-  const size_t smem = (size_t)g.max_pages * (sizeof(float) + sizeof(int));
-  if (smem > 48 * 1024) {
+  const size_t smem = (size_t)g.max_pages * sizeof(unsigned);
+  if (smem > 40 * 1024) {
     e = cudaFuncSetAttribute(select_pages_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(select_pages_kernel, dim3(g.batch), dim3(1024), smem, st, g, (const float *)scores, k,
+  return launch_pdl(select_pages_kernel, dim3(g.batch), dim3(SEL_THREADS), smem, st, g, (const float *)scores, k,
                     kept_table, kept_lens);
 }
 

@@ -12,7 +12,7 @@ namespace fbk {
 cudaError_t launch_page_means(const Geometry &g, float *means, cudaStream_t st);
 
 // Page scores and the top-k pages per sequence; qrot [b, B, Hq, d] fp32 and
-// scores [b, max_pages] fp32 are scratch; kept_table [b, k] and kept_lens [b].
+// scores [b, Hkv, max_pages] fp32 are scratch; kept_table [b, k] and kept_lens [b].
 cudaError_t launch_select_pages(const Geometry &g, const __nv_bfloat16 *q, const float *means, int k, float *qrot,
                                 float *scores, int *kept_table, int *kept_lens, int sms, cudaStream_t st);
 

@@ -446,7 +446,8 @@ fbk_status fbk_facache_step(const fbk_shape *shape, int32_t n_rows, const void *
  *
  * fbk_page_means: means fp32 [b, max_pages_per_seq, Hkv, d], the mean key of
  *   every logical page of the prefix (pages past prefix_lens untouched).
- * fbk_select_pages: q_blk bf16 [b, B, Hq, d] before RoPE; k >= 1 pages kept;
+ * fbk_select_pages: q_blk bf16 [b, B, Hq, d] before RoPE; means as written by
+ *   fbk_page_means (16-byte aligned, else FBK_ERR_UNSUPPORTED); k >= 1 pages kept;
  *   kept_table int32 [b, k] (physical page ids in increasing logical order,
  *   -1 past the kept count) and kept_lens int32 [b] (their token count, the
  *   partial last page included), both on the device; workspace of

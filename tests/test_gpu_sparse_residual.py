@@ -84,6 +84,73 @@ def test_page_means_and_selection(cfg):
                 assert abs(scores[bi][p] - kth) <= 1e-4 * max(1.0, abs(kth)), (bi, p)
 
 
+def selection_near_ties_only(got, want, scores_b, n_kept):
+    """The device's selection equals the oracle's, except for pages whose fp64
+    score lies within fp32 rounding of the k-th score."""
+    if np.array_equal(got, want):
+        return
+    kth = np.sort(scores_b)[::-1][n_kept - 1]
+    for p in set(got) ^ set(want):
+        assert abs(scores_b[p] - kth) <= 1e-4 * max(1.0, abs(kth)), p
+
+
+def test_selection_with_exact_ties_takes_the_lower_pages():
+    """Six full pages whose every key is one large vector x (per kv-head) tie
+    exactly on both sides: their mean is x exactly, so their scores are equal
+    bit for bit, and they are the best pages. With k = 3 the three lowest
+    logical indices among them are kept."""
+    b, hq, hkv, d, blk, ps = 2, 8, 2, 128, 16, 64
+    lens = (64 * 40, 64 * 23 + 5)
+    case = H.make_case(b, hq, hkv, d, blk, lens, ps, 1.0, seed=41, steps=1)
+    rng = np.random.Generator(np.random.PCG64(4141))
+    copies = {}
+    for bi in range(b):
+        x = (rng.standard_normal((hkv, d)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+        n_full = lens[bi] // ps
+        tied = sorted(int(p) for p in rng.choice(n_full, size=6, replace=False))
+        for p in tied:
+            case.k_pfx_bits[bi][:, p * ps:(p + 1) * ps, :] = x[:, None, :]
+        copies[bi] = tied
+    q0 = case.step_f64(0)[0]
+    case.upload()
+    k = 3
+    _, kept, kept_lens = run_selection(case, k)
+    table = case.dev["cache"].page_table.cpu().numpy()
+    kept_np = kept.cpu().numpy()
+    scores = sr.page_scores(q0, case.k_pfx(), case.lens, hkv, 1.0, case.base, ps)
+    want = sr.select_pages(scores, k)
+    for bi in range(b):
+        tied = copies[bi]
+        assert len({float(scores[bi][p]) for p in tied}) == 1 and scores[bi][tied[0]] == scores[bi].max()
+        got = logical_pages(table[bi], kept_np[bi], k)
+        np.testing.assert_array_equal(got, tied[:k])
+        np.testing.assert_array_equal(want[bi], tied[:k])
+        assert int(kept_lens[bi]) == k * ps
+
+
+@pytest.mark.parametrize("k", [1, 1000, 3004])
+def test_selection_over_thousands_of_pages(k):
+    """3001 pages of 16 tokens (a partial last page), several pages per thread
+    in the selection, several score tiles: the selection follows the oracle's,
+    and k at or above the page count keeps every page."""
+    b, hq, hkv, d, blk, ps = 1, 4, 2, 64, 16, 16
+    L = 16 * 3000 + 7
+    case = H.make_case(b, hq, hkv, d, blk, (L,), ps, 1.0, seed=43, steps=1).upload()
+    _, kept, kept_lens = run_selection(case, k)
+    table = case.dev["cache"].page_table.cpu().numpy()
+    kept_np = kept.cpu().numpy()
+    q0 = case.step_f64(0)[0]
+    scores = sr.page_scores(q0, case.k_pfx(), case.lens, hkv, 1.0, case.base, ps)
+    n_pages = len(scores[0])
+    n_kept = min(k, n_pages)
+    got = logical_pages(table[0], kept_np[0], n_kept)
+    assert np.all(np.diff(got) > 0) and np.all(kept_np[0][n_kept:] == -1)
+    assert int(kept_lens[0]) == sum(min(ps, L - p * ps) for p in got)
+    if k >= n_pages:
+        np.testing.assert_array_equal(got, np.arange(n_pages))
+    selection_near_ties_only(got, sr.select_pages(scores, k)[0], scores[0], n_kept)
+
+
 @pytest.mark.parametrize("cfg", CASES)
 def test_sparse_state_and_approximate_step(cfg):
     from cached_block_attention_b200 import fbk
