@@ -8,9 +8,11 @@ libcuda link: the tensor-map encoder is fetched through the runtime's driver
 entry-point query). Objects go to _build/ at the repository root.
 
 It also links libfbk_testhooks.so, the test build: the same objects except
-the prefix kernel's, which is compiled with FBK_TEST_HOOKS so that a test
-can shorten the kernel's bounded waits and withhold one of its loads
-(include/fbk_test_hooks.h). Only the bounded-wait test loads it.
+the prefix kernel's and the FP8 quantisation's, which are compiled with
+FBK_TEST_HOOKS so that a test can shorten the prefix kernel's bounded waits
+and withhold one of its loads, and run the FP8 kernel's per-group scale step
+on given values (include/fbk_test_hooks.h). Only the bounded-wait and the
+FP8 scale tests load it.
 """
 from __future__ import annotations
 
@@ -27,7 +29,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfbk.so")
 TEST_LIB = os.path.join(PKG, "libfbk_testhooks.so")
-HOOKED = "prefix_tc.cu"  # the one source the test build compiles differently
+HOOKED = ("prefix_tc.cu", "fp8_quant.cu")  # the sources the test build compiles differently
 
 SOURCES = ["abi.cu", "prefix_tc.cu", "prefix_fp32.cu", "split_reduce.cu", "block_merge.cu",
            "commit.cu", "full_ref.cu", "fp8_quant.cu", "facache_rows.cu", "sparse_prefix.cu"]
@@ -70,7 +72,7 @@ def build(verbose: bool = False, force: bool = False, ptxas_info: bool = False) 
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
         return obj, r.stderr
 
-    jobs = [(src, False) for src in SOURCES] + [(HOOKED, True)]
+    jobs = [(src, False) for src in SOURCES] + [(src, True) for src in HOOKED]
     with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         results = list(ex.map(compile_one, jobs))
     objs = {job: o for job, (o, _) in zip(jobs, results)}
@@ -87,7 +89,7 @@ def build(verbose: bool = False, force: bool = False, ptxas_info: bool = False) 
                 raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
 
     link(LIB, [objs[(s, False)] for s in SOURCES])
-    link(TEST_LIB, [objs[(s, s == HOOKED)] for s in SOURCES])
+    link(TEST_LIB, [objs[(s, s in HOOKED)] for s in SOURCES])
     return LIB
 
 

@@ -32,13 +32,13 @@ def test_exports_every_declared_symbol(fbk):
     assert set(fbk.EXPORTS) == set(names)
 
 
-def test_test_build_exports_its_hook_and_the_library_does_not(fbk):
-    """libfbk_testhooks.so exports every fbk.h entry point plus the hook of
-    include/fbk_test_hooks.h; the library proper has no hook."""
+def test_test_build_exports_its_hooks_and_the_library_does_not(fbk):
+    """libfbk_testhooks.so exports every fbk.h entry point plus the hooks of
+    include/fbk_test_hooks.h; the library proper has none."""
     from cached_block_attention_b200 import build
     hooks = ctypes.CDLL(build.TEST_LIB)
     hook_names = declared_entry_points("fbk_test_hooks.h")
-    assert hook_names == ["fbk_test_set_wait_fault"]
+    assert hook_names == ["fbk_test_fp8_group_scale", "fbk_test_set_wait_fault"]
     for n in declared_entry_points() + hook_names:
         assert hasattr(hooks, n), n
     for n in hook_names:

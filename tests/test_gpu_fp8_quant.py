@@ -138,3 +138,28 @@ def test_empty_is_a_no_op():
     scales = torch.empty(0, 2, dtype=torch.float32, device="cuda")
     fbk.fp8_group_quant(x, codes, scales)
     torch.cuda.synchronize()
+
+
+def test_scale_step_is_exact_for_every_group_max():
+    """The kernel's per-group scale step (test build entry point, run on the
+    device): for every positive finite bf16 max|x| A the scale is the IEEE
+    quotient RN(A / 448), and where A >= 2^-80 the reciprocal that the
+    quotient steps use is the correctly rounded RN(1 / scale)."""
+    import ctypes
+    from cached_block_attention_b200 import build
+    build.build()
+    lib = ctypes.CDLL(build.TEST_LIB)
+    lib.fbk_test_fp8_group_scale.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int]
+    lib.fbk_test_fp8_group_scale.restype = ctypes.c_int
+    A = (np.arange(1, 0x7F80, dtype=np.uint32) << 16).view(np.float32)
+    a_d = torch.from_numpy(A).cuda()
+    s_d, y_d = torch.empty_like(a_d), torch.empty_like(a_d)
+    assert lib.fbk_test_fp8_group_scale(ctypes.c_void_p(a_d.data_ptr()), ctypes.c_void_p(s_d.data_ptr()),
+                                        ctypes.c_void_p(y_d.data_ptr()), len(A)) == 0
+    s, y = s_d.cpu().numpy(), y_d.cpu().numpy()
+    want_s = (A / np.float32(448)).astype(np.float32)        # IEEE fp32 division on the host
+    np.testing.assert_array_equal(s.view(np.uint32), want_s.view(np.uint32))
+    big = A >= np.float32(2.0 ** -80)
+    want_y = (np.float32(1) / want_s[big]).astype(np.float32)
+    np.testing.assert_array_equal(y[big].view(np.uint32), want_y.view(np.uint32))
+    assert np.all(y[~big] == np.float32(1))
