@@ -114,7 +114,10 @@ __global__ void __launch_bounds__(FR_WARPS * 32) facache_rows_kernel(Geometry g,
   for (int idx = tid; idx < blk * (D / 2); idx += NTHREADS) {
     const int t = idx / (D / 2), i = idx % (D / 2);
     __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(Ks + t * RS);
-    const float2 cs = rope_cs_fast(c0 + t, g.inv_freq_over_pi[i]);
+    // the position in 64 bits (c0 may be any int32), the angle in turns reduced in fp64
+    const double turns = (double)((long long)c0 + t) * g.inv_freq_over_pi[i];
+    float2 cs;
+    __sincosf((float)((turns - 2.0 * rint(0.5 * turns)) * CUDART_PI), &cs.y, &cs.x);
     const float x1 = __bfloat162float(row[i]), x2 = __bfloat162float(row[i + D / 2]);
     row[i] = __float2bfloat16_rn(x1 * cs.x - x2 * cs.y);
     row[i + D / 2] = __float2bfloat16_rn(x2 * cs.x + x1 * cs.y);

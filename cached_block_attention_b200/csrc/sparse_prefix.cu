@@ -183,7 +183,9 @@ __global__ void __launch_bounds__(SCORE_THREADS) page_scores_kernel(Geometry g, 
 // largest of its kv-heads' scores; the k best pages are kept, ties to the
 // lower page index. The k-th largest score is found by a radix select over the
 // scores' order-preserving 32-bit keys (four 8-bit digits, most significant
-// first, one shared-memory histogram each); the pages above it are kept, and
+// first, one shared-memory histogram each, the lanes of a warp that share a
+// bin adding once: scores cluster, so their top digits do); the pages above
+// it are kept, and
 // of the pages equal to it the lowest-indexed ones that complete the k. The
 // kept pages' physical ids go to kept_table in increasing logical order (their
 // positions from a block-wide scan of the keep flags, each thread owning a run
@@ -248,9 +250,13 @@ __global__ void __launch_bounds__(SEL_THREADS) select_pages_kernel(Geometry g, c
   for (int shift = 24; shift >= 0 && !keep_all; shift -= 8) {
     for (int i = tid; i < 256; i += SEL_THREADS) hist[i] = 0;
     __syncthreads();  // keys written (first pass), histogram cleared
-    for (int p = tid; p < n_pages; p += SEL_THREADS) {
-      const unsigned key = sel_key[p];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    for (int p0 = warp * 32; p0 < n_pages; p0 += SEL_THREADS) {  // whole warps: the lanes of a bin add once
+      const int p = p0 + lane;
+      const unsigned key = p < n_pages ? sel_key[p] : 0u;
+      const bool in = p < n_pages && (key & mask) == prefix;
+      const int bin = in ? (int)((key >> shift) & 255u) : -1;
+      const unsigned same = __match_any_sync(0xffffffffu, bin);
+      if (in && lane == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
     }
     __syncthreads();
     if (warp == 0) {  // lane l holds digits 255 - 8l down to 248 - 8l

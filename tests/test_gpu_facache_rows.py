@@ -133,3 +133,20 @@ def test_llada8b_shape_with_synthetic_state():
     (ou, lu), _ = fc.facache_step(state, f(qu), f(ku), f(vu), f(qc), f(kc), f(vc), c0, hkv, 1.0, 1e4)
     H.assert_close(got, ou, "bf16", "llada8b shape")
     assert np.abs(got_lse - lu).max() <= 2e-2
+
+
+def test_block_position_near_int32_max():
+    """block_pos c0 = 2^31 - 6: the block's keys sit at c0 + t, past 2^31 for
+    t >= 6. Positions are formed in 64 bits, so the rows still match the
+    oracle, which rotates at the exact positions."""
+    from cached_block_attention_b200 import fbk
+    b, hq, hkv, d, blk, n = 1, 4, 2, 128, 32, 132
+    c0 = 2 ** 31 - 6
+    qu, ku, vu, qc, kc, vc = make_rows_case(b, hq, hkv, d, blk, n, (c0,), 1e4, seed=88)
+    f = orc.bits_to_f64
+    state = fc.uu_state(f(qu), f(ku), f(vu), hkv, 1.0)
+    shape = fbk.Shape(b, hq, hkv, d, blk, 1.0, 1e4)
+    got, got_lse = run_rows(shape, qu, state, kc, vc, [c0])
+    (ou, lu), _ = fc.facache_step(state, f(qu), f(ku), f(vu), f(qc), f(kc), f(vc), c0, hkv, 1.0, 1e4)
+    H.assert_close(got, ou, "bf16", "block at 2^31 - 6")
+    assert np.abs(got_lse - lu).max() <= 2e-2
