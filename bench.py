@@ -45,10 +45,11 @@ def parse():
     ap.add_argument("--keep", type=float, default=0.125,
                     help="--op sparse_prefix: fraction of each sequence's prefix pages kept (top-k)")
     ap.add_argument("--op", default="attention",
-                    choices=["attention", "fp8_group_quant", "facache_rows", "sparse_prefix"],
+                    choices=["attention", "fp8_group_quant", "facache_rows", "facache_step", "sparse_prefix"],
                     help="attention: the cached block attention block (default); fp8_group_quant: the "
                          "per-group FP8 activation quantisation on the FP8_WORKLOADS shapes; facache_rows: "
-                         "the FACache step of a whole sequence's unchanged rows (FACACHE_WORKLOADS)")
+                         "the FACache step of a whole sequence's unchanged rows (FACACHE_WORKLOADS); "
+                         "facache_step: the whole FACache step, unchanged rows and block rows")
     ap.add_argument("--layers", type=int, default=1,
                     help="attention layers per block; > 1 runs the whole block through fbk_decode_block")
     ap.add_argument("--adaptive", default="",
@@ -1217,6 +1218,213 @@ def run_facache(args, name, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+FACACHE_STEP_METRIC = "FACache over a whole sequence: denoising steps/s (1×B200)"
+
+
+def facache_step_inputs(name):
+    """Seeded inputs (host) of a whole FACache step: U's queries, U's keys (after
+    RoPE) and values in cache layout [b, Hkv, U, d], the block's Q/K/V (bf16 bits)."""
+    from cached_block_attention_b200 import synth
+    b, hq, hkv, d, blk, rows, c0, seed = FACACHE_WORKLOADS[name]
+    q, _, kb, vb = facache_inputs(name)
+    r = np.random.Generator(np.random.PCG64(seed + 1))
+    sc = np.float32(1.0 / np.sqrt(d))
+    ku = synth.bf16_bits(r.standard_normal((b, hkv, rows, d), dtype=np.float32) * sc)
+    vu = synth.bf16_bits(r.standard_normal((b, hkv, rows, d), dtype=np.float32) * sc)
+    qc = synth.bf16_bits(r.standard_normal((b, blk, hq, d), dtype=np.float32) * sc)
+    return q, ku, vu, qc, kb, vb
+
+
+def facache_step_bytes(b, hq, hkv, d, blk, rows):
+    """Algorithmic bytes of one whole step: the unchanged rows (facache_bytes),
+    U's K and V read once per kv-head for the block's rows, the block's queries
+    and outputs (bf16) and the block rows' state written and read back (fp32)."""
+    return (facache_bytes(b, hq, hkv, d, blk, rows) + 2 * b * hkv * rows * d * 2 + 2 * b * blk * hq * d * 2
+            + 2 * b * hq * blk * (d + 2) * 4)
+
+
+def oracle_facache_step_sample(name, n_rows=256, budget_s=10.0):
+    """The oracle's whole step (the block's rows attend to all of U's keys) with
+    n_rows and with 1 of the unchanged rows, repeated for about budget_s seconds;
+    the unchanged rows' time is scaled from the difference to all of them.
+    Returns (steps/s, runs)."""
+    from oracle import facache as fc
+    from oracle import fbk_oracle as orc
+    b, hq, hkv, d, blk, rows, c0, seed = FACACHE_WORKLOADS[name]
+    q, ku, vu, qc, kb, vb = facache_step_inputs(name)
+    _, (o, m, l), _, _ = facache_inputs(name)
+    f = orc.bits_to_f64
+    ku_s, vu_s = np.transpose(f(ku), (0, 2, 1, 3)), np.transpose(f(vu), (0, 2, 1, 3))  # [b, U, Hkv, d]
+    st = (o[:, :, :n_rows], m[:, :, :n_rows], l[:, :, :n_rows])
+    st1 = (o[:, :, :1], m[:, :, :1], l[:, :, :1])
+    qs, qcf, kbf, vbf = f(q[:, :n_rows]), f(qc), f(kb), f(vb)
+    t_many = t_one = 0.0
+    n = 0
+    t_end = time.perf_counter() + budget_s
+    while n == 0 or time.perf_counter() < t_end:
+        t0 = time.perf_counter()
+        fc.facache_step(st, qs, ku_s, vu_s, qcf, kbf, vbf, c0, hkv, 1.0, 1e4)
+        t1 = time.perf_counter()
+        fc.facache_step(st1, qs[:, :1], ku_s, vu_s, qcf, kbf, vbf, c0, hkv, 1.0, 1e4)
+        t2 = time.perf_counter()
+        t_many += t1 - t0
+        t_one += t2 - t1
+        n += 1
+    # the block's rows and one unchanged row, plus the other unchanged rows at the sample's rate
+    per_row = max(0.0, (t_many - t_one) / (n_rows - 1)) / n
+    per = t_one / n + per_row * (rows - 1)
+    return 1.0 / per, n
+
+
+def run_facache_step(args, name, rank, world, local):
+    """One bench step = one fbk_facache_step (the unchanged rows and the block's
+    rows) on a LLaDA-8B-shaped sequence, one CUDA graph, inputs resident in HBM,
+    L2 flushed before it. The U x U state comes from fbk_facache_refresh (once per
+    block), timed separately as refresh_us."""
+    import torch
+    from cached_block_attention_b200 import fbk
+    dev = torch.device("cuda", local)
+    b, hq, hkv, d, blk, rows, c0, seed = FACACHE_WORKLOADS[name]
+    q, ku, vu, qc, kb, vb = facache_step_inputs(name)
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    cache = fbk.KVCache(to(ku), to(vu), torch.full((b,), rows, dtype=torch.int32, device=dev), None,
+                        torch.zeros(1, dtype=torch.int32, device=dev))
+    d_q, d_qc, d_kb, d_vb = to(q), to(qc), to(kb), to(vb)
+    h_qc, h_kb, h_vb = (torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+                        for a in (qc, kb, vb))
+    state = fbk.Partial(torch.empty(b, hq, rows, d, device=dev), torch.empty(b, hq, rows, device=dev),
+                        torch.empty(b, hq, rows, device=dev))
+    pos = torch.full((b,), c0, dtype=torch.int32, device=dev)
+    out_u = torch.empty(b, rows, hq, d, dtype=torch.bfloat16, device=dev)
+    out_c = torch.empty(b, blk, hq, d, dtype=torch.bfloat16, device=dev)
+    h_ou = torch.empty(out_u.shape, dtype=torch.bfloat16).pin_memory()
+    h_oc = torch.empty(out_c.shape, dtype=torch.bfloat16).pin_memory()
+    shape = fbk.Shape(b, hq, hkv, d, blk, 1.0, 1e4)
+    ws = torch.empty(fbk.facache_workspace_bytes(shape, rows, 0), dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    nbytes = facache_step_bytes(b, hq, hkv, d, blk, rows)
+
+    def refresh():
+        fbk.facache_refresh(shape, d_q, [c0] * b, cache, state, ws)
+
+    def step():
+        fbk.facache_step(shape, d_q, state, d_qc, d_kb, d_vb, pos, cache, out_u, out_c, ws)
+
+    for _ in range(2):
+        refresh()
+        step()
+    torch.cuda.synchronize()
+    assert int(cache.error_flags.item()) == 0, "device error flags"
+    st = torch.cuda.Stream(dev)
+    st.wait_stream(torch.cuda.current_stream(dev))
+    graphs = []
+    with torch.cuda.stream(st):
+        for fn in (step, refresh):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st, capture_error_mode="thread_local"):
+                fn()
+            graphs.append(g)
+    torch.cuda.synchronize()
+    g_step, g_refresh = graphs
+
+    def timed(g, n):
+        evs = []
+        with torch.cuda.stream(st):
+            for _ in range(n):
+                flush.zero_()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e[0].record(st)
+                g.replay()
+                e[1].record(st)
+                evs.append(e)
+        return evs
+
+    timed(g_step, max(3, args.warmup))
+    barrier(world)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    evs = timed(g_step, args.steps)
+    barrier(world)
+    clock_info = clocks.stop()
+    t = [e[0].elapsed_time(e[1]) for e in evs]
+    total_ms = max_over_ranks(sum(t), world)
+    step_ms = sum(t) / len(t)
+    rev = timed(g_refresh, max(3, args.steps // 2))
+    torch.cuda.synchronize()
+    refresh_ms = statistics.mean(a.elapsed_time(c) for a, c in rev)
+
+    # end to end: the block's Q/K/V H2D, the step through the API, both outputs D2H
+    def e2e(n):
+        with torch.cuda.stream(st):
+            for _ in range(n):
+                d_qc.copy_(h_qc, non_blocking=True)
+                d_kb.copy_(h_kb, non_blocking=True)
+                d_vb.copy_(h_vb, non_blocking=True)
+                fbk.facache_step(shape, d_q, state, d_qc, d_kb, d_vb, pos, cache, out_u, out_c, ws, stream=st)
+                h_ou.copy_(out_u, non_blocking=True)
+                h_oc.copy_(out_c, non_blocking=True)
+    e2e(1)
+    torch.cuda.synchronize()
+    a, bev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, args.steps // 2)
+    a.record(st)
+    e2e(n_e2e)
+    bev.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(bev) / n_e2e, world)
+
+    hbm_gbs, _, _, peak_kind = load_peaks()
+    achieved = nbytes / (step_ms * 1e-3) / 1e9
+    line = {
+        "metric": FACACHE_STEP_METRIC, "value": world * args.steps / (total_ms * 1e-3), "unit": "denoising steps/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": name, "batch": b, "q_heads": hq, "kv_heads": hkv, "head_dim": d, "block": blk,
+                   "unchanged_rows": rows, "block_pos": c0,
+                   "description": "LLaDA-8B-shaped layer, 4096-token prompt + 32-token block + 1024-token "
+                                  "masked suffix; the U x U state from fbk_facache_refresh",
+                   "bench_step": "one fbk_facache_step (unchanged rows + the block's rows over all keys), "
+                                 "one CUDA graph",
+                   "l2": "flushed (2x L2 memset) before every timed step, outside the events",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "refresh_us": refresh_ms * 1e3,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                     "frac": achieved / hbm_gbs, "peak_kind": f"{peak_kind} hbm_gbs", "traffic": None,
+                     "traffic_key": None, "kernel": "fbk_facache_step (all launches)",
+                     "algorithmic_bytes_per_launch": nbytes, "launch_us": step_ms * 1e3},
+        "e2e": {"value": world / (e2e_ms * 1e-3), "unit": "denoising steps/s",
+                "h2d_bytes_per_step": (h_qc.numel() + h_kb.numel() + h_vb.numel()) * 2,
+                "d2h_bytes_per_step": (h_ou.numel() + h_oc.numel()) * 2,
+                "note": "the block's Q/K/V H2D, the API call, both outputs D2H, one stream"},
+        "gpu_launches": None,
+        "clocks": clock_info,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n = oracle_facache_step_sample(name)
+        line["cpu_baseline"] = {"value": v, "unit": "denoising steps/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{n} runs of the step with 256 of the {rows} unchanged rows (their "
+                                          f"time scaled to all rows) and the block's rows over all keys, numpy"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_facache_step_reference(args, name, rank):
+    if rank != 0:
+        return
+    v, n = oracle_facache_step_sample(name, budget_s=max(1.0, 0.5 * args.steps))
+    line = {"impl": "reference", "metric": FACACHE_STEP_METRIC, "value": v, "unit": "denoising steps/s",
+            "n_gpus": args.gpus, "steps": n, "warmup": args.warmup, "ms_per_step": 1e3 / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name},
+            "cpu_baseline": {"value": v, "unit": "denoising steps/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{n} runs of the step with 256 unchanged rows (scaled) and the block's "
+                                       "rows, numpy"},
+            "e2e": {"value": v, "unit": "denoising steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ sparse prefix + cached residual
 
 SPARSE_METRIC = "sparse block-external attention with a cached residual: denoising steps/s (1×B200)"
@@ -1375,6 +1583,19 @@ def main():
         rank, world, local = dist_setup(args.gpus)
         try:
             run_facache(args, name, rank, world, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
+    if args.op == "facache_step":
+        name = args.workload if args.workload in FACACHE_WORKLOADS else "llada8b_seq"
+        if args.impl == "reference":
+            run_facache_step_reference(args, name, int(os.environ.get("RANK", "0")))
+            return
+        rank, world, local = dist_setup(args.gpus)
+        try:
+            run_facache_step(args, name, rank, world, local)
         finally:
             if world > 1:
                 import torch.distributed as dist
