@@ -1398,7 +1398,7 @@ def run_facache_step(args, name, rank, world, local):
                 "h2d_bytes_per_step": (h_qc.numel() + h_kb.numel() + h_vb.numel()) * 2,
                 "d2h_bytes_per_step": (h_ou.numel() + h_oc.numel()) * 2,
                 "note": "the block's Q/K/V H2D, the API call, both outputs D2H, one stream"},
-        "gpu_launches": None,
+        "gpu_launches": 5 * args.steps,  # unchanged rows (1), the block rows' prefix (3), the step kernel (1)
         "clocks": clock_info,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -1556,7 +1556,9 @@ def run_sparse(args, wl, rank, world, local):
                      "algorithmic_bytes_per_launch": sparse_bytes, "launch_us": part["sparse"] * 1e3},
         "select_us": part["select"] * 1e3, "dense_prefix_us": part["dense"] * 1e3,
         "sparse_prefix_us": part["sparse"] * 1e3,
-        "gpu_launches": None,
+        # per block: means (1), selection (rotation, scores, top-k: 3), dense and sparse prefix (3 + 3),
+        # residual capture (1) and step (1) at step 0; then sparse prefix (3), residual apply (1), step (1)
+        "gpu_launches": (12 + 5 * (S - 1)) * args.steps,
         "clocks": clock_info,
     }
     if rank == 0:
