@@ -583,7 +583,9 @@ def run_ours(args, wl, rank, world, local):
                            "kv_bytes": kv_bytes, "flops": pfx_flops},
         "step_us": step_launch_ms * 1e3, "commit_us": commit_ms * 1e3,
         "recompute_schedule": {"value": world * S / (rec_ms * 1e-3), "unit": "denoising steps/s",
-                               "ms_per_block": rec_ms},
+                               "ms_per_block": rec_ms,
+                               # reuse over recompute, both from the per-block device times
+                               "reuse_speedup": rec_ms / (sum(t_blocks) / len(t_blocks))},
         "e2e": {"value": aggregate_steps_per_s(world, 1, S, e2e_ms), "unit": "denoising steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "eager API calls per block; each block's inputs H2D from pinned host and its outputs "
