@@ -14,9 +14,10 @@
 //    residual is turned into a state (O, lse, 1) that the step kernel merges
 //    with the fresh in-block attention.
 //
-// All of it is small next to the prefix itself: the mean keys read the cache
-// once per committed block, the scores read the means and the block's queries,
-// and the residual kernels touch one state.
+// The mean keys read every K byte of the prefix once (a committed block only
+// changes its own pages, so a decoder needs them once per page); the scores
+// read the means and the block's queries; the residual kernels touch one
+// state.
 #include "launch.h"
 #include "sparse_prefix.h"
 
