@@ -455,7 +455,15 @@ fbk_status fbk_facache_step(const fbk_shape *shape, int32_t n_rows, const void *
  * fbk_residual_capture: r_o fp32 [b, Hq, B, d] and r_lse fp32 [b, Hq, B] from
  *   the dense and the sparse state of the same queries (r_lse = -inf marks a
  *   row with no prefix).
- * fbk_residual_apply: ext = ((O~/l)_sparse + r_o, lse_sparse + r_lse, 1). */
+ * fbk_residual_apply: ext = ((O~/l)_sparse + r_o, lse_sparse + r_lse, 1).
+ * Errors, before any launch: FBK_ERR_INVALID_ARG for a missing pointer or
+ * k < 1; FBK_ERR_UNSUPPORTED for a contiguous cache, misaligned means or
+ * max_pages_per_seq above 25,600 (the selection holds a sequence's scores in
+ * shared memory); FBK_ERR_WORKSPACE for a missing or short workspace; the
+ * shape and cache codes of fbk_prefix_partial otherwise (the residual calls
+ * accept B up to 256, with G*B <= 256). On the device, a page id outside
+ * [0, num_pages) raises FBK_DEVERR_PAGE_ID and that page is skipped, and a bad
+ * prefix length FBK_DEVERR_PREFIX_LEN (the sequence then counts as empty). */
 fbk_status fbk_page_means(const fbk_shape *shape, const fbk_kv_cache *cache, float *means, void *cuda_stream);
 size_t fbk_select_pages_workspace_bytes(const fbk_shape *shape, const fbk_kv_cache *cache);
 fbk_status fbk_select_pages(const fbk_shape *shape, const void *q_blk, const fbk_kv_cache *cache, const float *means,
