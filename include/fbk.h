@@ -423,7 +423,14 @@ fbk_status fbk_facache_unchanged_rows(const fbk_shape *shape, int32_t n_rows, co
  *  out_blk: bf16 [b, B, Hq, d]; lse_blk fp32 [b, Hq, B] or NULL.
  *  Launches: fbk_facache_unchanged_rows's kernel for U's rows; for the block's
  *  rows, the prefix computation over U's keys with the rows rotated at c0 + t,
- *  then fbk_block_attn_merge's kernel. */
+ *  then fbk_block_attn_merge's kernel.
+ * Errors, before any launch: the shape and cache codes of fbk_prefix_partial
+ * (u_cache must be contiguous, else FBK_ERR_UNSUPPORTED); FBK_ERR_INVALID_ARG
+ * for n_rows < 0, num_splits < 0, a missing pointer or (refresh) a host c0
+ * outside [0, n_rows]; FBK_ERR_CAPACITY when (step) b * n_rows * Hq reaches
+ * 2^31 or (refresh) the cache's capacity is below n_rows;
+ * FBK_ERR_UNSUPPORTED for misaligned pointers (16 bytes) or a workspace not
+ * 256-byte aligned; FBK_ERR_WORKSPACE for a missing or short workspace. */
 size_t fbk_facache_workspace_bytes(const fbk_shape *shape, int32_t n_rows, int32_t num_splits);
 fbk_status fbk_facache_refresh(const fbk_shape *shape, int32_t n_rows, const void *q_u_raw,
                                const int32_t *block_pos_host, const fbk_kv_cache *u_cache,
