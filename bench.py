@@ -1435,6 +1435,54 @@ def run_facache_step_reference(args, name, rank):
 SPARSE_METRIC = "sparse block-external attention with a cached residual: denoising steps/s (1×B200)"
 
 
+def oracle_sparse_block(case, steps, keep, page):
+    """The oracle's sparse schedule for one block (FlashBlock, Abstract; the
+    reading of oracle/sparse_residual.py): page scores and the top-k pages from
+    step 0's queries, the dense and the sparse state and their residual at step
+    0 (whose output is exact), then `steps` - 1 steps of sparse attention plus
+    the residual: fp64 numpy on the host cores."""
+    from oracle import fbk_oracle as orc
+    from oracle import sparse_residual as sr
+    kp, vp, lens, hkv, base = case["kp"], case["vp"], case["lens"], case["hkv"], case["base"]
+    pages = (np.asarray(lens) + page - 1) // page
+    k = max(1, int(round(keep * float(pages.mean()))))
+    q0, k0, v0 = case["steps"][0]
+    sel = sr.select_pages(sr.page_scores(q0, kp, lens, hkv, 1.0, base, page), k)
+    dense = orc.prefix_partial(q0, kp, vp, lens, hkv, 1.0, base)
+    res = sr.residual(dense, sr.sparse_prefix_partial(q0, kp, vp, lens, sel, page, hkv, 1.0, base))
+    orc.step_output(dense, q0, k0, v0, lens, hkv, 1.0, base)
+    for s_ in range(1, steps):
+        q, kb, vb = case["steps"][s_ % len(case["steps"])]
+        sr.approx_step_output(q, kb, vb, kp, vp, lens, sel, page, res, hkv, 1.0, base)
+
+
+def run_sparse_reference(args, wl, rank):
+    """The reference arm of --op sparse_prefix: the oracle's sparse schedule on
+    a bounded sample, one block with at most 4 denoising steps per bench step."""
+    if rank != 0:
+        return
+    case = oracle_case(wl)
+    page = wl.page_size or 64
+    s = min(wl.steps, 4)
+    for _ in range(args.warmup):
+        oracle_sparse_block(case, s, args.keep, page)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sparse_block(case, s, args.keep, page)
+    dt = time.perf_counter() - t0
+    v = args.steps * s / dt
+    sample = f"one block with {s} of {wl.steps} steps per bench step (keep {args.keep}, {page}-token pages)"
+    line = {"impl": "reference", "metric": SPARSE_METRIC, "value": v, "unit": "denoising steps/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "keep": args.keep, "page_size": page},
+            "cpu_baseline": {"value": v, "unit": "denoising steps/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "denoising steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def run_sparse(args, wl, rank, world, local):
     """One bench step = one block of the sparse schedule (FlashBlock, Abstract:
     sparse attention with complementary residual reuse; the reading of
@@ -1566,6 +1614,14 @@ def run_sparse(args, wl, rank, world, local):
         "gpu_launches": (12 + 5 * (S - 1)) * args.steps,
         "clocks": clock_info,
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        case = oracle_case(wl)
+        s_o = min(S, 4)
+        t0 = time.perf_counter()
+        oracle_sparse_block(case, s_o, args.keep, wl.page_size)
+        v_o = s_o / (time.perf_counter() - t0)
+        line["cpu_baseline"] = {"value": v_o, "unit": "denoising steps/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"one block with {s_o} of {S} steps (keep {args.keep}), fp64 numpy"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     graphs.clear()
@@ -1624,8 +1680,7 @@ def main():
     wl = synth.WORKLOADS[args.workload]
     if args.op == "sparse_prefix":
         if args.impl == "reference":
-            print(json.dumps({"impl": "reference", "unavailable": "the sparse schedule has no timed oracle arm; "
-                                                                  "its oracle is exercised by the tests"}))
+            run_sparse_reference(args, wl, int(os.environ.get("RANK", "0")))
             return
         rank, world, local = dist_setup(args.gpus)
         try:

@@ -20,6 +20,7 @@ KEYS = {"impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_
     ["--op", "fp8_group_quant", "--workload", "ffn_in_llada8b"],
     ["--op", "facache_rows"],
     ["--op", "facache_step"],
+    ["--op", "sparse_prefix", "--workload", "tiny"],
 ])
 def test_reference_arm_prints_one_contract_line(extra):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
