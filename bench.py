@@ -322,10 +322,20 @@ def cpu_baseline(wl, budget_s=12.0):
     for _ in range(n):
         oracle_block(case, wl.steps)
     dt = time.perf_counter() - t0
-    return {"value": n * wl.steps / dt, "unit": "denoising steps/s", "cores": blas_threads(),
-            "kind": "oracle",
-            "sample": f"{n} whole blocks of {wl.name} ({wl.steps} steps each, prefix state once, "
-                      f"commit), fp64 numpy"}
+    out = {"value": n * wl.steps / dt, "unit": "denoising steps/s", "cores": blas_threads(),
+           "kind": "oracle",
+           "sample": f"{n} whole blocks of {wl.name} ({wl.steps} steps each, prefix state once, "
+                     f"commit), fp64 numpy"}
+    try:  # the same block on one host thread
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            oracle_block(case, wl.steps)
+            t1 = time.perf_counter() - t0
+        out["single_thread"] = {"value": wl.steps / t1, "cores": 1, "sample": f"one whole block of {wl.name}"}
+    except ImportError:
+        pass
+    return out
 
 
 def run_reference(args, wl, rank, world):
