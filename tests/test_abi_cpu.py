@@ -342,3 +342,42 @@ def test_facache_refresh_and_step_argument_checks(fbk):
     assert st(ctypes.byref(_shape(fbk, mode=1)), 100, *args, ptr(0x100000), n, 4, None) == -2
     assert st(ctypes.byref(s), 100, *args, ptr(0x100000), n - 1, 4, None) == -4
     assert st(ctypes.byref(s), 100, *args, ptr(0x100010), n, 4, None) == -2
+
+
+def test_sparse_argument_checks(fbk):
+    """Host checks of the sparse-prefix calls; none reach a CUDA call."""
+    s = _shape(fbk)
+    ptr = ctypes.c_void_p
+    c = _cache(fbk)
+    paged = _cache(fbk, paged=1, page_size=64, max_pages_per_seq=4, num_pages=8, page_table=0x1000)
+    huge = _cache(fbk, paged=1, page_size=64, max_pages_per_seq=25601, num_pages=8, page_table=0x1000)
+    means = ctypes.cast(ctypes.c_void_p(0x200000), ctypes.POINTER(ctypes.c_float))
+    odd_means = ctypes.cast(ctypes.c_void_p(0x200004), ctypes.POINTER(ctypes.c_float))
+    kept = ctypes.cast(ctypes.c_void_p(0x210000), ctypes.POINTER(ctypes.c_int32))
+    lens = ctypes.cast(ctypes.c_void_p(0x220000), ctypes.POINTER(ctypes.c_int32))
+    pm = fbk.lib.fbk_page_means
+    assert pm(ctypes.byref(s), ctypes.byref(c), means, None) == -2            # contiguous cache
+    assert pm(ctypes.byref(s), ctypes.byref(paged), None, None) == -1
+    assert fbk.lib.fbk_select_pages_workspace_bytes(ctypes.byref(s), ctypes.byref(c)) == 0
+    n = fbk.lib.fbk_select_pages_workspace_bytes(ctypes.byref(s), ctypes.byref(paged))
+    # rotated queries fp32 [b, B, Hq, d] and the scores fp32 [b, Hkv, max_pages], each 256-byte aligned
+    assert n == 1 * 32 * 4 * 128 * 4 + 256
+    sp = fbk.lib.fbk_select_pages
+    q, ws = ptr(0x70000), ptr(0x300000)
+    assert sp(ctypes.byref(s), q, ctypes.byref(c), means, 2, kept, lens, ws, n, None) == -2
+    assert sp(ctypes.byref(s), q, ctypes.byref(paged), means, 0, kept, lens, ws, n, None) == -1
+    assert sp(ctypes.byref(s), q, ctypes.byref(paged), None, 2, kept, lens, ws, n, None) == -1
+    assert sp(ctypes.byref(s), q, ctypes.byref(paged), odd_means, 2, kept, lens, ws, n, None) == -2
+    assert sp(ctypes.byref(s), q, ctypes.byref(huge), means, 2, kept, lens, ws, 1 << 30, None) == -2
+    assert sp(ctypes.byref(s), q, ctypes.byref(paged), means, 2, kept, lens, ws, n - 1, None) == -4
+    assert sp(ctypes.byref(s), q, ctypes.byref(paged), means, 2, kept, lens, ptr(0x300010), n, None) == -2
+    p = fbk.CPartial(0x40000, 0x50000, 0x60000)
+    bad = fbk.CPartial(0x40000, None, 0x60000)
+    ro = ctypes.cast(ctypes.c_void_p(0x230000), ctypes.POINTER(ctypes.c_float))
+    rl = ctypes.cast(ctypes.c_void_p(0x240000), ctypes.POINTER(ctypes.c_float))
+    rc, ra = fbk.lib.fbk_residual_capture, fbk.lib.fbk_residual_apply
+    assert rc(ctypes.byref(s), ctypes.byref(p), ctypes.byref(bad), ro, rl, None) == -1
+    assert rc(ctypes.byref(s), ctypes.byref(p), ctypes.byref(p), None, rl, None) == -1
+    assert ra(ctypes.byref(s), ctypes.byref(bad), ro, rl, ctypes.byref(p), None) == -1
+    big = _shape(fbk, n_q_heads=4, n_kv_heads=2, block_len=129)            # G*B = 258
+    assert rc(ctypes.byref(big), ctypes.byref(p), ctypes.byref(p), ro, rl, None) == -2
